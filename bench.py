@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Benchmark of the POET-X layer step on B200: tokens/s and TFLOP/s against the bf16 roofline.
+
+A step is one pass of the whole hot path over one batch of synthetic tokens: CNP forward of
+both sides, layer forward, layer backward (including the CNP adjoint that writes the packed
+gradients).  Default workload: the Llama-8B attention projection (4096 x 4096, b = 256, k = 3,
+2048 tokens, bf16, fast mode), the single-layer configuration the POET-X pages time (SAI
+replication review, "Reproducibility & code", first item).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl poetx|reference] [--workload NAME]
+
+Multi-GPU (torchrun, one process per GPU): each rank runs an independent replica of the layer on
+its own tokens (data parallel, weak scaling); no collective is on the timed path.  Timing: CUDA
+events around each step on the launching stream, an L2 flush (256 MiB write) between steps
+outside the timed intervals, barrier + synchronize around the timed region, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import poetx_inputs as I  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama8b_attn_4096_b256_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+METRIC = "POET-X linear fwd+bwd tokens/s & TFLOP/s (4096², b=256) vs bf16 roofline"
+
+
+# ------------------------------------------------------------------------------ work model
+def step_flops(s: I.LayerShape) -> dict:
+    """Algorithmic FLOPs of one step (what the method must compute; W0 is frozen, no dW0).
+
+    fwd = 2N d_in d_out + 2N b (d_in + d_out); bwd = 2N d_in d_out + 4N b (d_in + d_out)
+    (+ 2N d_in d_out + 2N b d_in recomputed in mem mode); CNP fwd = nb k b^3 (each power of a
+    skew block is symmetric or skew, so half of each product is needed); CNP adjoint = nb 2k 2b^3."""
+    N, di, do, b, k = s.n_tokens, s.d_in, s.d_out, s.b, s.k
+    nb = s.nb_in + s.nb_out
+    fwd = 2 * N * di * do + 2 * N * b * (di + do)
+    bwd = 2 * N * di * do + 4 * N * b * (di + do)
+    if s.mode == "mem":
+        bwd += 2 * N * di * do + 2 * N * b * di
+    cnp = nb * k * b ** 3 + nb * 2 * k * 2 * b ** 3
+    return {"fwd": fwd, "bwd": bwd, "cnp": cnp, "total": fwd + bwd + cnp}
+
+
+def w_gemm_flops(s: I.LayerShape) -> int:
+    """FLOPs of one launch of the dominant kernel, the W0' GEMM (Z = V W0'^T or dV = dZ W0')."""
+    return 2 * s.n_tokens * s.d_in * s.d_out
+
+
+def read_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+# --------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    QUERY = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, period_ms: int = 100):
+        self.period_ms = period_ms
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="poetx_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", f"-lms", str(self.period_ms),
+                 "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self, uuid: str) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9 or (uuid and not parts[0].lower().endswith(uuid.lower())):
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+def gpu_uuid(dev) -> str:
+    import torch
+    try:
+        return str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    except Exception:
+        return ""
+
+
+# ---------------------------------------------------------------------------- distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own tokens (the layer state is shared by construction)."""
+    return base_seed + 7919 * rank
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_step(inp: I.LayerInputs, n_tok: int):
+    """The float64 oracle's layer step on the first n_tok tokens (CNP, forward, backward + CNP adjoint)."""
+    import oracle as O
+    s = inp.shape
+    X, dY = inp.X[:n_tok], inp.dY[:n_tok]
+    W0p = O.absorb(inp.W0, inp.pi_L, inp.pi_R)
+    Q_R, Q_P = O.cnp(inp.theta_R, s.b, s.k), O.cnp(inp.theta_P, s.b, s.k)
+    O.forward_chain(X, W0p, Q_R, Q_P, inp.pi_L, inp.pi_R)
+    O.backward_chain(X, dY, W0p, inp.theta_R, inp.theta_P, inp.pi_L, inp.pi_R, s.b, s.k)
+
+
+def cpu_baseline(inp: I.LayerInputs, budget_s: float = 20.0) -> dict:
+    n = inp.X.shape[0]
+    t0 = time.perf_counter()
+    oracle_step(inp, n)
+    t1 = time.perf_counter()
+    reps, total = 1, t1 - t0
+    while total + (t1 - t0) <= budget_s and reps < 5:
+        t2 = time.perf_counter()
+        oracle_step(inp, n)
+        total += time.perf_counter() - t2
+        reps += 1
+    return {"value": reps * n / total, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{reps} full oracle step(s) of the workload ({n} tokens each, float64 numpy), "
+                      f"{total:.1f} s"}
+
+
+# ------------------------------------------------------------------------------ main arm
+def run_poetx(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    import orthogonal_equivalence_cnp_b200 as P
+    from orthogonal_equivalence_cnp_b200.layer import PoetxLayer, make_desc
+
+    s = I.WORKLOADS[args.workload]
+    seed = I.WORKLOAD_SEEDS[args.workload]
+    state = I.make_layer(s, seed, with_activations=False)
+    acts = I.make_layer(s, shard_seed(seed, rank))
+    layer = PoetxLayer(make_desc(s.d_in, s.d_out, s.b, s.k, s.dtype, s.mode), s.n_tokens, device=dev)
+    layer.load_state(state.W0, state.theta_R, state.theta_P, state.pi_L, state.pi_R)
+    X, dY = layer.to_dev(acts.X), layer.to_dev(acts.dY)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        layer.step(X, dY)
+    torch.cuda.synchronize()
+    st, det = P.poetx_device_status()
+    if st != 0:
+        raise RuntimeError(f"device-side timeout during warm-up ({det:#x})")
+
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler()
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = P.poetx_launch_count()
+    for i in range(K):
+        flush.zero_()
+        ev0[i].record(stream)
+        layer.step(X, dY)
+        ev1[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = P.poetx_launch_count() - launches0
+    clk = clocks.stop(gpu_uuid(dev))
+    times = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
+    t_ms = max_over_ranks(sum(times), world, dev)
+    st, det = P.poetx_device_status()
+    if st != 0:
+        raise RuntimeError(f"device-side timeout in the timed region ({det:#x})")
+
+    # Live per-kernel durations: the same K steps again with the library's event pairs around
+    # every launch (separate pass, so the headline timing carries no bookkeeping).
+    P.poetx_profile_enable(True)
+    for i in range(K):
+        flush.zero_()
+        layer.step(X, dY)
+    torch.cuda.synchronize()
+    prof = P.poetx_profile_summary()
+    P.poetx_profile_enable(False)
+
+    # End to end through the public API with host buffers: H2D of X and dY from pinned memory,
+    # the step, D2H of dX and the packed gradients, all inside the timed interval.
+    hX = torch.from_numpy(acts.X).to(layer.dtype).pin_memory()
+    hdY = torch.from_numpy(acts.dY).to(layer.dtype).pin_memory()
+    h_dX = torch.empty(layer.dX.shape, dtype=layer.dtype).pin_memory()
+    h_gR = torch.empty(layer.g_R.shape, dtype=torch.float32).pin_memory()
+    h_gP = torch.empty(layer.g_P.shape, dtype=torch.float32).pin_memory()
+    Xe, dYe = torch.empty_like(X), torch.empty_like(dY)
+    Ke = K
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(Ke):
+        flush.zero_()
+        e0[i].record(stream)
+        Xe.copy_(hX, non_blocking=True)
+        dYe.copy_(hdY, non_blocking=True)
+        layer.step(Xe, dYe)
+        h_dX.copy_(layer.dX, non_blocking=True)
+        h_gR.copy_(layer.g_R, non_blocking=True)
+        h_gP.copy_(layer.g_P, non_blocking=True)
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    te_ms = max_over_ranks(sum(e0[i].elapsed_time(e1[i]) for i in range(Ke)), world, dev)
+    h2d = hX.numel() * hX.element_size() + hdY.numel() * hdY.element_size()
+    d2h = (h_dX.numel() * h_dX.element_size() + h_gR.numel() * 4 + h_gP.numel() * 4)
+
+    fl = step_flops(s)
+    value = world * s.n_tokens * K / (t_ms / 1e3)
+    tflops = world * fl["total"] * K / (t_ms / 1e3) / 1e12
+    peaks = read_peaks()
+    wcnt, wms = prof["w_gemm"]
+    w_avg_ms = wms / max(wcnt, 1)
+    achieved = w_gemm_flops(s) / (w_avg_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    total_prof_ms = sum(v[1] for v in prof.values())
+    out = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "tflops": round(tflops, 2),
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": s.dtype,
+        "data": "synthetic (seeded numpy draws, see poetx_inputs.py)",
+        "config": {"workload": args.workload, "d_in": s.d_in, "d_out": s.d_out, "b": s.b, "k": s.k,
+                   "n_tokens_per_gpu": s.n_tokens, "mode": s.mode,
+                   "step": "CNP fwd (R,P) + forward + backward incl. CNP adjoint",
+                   "l2": "flushed between steps (256 MiB write outside the timed intervals)",
+                   "parallelism": f"replicas x{world} (data parallel over tokens, no collective on the path)",
+                   "algorithmic_gflop_per_step": round(fl["total"] / 1e9, 2)},
+        "roofline": {"bound": "tensor", "kernel": "w0_gemm (Z = V W0'^T, dV = dZ W0')",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "frac_of_sustained": round(achieved / float(peaks["bf16_tflops_sustained"]), 4),
+                     "launch_ms": round(w_avg_ms, 4), "launches": wcnt},
+        "step_roofline": {"t_flop_us": round(fl["total"] / (peak * 1e12) * 1e6, 1),
+                          "frac": round((fl["total"] / (peak * 1e12)) / (t_ms / K / 1e3), 4)},
+        "kernel_share": {k: round(v[1] / total_prof_ms, 4) for k, v in prof.items() if v[0]},
+        "kernel_ms_per_step": {k: round(v[1] / K, 4) for k, v in prof.items() if v[0]},
+        "gpu_launches": int(launches),
+        "e2e": {"value": round(world * s.n_tokens * Ke / (te_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(acts)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The float64 oracle on the host cores, on a bounded token sample per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    s = I.WORKLOADS[args.workload]
+    inp = I.make_workload(args.workload)
+    n_full = s.n_tokens
+    # Size the per-step sample so the whole run stays within ~150 s.
+    t0 = time.perf_counter()
+    oracle_step(inp, min(64, n_full))
+    t64 = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n_tok = min(64, n_full)
+    while n_tok * 2 <= n_full and t64 * (n_tok * 2) / 64 <= budget:
+        n_tok *= 2
+    for _ in range(args.warmup):
+        oracle_step(inp, n_tok)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(inp, n_tok)
+        times.append(time.perf_counter() - t0)
+    t = sum(times)
+    value = n_tok * args.steps / t
+    fl = step_flops(s)
+    out = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t / args.steps, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded numpy draws, see poetx_inputs.py)",
+        "config": {"workload": args.workload, "d_in": s.d_in, "d_out": s.d_out, "b": s.b, "k": s.k,
+                   "n_tokens_per_gpu": s.n_tokens, "mode": s.mode,
+                   "algorithmic_gflop_per_step": round(fl["total"] / 1e9, 2)},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"per step: the oracle's full layer step (all CNP blocks) on the first "
+                                   f"{n_tok} of {n_full} tokens"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
+    ap.add_argument("--workload", choices=sorted(I.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_poetx(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * poetx.h — C ABI of the POET-X layer library (libpoetx.so, CUDA, sm_100a).
+ *
+ * The layer computes y = R · W0 · P · x for every token x (tokens are rows), where W0 is a
+ * frozen base weight and R, P are trainable orthogonal transforms.  R and P are
+ * block-diagonal in a randomly permuted basis, and every b×b block is the Cayley–Neumann
+ * parameterisation (CNP) of a skew-symmetric block stored as its packed upper triangle.
+ * Sources, by page and section:
+ *   - agidaily.cc article on POET-X, section on fixing the base weight and training the
+ *     two orthogonal transforms: W_RP = R · W0 · P, fast and mem implementations;
+ *   - SAI replication review of POET-X (sai.science), "Summary": input-centric matrix-free
+ *     chain, compact upper-triangular skew storage, batch-parallel block-diagonal matmul,
+ *     two of the four permutations absorbed into W in advance, fused Cayley–Neumann kernel,
+ *     POET-Xfast / POET-Xmem; "Reproducibility & code": k = 3, n_elements = b(b-1)/2,
+ *     merge_then_reinitialize; "Weaknesses": first-order form I + 2Q of the Cayley map.
+ *
+ * Conventions (readings of the pages where they are silent; one per line in the design notes):
+ *   X [N, d_in], Y [N, d_out], row-major; Y = X · (R · W0 · P)^T.
+ *   P acts on the input side (nb_in = d_in / b blocks), R on the output side (nb_out = d_out / b).
+ *   Permutations gather: (Π a)_i = a_{π(i)}.  R = Π_L^T · BD_R · Π_L, P = Π_R^T · BD_P · Π_R.
+ *   Pre-permuted base weight W0' = Π_L · W0 · Π_R^T, i.e. W0'[i][j] = W0[π_L(i)][π_R(j)].
+ *   So y = Π_L^T · BD_R · W0' · BD_P · Π_R · x, evaluated on the activations.
+ *   Packed skew block: θ[p] = S[i][j] = -S[j][i] for i < j, p = i·b - i(i+1)/2 + (j - i - 1).
+ *   CNP: Q = (I + S)(I + S + S^2 + ... + S^k)  (Neumann truncation of (I+S)(I-S)^-1).
+ *
+ * Memory and execution model (every entry point):
+ *   - All array arguments are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or retains them.  Every pointer must be 16-byte aligned.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Arguments are validated on the host before anything is launched: an invalid call
+ *     returns an error status and launches nothing.
+ *   - Activations, W0' and Q use `desc->dtype` (POETX_F32 or POETX_BF16); packed parameters
+ *     θ and their gradients are always float32.  Dense arrays are row-major and contiguous.
+ *   - Gradients overwrite their outputs (they do not accumulate).
+ *   - `workspace` is caller-owned device scratch of at least poetx_workspace_size() bytes;
+ *     its contents need not be preserved between calls.  Calls that share a workspace must
+ *     not overlap in time (use one stream, or one workspace per stream).
+ *   - Device-side waits are bounded; a wait that runs out records POETX_ERR_DEVICE_TIMEOUT,
+ *     which poetx_device_status() returns.
+ */
+#ifndef POETX_H_
+#define POETX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* poetx_stream;   /* same type as cudaStream_t */
+
+typedef enum {
+  POETX_OK = 0,
+  POETX_ERR_INVALID_ARG = 1,        /* NULL pointer, negative size, bad enum value      */
+  POETX_ERR_UNSUPPORTED_SHAPE = 2,  /* d % b != 0, b or k outside the supported set     */
+  POETX_ERR_ALIGNMENT = 3,          /* a pointer is not 16-byte aligned                 */
+  POETX_ERR_WORKSPACE = 4,          /* workspace NULL or smaller than required          */
+  POETX_ERR_CUDA = 5,               /* a CUDA runtime call or kernel launch failed      */
+  POETX_ERR_DEVICE_TIMEOUT = 6      /* a bounded device-side wait ran out               */
+} poetx_status;
+
+typedef enum { POETX_F32 = 0, POETX_BF16 = 1 } poetx_dtype;
+
+/* POET-Xfast keeps the W0'-GEMM output Z for the backward pass; POET-Xmem keeps only X and
+ * recomputes Π_R·x, BD_P·(·) and Z in the backward pass (replication review, "Summary":
+ * POET-Xfast and checkpointed POET-Xmem; agidaily.cc article: the mem variant recomputes part
+ * of the activations). */
+typedef enum { POETX_FAST = 0, POETX_MEM = 1 } poetx_mode;
+
+typedef struct {
+  int d_in;          /* input features, multiple of b                                     */
+  int d_out;         /* output features, multiple of b                                    */
+  int b;             /* block size: 32, 64, 128, 256 or 512 (BF16: 64..512)              */
+  int k;             /* Neumann order, 0 <= k <= 8 (the pages use k = 3)                  */
+  poetx_dtype dtype; /* storage type of activations, W0', Q                               */
+  poetx_mode mode;   /* POETX_FAST or POETX_MEM                                           */
+} poetx_desc;
+
+/* Bytes of device workspace that every entry point below needs for this layer and n_tokens
+ * (the maximum over cnp / forward / backward / merge / absorb).  Returns 0 for an invalid
+ * descriptor. */
+size_t poetx_workspace_size(const poetx_desc* desc, int n_tokens);
+
+/* CNP forward for both sides of one layer (replication review, "Summary": fused
+ * Cayley–Neumann series; "Reproducibility & code": k = 3, n_elements = b(b-1)/2).
+ *   theta_R  float32 [d_out/b, b(b-1)/2]   packed skew parameters of R's blocks (in)
+ *   theta_P  float32 [d_in/b,  b(b-1)/2]   packed skew parameters of P's blocks (in)
+ *   Q_R      dtype   [d_out/b, b, b]       Q_i = (I + S_i) Σ_{j<=k} S_i^j, row-major (out)
+ *   Q_P      dtype   [d_in/b,  b, b]       (out)
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, WORKSPACE, CUDA. */
+poetx_status poetx_cnp(const poetx_desc* desc, const float* theta_R, const float* theta_P,
+                       void* Q_R, void* Q_P, void* workspace, size_t ws_bytes, poetx_stream stream);
+
+/* CNP forward over a flat batch of n_blocks blocks that share b and k (e.g. every block of
+ * every layer of a model in one launch).  Uses desc->b, desc->k, desc->dtype only.
+ *   theta float32 [n_blocks, b(b-1)/2] (in); Q dtype [n_blocks, b, b] (out).
+ * Workspace: poetx_cnp_blocks_workspace_size(desc, n_blocks) bytes. */
+size_t poetx_cnp_blocks_workspace_size(const poetx_desc* desc, int n_blocks);
+poetx_status poetx_cnp_blocks(const poetx_desc* desc, int n_blocks, const float* theta, void* Q,
+                              void* workspace, size_t ws_bytes, poetx_stream stream);
+
+/* Absorb two of the four permutations into the base weight in advance (replication review,
+ * "Summary": permutation reduction): W0'[i][j] = W0[perm_L[i]][perm_R[j]].
+ *   W0 dtype [d_out, d_in] (in); perm_L int32 [d_out], perm_R int32 [d_in] bijections (in);
+ *   W0p dtype [d_out, d_in] (out; must not alias W0). */
+poetx_status poetx_absorb(const poetx_desc* desc, const void* W0, const int32_t* perm_L,
+                          const int32_t* perm_R, void* W0p, poetx_stream stream);
+
+/* Forward pass, input-centric (replication review, "Summary"):
+ *   U = X[:, π_R] (gather), V_i = U_i · Q_P,i^T (batched per block), Z = V · W0'^T,
+ *   Y'_i = Z_i · Q_R,i^T, Y[:, π_L] = Y' (scatter).
+ *   X       dtype [N, d_in]  (in)          W0p dtype [d_out, d_in] (in)
+ *   perm_L  int32 [d_out], perm_R int32 [d_in] (in)
+ *   Q_R     dtype [d_out/b, b, b], Q_P dtype [d_in/b, b, b] (in, from poetx_cnp)
+ *   Y       dtype [N, d_out] (out)
+ *   Z_saved dtype [N, d_out] (out) in POETX_FAST mode — pass it back to poetx_backward;
+ *           must be NULL in POETX_MEM mode.
+ * n_tokens == 0 is valid and launches nothing. */
+poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                           const int32_t* perm_L, const int32_t* perm_R, const void* Q_R,
+                           const void* Q_P, void* Y, void* Z_saved, void* workspace,
+                           size_t ws_bytes, poetx_stream stream);
+
+/* Backward pass: dX and the gradients w.r.t. the PACKED skew parameters (only the packed form
+ * is written; replication review, "Summary": compact skew storage; W0 is frozen, so there is
+ * no dW0).  In POETX_MEM mode Z_saved must be NULL and Z is recomputed from X.
+ *   dY dtype [N, d_out], X dtype [N, d_in], W0p, perm_L, perm_R, Q_R, Q_P as in forward (in)
+ *   theta_R, theta_P float32 packed (in; the CNP adjoint needs S)
+ *   Z_saved dtype [N, d_out] (in, FAST) or NULL (MEM)
+ *   dX dtype [N, d_in] (out); grad_theta_R float32 [d_out/b, b(b-1)/2] (out);
+ *   grad_theta_P float32 [d_in/b, b(b-1)/2] (out).
+ * n_tokens == 0 writes zero gradients. */
+poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
+                            const void* W0p, const int32_t* perm_L, const int32_t* perm_R,
+                            const void* Q_R, const void* Q_P, const float* theta_R,
+                            const float* theta_P, const void* Z_saved, void* dX,
+                            float* grad_theta_R, float* grad_theta_P, void* workspace,
+                            size_t ws_bytes, poetx_stream stream);
+
+/* Merge-then-reinitialise (agidaily.cc article: transforms are merged into the weight and
+ * re-initialised during training; replication review, "Reproducibility & code":
+ * merge_then_reinitialize).  Folds R and P into the weight and absorbs fresh permutations:
+ *   M = BD_R · W0' · BD_P;  W0'_new[i][j] = M[π_L^-1(π_L,new(i))][π_R^-1(π_R,new(j))];
+ *   theta_R = theta_P = 0.
+ *   W0p dtype [d_out, d_in] (in/out); Q_R, Q_P (in, the Q the forward used);
+ *   perm_*_old, perm_*_new int32 bijections (in); theta_R, theta_P float32 (out, zeroed). */
+poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, const void* Q_P,
+                         const int32_t* perm_L_old, const int32_t* perm_R_old,
+                         const int32_t* perm_L_new, const int32_t* perm_R_new, float* theta_R,
+                         float* theta_P, void* workspace, size_t ws_bytes, poetx_stream stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* poetx_status_string(poetx_status s);
+
+/* Synchronises the current device, then returns and clears the device-side error word:
+ * POETX_OK, or POETX_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since the last
+ * call.  *detail (if not NULL) receives the raw word (kernel id and wait site). */
+poetx_status poetx_device_status(int* detail);
+
+/* ---------------------------------------------------------------------------- measurement
+ * Launch accounting for benchmarks and profilers (not part of the layer's arithmetic). */
+
+/* Kernel classes of the library's launches. */
+typedef enum {
+  POETX_KC_W_GEMM = 0,       /* Z = V W0'^T and dV = dZ W0' (tensor cores)                 */
+  POETX_KC_BD_GEMM = 1,      /* block-diagonal products BD_P, BD_R and their adjoints       */
+  POETX_KC_GRAD_GEMM = 2,    /* per-block gradient products G = dY'^T Z, dV^T U (split-K)   */
+  POETX_KC_CNP_GEMM = 3,     /* Cayley-Neumann power products (forward and adjoint)         */
+  POETX_KC_MERGE_GEMM = 4,   /* BD_R W0' BD_P of the merge                                  */
+  POETX_KC_PERMUTE = 5,      /* feature-dimension gather / scatter                          */
+  POETX_KC_ELEMENTWISE = 6,  /* unpack, pack, split-K reduction, permutation inverse        */
+  POETX_KC_TEST_GEMM = 7,    /* poetx_test_gemm                                              */
+  POETX_KC_COUNT = 8
+} poetx_kernel_class;
+
+/* Number of kernels this library has launched in the process so far. */
+unsigned long long poetx_launch_count(void);
+
+/* on != 0: forget earlier records and bracket every following launch with a CUDA event pair
+ * on its stream (host-side bookkeeping only; events are created on first use and reused).
+ * on == 0: stop recording. */
+poetx_status poetx_profile_enable(int on);
+
+/* Waits for the recorded events and writes, per kernel class, the number of recorded launches
+ * (counts[POETX_KC_COUNT]) and their summed device time in ms (total_ms[POETX_KC_COUNT]). */
+poetx_status poetx_profile_summary(int* counts, float* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* POETX_H_ */

@@ -135,12 +135,14 @@ def perm_matrix(pi: np.ndarray) -> np.ndarray:
 
 def absorb(W0: np.ndarray, pi_L: np.ndarray, pi_R: np.ndarray) -> np.ndarray:
     """W0' = Pi_L W0 Pi_R^T, i.e. W0'[i, j] = W0[pi_L(i), pi_R(j)] (two permutations absorbed)."""
-    return perm_matrix(pi_L) @ np.asarray(W0, np.float64) @ perm_matrix(pi_R).T
+    return np.asarray(W0, np.float64)[np.asarray(pi_L)][:, np.asarray(pi_R)]
 
 
 def unabsorb(W0p: np.ndarray, pi_L: np.ndarray, pi_R: np.ndarray) -> np.ndarray:
-    """Inverse of absorb: W0 = Pi_L^T W0' Pi_R."""
-    return perm_matrix(pi_L).T @ np.asarray(W0p, np.float64) @ perm_matrix(pi_R)
+    """Inverse of absorb: W0 = Pi_L^T W0' Pi_R, i.e. W0[pi_L(i), pi_R(j)] = W0'[i, j]."""
+    W0 = np.empty_like(np.asarray(W0p, np.float64))
+    W0[np.ix_(np.asarray(pi_L), np.asarray(pi_R))] = W0p
+    return W0
 
 
 def dense_transforms(Q_R, Q_P, pi_L, pi_R):

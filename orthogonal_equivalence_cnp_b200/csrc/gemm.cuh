@@ -1,0 +1,349 @@
+// Batched GEMM core of the POET-X layer.
+//
+// Every contraction of the layer — the block-diagonal products BD_P·x and BD_R·z (replication
+// review of POET-X, "Summary": batch-parallel block-diagonal matmul that never builds the
+// sparse matrix), the W0' products, the per-block gradient products, the Cayley–Neumann
+// power products and the merge — is one call of
+//
+//     D[z][m][n] = sum_k A[z][m][k] * B[z][n][k]          z < batch, m < M, n < N
+//
+// where A and B are views of row-major 2-D arrays.  A view is (base, rows, cols, ld) plus a
+// per-batch coordinate offset (zrow, zcol); "K-major" means A[z][m][k] = mem[z*zrow+m][z*zcol+k]
+// and "MN-major" means A[z][m][k] = mem[z*zrow+k][z*zcol+m] (likewise for B with n).  Split-K
+// writes one partial result per split.  The epilogue is
+//
+//     D1 = alpha1*acc + beta1*C (+ I if diag1)          (bf16 or f32, partial `split` offset)
+//     D2 = alpha2*acc + beta2*C (+ D2 if accum2)        (f32)
+//
+// with an optional addend C.  The bf16 path runs on tcgen05 tensor cores (fp32 accumulation in
+// TMEM, operands staged by TMA into 128-byte-swizzled shared memory); the f32 path runs on the
+// CUDA cores in plain fp32 FMA (no tf32), for the fp32 workloads.
+#pragma once
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace poetx {
+
+struct Operand {
+  const void* base = nullptr;
+  long rows = 0, cols = 0, ld = 0;  // extent and row stride of the whole 2-D array (elements)
+  long zrow = 0, zcol = 0;          // coordinate offset per batch index
+};
+
+struct Epilogue {
+  void* d1 = nullptr;
+  long ld1 = 0, zrow1 = 0, zcol1 = 0, split_stride1 = 0;
+  int d1_dtype = F32;
+  float alpha1 = 1.f, beta1 = 0.f;
+  int diag1 = 0;
+  float* d2 = nullptr;
+  long ld2 = 0, zrow2 = 0, zcol2 = 0;
+  float alpha2 = 1.f, beta2 = 0.f;
+  int accum2 = 0;
+  const void* c = nullptr;
+  long ldc = 0, zrowc = 0, zcolc = 0;
+  int c_dtype = F32;
+};
+
+struct GemmDesc {
+  int M = 0, N = 0, K = 0, batch = 1, splits = 1;
+  Operand A, B;
+  bool a_mn = false, b_mn = false;
+  Epilogue epi;
+};
+
+// Kernel ids recorded in the device error word.
+enum KernelId : int { KID_GEMM_TC = 1 };
+
+// ------------------------------------------------------------------------------- epilogue
+__device__ __forceinline__ void load32(const void* base, long off, int dt, float (&v)[32]) {
+  if (dt == BF16) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(base) + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 u = p[q];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        v[q * 8 + 2 * t] = __uint_as_float(w[t] << 16);
+        v[q * 8 + 2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 f = p[q];
+      v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void store32(void* base, long off, int dt, const float (&v)[32]) {
+  if (dt == BF16) {
+    uint4* p = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      p[q] = make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]), pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
+                        pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]), pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]));
+  } else {
+    float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + off);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  }
+}
+
+// Applies the epilogue to 32 consecutive columns n..n+31 of row m (batch z, split `split`).
+__device__ __forceinline__ void epilogue32(const Epilogue& e, int z, int split, int m, int n,
+                                           const float (&acc)[32]) {
+  float cv[32];
+  const bool has_c = e.c != nullptr;
+  if (has_c) load32(e.c, (long)z * e.zrowc * e.ldc + (long)m * e.ldc + (long)z * e.zcolc + n, e.c_dtype, cv);
+  if (e.d1 != nullptr) {
+    float o[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float v = e.alpha1 * acc[j];
+      if (has_c) v += e.beta1 * cv[j];
+      if (e.diag1 && m == n + j) v += 1.f;
+      o[j] = v;
+    }
+    const long off = ((long)z * e.zrow1 + m) * e.ld1 + (long)z * e.zcol1 + n + (long)split * e.split_stride1;
+    store32(e.d1, off, e.d1_dtype, o);
+  }
+  if (e.d2 != nullptr) {
+    const long off = ((long)z * e.zrow2 + m) * e.ld2 + (long)z * e.zcol2 + n;
+    float o[32];
+    if (e.accum2) load32(e.d2, off, F32, o);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float v = e.alpha2 * acc[j];
+      if (has_c) v += e.beta2 * cv[j];
+      o[j] = e.accum2 ? o[j] + v : v;
+    }
+    store32(e.d2, off, F32, o);
+  }
+}
+
+__device__ __forceinline__ void epilogue1(const Epilogue& e, int z, int split, int m, int n, float acc) {
+  float c = 0.f;
+  if (e.c != nullptr) c = load_elem(e.c, ((long)z * e.zrowc + m) * e.ldc + (long)z * e.zcolc + n, e.c_dtype);
+  if (e.d1 != nullptr) {
+    float v = e.alpha1 * acc + e.beta1 * c + ((e.diag1 && m == n) ? 1.f : 0.f);
+    store_elem(e.d1, ((long)z * e.zrow1 + m) * e.ld1 + (long)z * e.zcol1 + n + (long)split * e.split_stride1,
+               e.d1_dtype, v);
+  }
+  if (e.d2 != nullptr) {
+    const long off = ((long)z * e.zrow2 + m) * e.ld2 + (long)z * e.zcol2 + n;
+    float v = e.alpha2 * acc + e.beta2 * c;
+    e.d2[off] = e.accum2 ? e.d2[off] + v : v;
+  }
+}
+
+// ------------------------------------------------------------------------ tcgen05 kernel
+struct TcArgs {
+  int M, N, K, splits;
+  int a_zrow, a_zcol, b_zrow, b_zcol;
+  Epilogue epi;
+};
+
+constexpr int TC_BM = 128;
+constexpr int TC_BK = 64;  // 64 bf16 = 128 B = one swizzle span
+
+template <int BN, int STAGES>
+__host__ __device__ constexpr size_t tc_smem_bytes() {
+  return (size_t)STAGES * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) + 1024 /*align*/ + 256 /*barriers*/;
+}
+
+// One CTA computes one BM x BN output tile of one (batch, split).  Warp 0 lane 0 streams A/B
+// k-tiles with TMA into a STAGES-deep ring; warp 1 lane 0 issues tcgen05.mma (M=128, N=BN,
+// K=16) into a TMEM accumulator of BN fp32 columns and frees ring slots with tcgen05.commit;
+// then all four warps drain TMEM (warp w owns TMEM lanes 32w..32w+31 = tile rows) through the
+// epilogue.  Every wait is bounded (kWaitLimitNs); on a timeout the CTA records the error,
+// skips the rest of its work and still releases its TMEM.
+template <int BN, int STAGES, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(128, 1)
+    gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const TcArgs args) {
+  constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
+  constexpr uint32_t B_BYTES = BN * TC_BK * 2;
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t IDESC = sm100::idesc_bf16_f32(TC_BM, BN, A_MN, B_MN);
+  using namespace sm100;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  const uint32_t smem0 = smem_u32(smem);
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int z = blockIdx.z / args.splits, split = blockIdx.z % args.splits;
+  const int m0 = blockIdx.y * TC_BM, n0 = blockIdx.x * BN;
+  const int KT = (args.K + TC_BK - 1) / TC_BK;
+  const int kt0 = (int)((long)KT * split / args.splits);
+  const int kt1 = (int)((long)KT * (split + 1) / args.splits);
+  const int nkt = kt1 - kt0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(accum_bar, 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 1)) break;
+      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+      const int k0 = (kt0 + i) * TC_BK;
+      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+      if (!A_MN) {
+        tma_load_2d(sa, &tmA, full_bar(s), z * args.a_zcol + k0, z * args.a_zrow + m0);
+      } else {
+#pragma unroll
+        for (int h = 0; h < TC_BM / 64; ++h)
+          tma_load_2d(sa + h * 8192, &tmA, full_bar(s), z * args.a_zcol + m0 + 64 * h, z * args.a_zrow + k0);
+      }
+      if (!B_MN) {
+        tma_load_2d(sb, &tmB, full_bar(s), z * args.b_zcol + k0, z * args.b_zrow + n0);
+      } else {
+#pragma unroll
+        for (int h = 0; h < BN / 64; ++h)
+          tma_load_2d(sb + h * 8192, &tmB, full_bar(s), z * args.b_zcol + n0 + 64 * h, z * args.b_zrow + k0);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (!mbar_wait(full_bar(s), ph, KID_GEMM_TC, 2)) break;
+      tc_fence_after();
+      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk) {
+        const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024) : smem_desc_sw128(sa + kk * 32, 16, 1024);
+        const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+        mma_bf16(tmem_d, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(empty_bar(s));
+    }
+    mma_commit(accum_bar);
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: TMEM -> registers -> global
+  bool ok = mbar_wait(accum_bar, 0, KID_GEMM_TC, 3);
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after();
+  if (ok) {
+    const int m = m0 + warp * 32 + lane;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, r);
+      tmem_wait_ld();
+      float acc[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc[j] = nkt > 0 ? __uint_as_float(r[j]) : 0.f;
+      if (m < args.M) epilogue32(args.epi, z, split, m, n0 + c, acc);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem_d, BN);
+}
+
+// ---------------------------------------------------------------------------- f32 SIMT kernel
+struct SimtArgs {
+  int M, N, K, splits;
+  const float* A;
+  long lda, a_zrow, a_zcol;
+  int a_mn;
+  const float* B;
+  long ldb, b_zrow, b_zcol;
+  int b_mn;
+  Epilogue epi;
+};
+
+// 64x64 output tile per 256-thread block, 4x4 per thread, k-steps of 16 staged in smem.
+__global__ void __launch_bounds__(256) gemm_f32_simt(const SimtArgs p) {
+  __shared__ float As[16][65];
+  __shared__ float Bs[16][65];
+  const int z = blockIdx.z / p.splits, split = blockIdx.z % p.splits;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int KT = (p.K + 15) / 16;
+  const int kt0 = (int)((long)KT * split / p.splits), kt1 = (int)((long)KT * (split + 1) / p.splits);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int kt = kt0; kt < kt1; ++kt) {
+    const int k0 = kt * 16;
+    for (int e = threadIdx.x; e < 1024; e += 256) {
+      int mm, kk;
+      if (p.a_mn) { mm = e & 63; kk = e >> 6; } else { kk = e & 15; mm = e >> 4; }
+      const int m = m0 + mm, k = k0 + kk;
+      float v = 0.f;
+      if (m < p.M && k < p.K)
+        v = p.a_mn ? p.A[((long)z * p.a_zrow + k) * p.lda + (long)z * p.a_zcol + m]
+                   : p.A[((long)z * p.a_zrow + m) * p.lda + (long)z * p.a_zcol + k];
+      As[kk][mm] = v;
+      int nn, kb;
+      if (p.b_mn) { nn = e & 63; kb = e >> 6; } else { kb = e & 15; nn = e >> 4; }
+      const int n = n0 + nn, kq = k0 + kb;
+      float w = 0.f;
+      if (n < p.N && kq < p.K)
+        w = p.b_mn ? p.B[((long)z * p.b_zrow + kq) * p.ldb + (long)z * p.b_zcol + n]
+                   : p.B[((long)z * p.b_zrow + n) * p.ldb + (long)z * p.b_zcol + kq];
+      Bs[kb][nn] = w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int m = m0 + ty + 16 * i, n = n0 + tx + 16 * j;
+      if (m < p.M && n < p.N) epilogue1(p.epi, z, split, m, n, acc[i][j]);
+    }
+}
+
+}  // namespace poetx

@@ -1,0 +1,813 @@
+// libpoetx: C ABI of the POET-X layer (see include/poetx.h for the contract of every call).
+//
+// Single translation unit: the kernels live in the included headers.  This file holds the
+// host side: argument validation, workspace planning, TMA tensor-map encoding, and the
+// orchestration of the input-centric chain (replication review of POET-X, "Summary").
+#include <algorithm>
+#include <atomic>
+#include <utility>
+#include <vector>
+#include <initializer_list>
+#include <mutex>
+
+#include "../../include/poetx_testing.h"
+#include "common.cuh"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+#include "sm100.cuh"
+
+using namespace poetx;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kNumSms = 148;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int esize(int dt) { return dt == BF16 ? 2 : 4; }
+
+// Sequential carve-out of the caller's workspace (offsets only; nothing is allocated).
+struct Plan {
+  size_t total = 0;
+  size_t take(size_t bytes) {
+    size_t o = total;
+    total += align256(bytes);
+    return o;
+  }
+};
+
+#define POETX_TRY(expr)                  \
+  do {                                   \
+    poetx_status _s = (expr);            \
+    if (_s != POETX_OK) return _s;       \
+  } while (0)
+
+inline poetx_status last_launch() {
+  return cudaGetLastError() == cudaSuccess ? POETX_OK : POETX_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ launch accounting
+// Every kernel launch of the library goes through a LaunchScope: it counts the launch and, when
+// profiling is on, brackets it with a CUDA event pair on the launching stream.
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> recs;
+  std::atomic<unsigned long long> launches{0};
+  cudaEvent_t take() {
+    if (used == pool.size()) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+};
+Profiler& prof() {
+  static Profiler* p = new Profiler();  // never destroyed: events may outlive static teardown
+  return *p;
+}
+
+struct LaunchScope {
+  int cls;
+  cudaStream_t st;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  LaunchScope(int c, cudaStream_t s) : cls(c), st(s) {
+    Profiler& p = prof();
+    p.launches.fetch_add(1, std::memory_order_relaxed);
+    if (p.on) {
+      std::lock_guard<std::mutex> g(p.mu);
+      e0 = p.take();
+      e1 = p.take();
+      if (e0 && e1) cudaEventRecord(e0, st);
+    }
+  }
+  ~LaunchScope() {
+    if (e0 && e1) {
+      Profiler& p = prof();
+      cudaEventRecord(e1, st);
+      std::lock_guard<std::mutex> g(p.mu);
+      p.recs.push_back({cls, {e0, e1}});
+    }
+  }
+};
+
+poetx_status check_desc(const poetx_desc* d) {
+  if (d == nullptr) return POETX_ERR_INVALID_ARG;
+  if (d->dtype != POETX_F32 && d->dtype != POETX_BF16) return POETX_ERR_INVALID_ARG;
+  if (d->mode != POETX_FAST && d->mode != POETX_MEM) return POETX_ERR_INVALID_ARG;
+  if (d->d_in <= 0 || d->d_out <= 0 || d->b <= 0 || d->k < 0) return POETX_ERR_INVALID_ARG;
+  const int b = d->b;
+  if (b != 32 && b != 64 && b != 128 && b != 256 && b != 512) return POETX_ERR_UNSUPPORTED_SHAPE;
+  if (d->dtype == POETX_BF16 && b < 64) return POETX_ERR_UNSUPPORTED_SHAPE;
+  if (d->k > 8) return POETX_ERR_UNSUPPORTED_SHAPE;
+  if (d->d_in % b != 0 || d->d_out % b != 0) return POETX_ERR_UNSUPPORTED_SHAPE;
+  // One feature row (d * element size) must fit in a block's shared memory for the
+  // permutation kernel: at most 128 KiB.
+  const int dmax = d->dtype == POETX_BF16 ? 65536 : 32768;
+  if (d->d_in > dmax || d->d_out > dmax) return POETX_ERR_UNSUPPORTED_SHAPE;
+  return POETX_OK;
+}
+
+// ------------------------------------------------------------------------------ GEMM dispatch
+// Checks that every element a GEMM may address lies inside its arrays (the tensor-core path
+// relies on TMA zero-fill beyond the array extent; the SIMT path masks m < M, n < N, k < K).
+bool view_fits(const Operand& op, bool mn, long mnext, long kext, long batch) {
+  if (op.base == nullptr || op.ld < op.cols || op.rows <= 0 || op.cols <= 0) return false;
+  const long r_last = (batch - 1) * op.zrow + (mn ? kext : mnext);
+  const long c_last = (batch - 1) * op.zcol + (mn ? mnext : kext);
+  return r_last <= op.rows && c_last <= op.cols;
+}
+
+poetx_status check_gemm(const GemmDesc& g, int dt) {
+  if (g.M <= 0 || g.N <= 0 || g.K < 0 || g.batch <= 0 || g.splits <= 0) return POETX_ERR_INVALID_ARG;
+  if (g.batch * (long)g.splits > 65535) return POETX_ERR_UNSUPPORTED_SHAPE;
+  if (g.K > 0) {
+    if (!view_fits(g.A, g.a_mn, g.M, g.K, g.batch)) return POETX_ERR_INVALID_ARG;
+    if (!view_fits(g.B, g.b_mn, g.N, g.K, g.batch)) return POETX_ERR_INVALID_ARG;
+  }
+  if (dt == BF16) {
+    // Tensor-core path: N in whole 64-column tiles, 16-byte aligned rows and coordinates.
+    if (g.N % 64 != 0) return POETX_ERR_UNSUPPORTED_SHAPE;
+    const Operand* ops[2] = {&g.A, &g.B};
+    for (const Operand* op : ops)
+      if (!aligned16(op->base) || op->ld % 8 || op->zcol % 8) return POETX_ERR_ALIGNMENT;
+    const Epilogue& e = g.epi;
+    if (e.d1 && (!aligned16(e.d1) || e.ld1 % 8 || e.zcol1 % 8 || e.split_stride1 % 8)) return POETX_ERR_ALIGNMENT;
+    if (e.d2 && (!aligned16(e.d2) || e.ld2 % 4 || e.zcol2 % 4)) return POETX_ERR_ALIGNMENT;
+    if (e.c && (!aligned16(e.c) || e.ldc % 8 || e.zcolc % 8)) return POETX_ERR_ALIGNMENT;
+  }
+  return POETX_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 2-D tensor map over a whole operand array with a box of (inner x outer) elements and
+// 128-byte swizzle; reads beyond the array extent return zeros.
+bool make_tmap(CUtensorMap* m, const Operand& op, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)op.cols, (cuuint64_t)op.rows};
+  cuuint64_t strides[1] = {(cuuint64_t)op.ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(op.base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int ST, bool AMN, bool BMN>
+poetx_status launch_tc(const GemmDesc& g, cudaStream_t st, int cls) {
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
+  constexpr size_t smem = tc_smem_bytes<BN, ST>();
+  auto kern = gemm_bf16_tc<BN, ST, AMN, BMN>;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return POETX_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, g.A, 64, AMN ? 64 : TC_BM)) return POETX_ERR_CUDA;
+  if (!make_tmap(&tb, g.B, 64, BMN ? 64 : BN)) return POETX_ERR_CUDA;
+  TcArgs a;
+  a.M = g.M; a.N = g.N; a.K = g.K; a.splits = g.splits;
+  a.a_zrow = (int)g.A.zrow; a.a_zcol = (int)g.A.zcol; a.b_zrow = (int)g.B.zrow; a.b_zcol = (int)g.B.zcol;
+  a.epi = g.epi;
+  dim3 grid(g.N / BN, (g.M + TC_BM - 1) / TC_BM, g.batch * g.splits);
+  LaunchScope ls(cls, st);
+  kern<<<grid, 128, smem, st>>>(ta, tb, a);
+  return last_launch();
+}
+
+template <int BN, int ST>
+poetx_status launch_tc_major(const GemmDesc& g, cudaStream_t st, int cls) {
+  if (!g.a_mn && !g.b_mn) return launch_tc<BN, ST, false, false>(g, st, cls);
+  if (!g.a_mn && g.b_mn) return launch_tc<BN, ST, false, true>(g, st, cls);
+  if (g.a_mn && !g.b_mn) return launch_tc<BN, ST, true, false>(g, st, cls);
+  return launch_tc<BN, ST, true, true>(g, st, cls);
+}
+
+poetx_status run_gemm(int dt, const GemmDesc& g, cudaStream_t st, int cls) {
+  POETX_TRY(check_gemm(g, dt));
+  if (dt == BF16) {
+    if (g.N % 256 == 0) return launch_tc_major<256, 4>(g, st, cls);
+    if (g.N % 128 == 0) return launch_tc_major<128, 6>(g, st, cls);
+    return launch_tc_major<64, 8>(g, st, cls);
+  }
+  SimtArgs p;
+  p.M = g.M; p.N = g.N; p.K = g.K; p.splits = g.splits;
+  p.A = static_cast<const float*>(g.A.base); p.lda = g.A.ld; p.a_zrow = g.A.zrow; p.a_zcol = g.A.zcol; p.a_mn = g.a_mn;
+  p.B = static_cast<const float*>(g.B.base); p.ldb = g.B.ld; p.b_zrow = g.B.zrow; p.b_zcol = g.B.zcol; p.b_mn = g.b_mn;
+  p.epi = g.epi;
+  dim3 grid((g.N + 63) / 64, (g.M + 63) / 64, g.batch * g.splits);
+  LaunchScope ls(cls, st);
+  gemm_f32_simt<<<grid, 256, 0, st>>>(p);
+  return last_launch();
+}
+
+// -------------------------------------------------------------------- elementwise launches
+int ew_grid(long n) { return (int)std::min<long>((n + 255) / 256, (long)kNumSms * 16); }
+
+poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld_out, long rows, int cols,
+                          const int32_t* colmap, const int32_t* rowmap, bool scatter, cudaStream_t st) {
+  if (rows <= 0) return POETX_OK;
+  const size_t row_bytes = (size_t)cols * esize(dt);
+  int rb = (int)std::max<size_t>(1, std::min<size_t>(4, (96 * 1024) / row_bytes));
+  const size_t smem = rb * row_bytes;
+  const int grid = (int)std::min<long>((rows + rb - 1) / rb, (long)kNumSms * 8);
+  if (dt == BF16) {
+    auto k = permute_cols_kernel<__nv_bfloat16>;
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return POETX_ERR_CUDA;
+    LaunchScope ls(POETX_KC_PERMUTE, st);
+    k<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(in), ld_in, static_cast<__nv_bfloat16*>(out), ld_out,
+                               rows, cols, colmap, rowmap, scatter ? 1 : 0, rb);
+  } else {
+    auto k = permute_cols_kernel<float>;
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return POETX_ERR_CUDA;
+    LaunchScope ls(POETX_KC_PERMUTE, st);
+    k<<<grid, 256, smem, st>>>(static_cast<const float*>(in), ld_in, static_cast<float*>(out), ld_out, rows, cols,
+                               colmap, rowmap, scatter ? 1 : 0, rb);
+  }
+  return last_launch();
+}
+
+poetx_status unpack(const float* theta, long nblocks, int b, void* o1, int dt1, long ld1, void* o2, int dt2,
+                    long ld2, float* of32, bool add_identity, cudaStream_t st) {
+  const long total = nblocks * (long)b * b;
+  if (total == 0) return POETX_OK;
+  LaunchScope ls(POETX_KC_ELEMENTWISE, st);
+  unpack_skew_kernel<<<ew_grid(total), 256, 0, st>>>(theta, nblocks, b, o1, dt1, ld1, o2, dt2, ld2, of32,
+                                                      add_identity ? 1 : 0);
+  return last_launch();
+}
+
+poetx_status pack(const float* GS, long nblocks, int b, float* g, cudaStream_t st) {
+  const long total = nblocks * (long)b * b;
+  if (total == 0) return POETX_OK;
+  LaunchScope ls(POETX_KC_ELEMENTWISE, st);
+  pack_antisym_kernel<<<ew_grid(total), 256, 0, st>>>(GS, nblocks, b, g);
+  return last_launch();
+}
+
+poetx_status reduce_splits(const float* part, int splits, long rows, int cols, float* out, void* out2, int dt2,
+                           long ld2, cudaStream_t st) {
+  const long total = rows * cols;
+  if (total == 0) return POETX_OK;
+  LaunchScope ls(POETX_KC_ELEMENTWISE, st);
+  reduce_splits_kernel<<<ew_grid(total), 256, 0, st>>>(part, splits, total, rows, cols, out, out2, dt2, ld2);
+  return last_launch();
+}
+
+// -------------------------------------------------------------------- GEMM building blocks
+Operand view(const void* base, long rows, long cols, long ld, long zrow = 0, long zcol = 0) {
+  Operand o;
+  o.base = base; o.rows = rows; o.cols = cols; o.ld = ld; o.zrow = zrow; o.zcol = zcol;
+  return o;
+}
+
+// Out[:, blk z] = In[:, blk z] . Q_z^T  (forward block-diagonal application; tokens are rows).
+poetx_status bd_forward(int dt, long n, int d, int b, const void* in, const void* Q, void* out, cudaStream_t st) {
+  GemmDesc g;
+  g.M = (int)n; g.N = b; g.K = b; g.batch = d / b;
+  g.A = view(in, n, d, d, 0, b);
+  g.B = view(Q, d, b, b, b, 0);
+  g.epi.d1 = out; g.epi.d1_dtype = dt; g.epi.ld1 = d; g.epi.zcol1 = b;
+  return run_gemm(dt, g, st, POETX_KC_BD_GEMM);
+}
+
+// Out[:, blk z] = In[:, blk z] . Q_z  (adjoint of bd_forward w.r.t. its input).
+poetx_status bd_backward(int dt, long n, int d, int b, const void* in, const void* Q, void* out, cudaStream_t st) {
+  GemmDesc g;
+  g.M = (int)n; g.N = b; g.K = b; g.batch = d / b;
+  g.A = view(in, n, d, d, 0, b);
+  g.B = view(Q, d, b, b, b, 0);
+  g.b_mn = true;
+  g.epi.d1 = out; g.epi.d1_dtype = dt; g.epi.ld1 = d; g.epi.zcol1 = b;
+  return run_gemm(dt, g, st, POETX_KC_BD_GEMM);
+}
+
+// Gpart[s][z] = Lhs[:, blk z]^T . Rhs[:, blk z] over split s of the tokens (f32 partials).
+int grad_splits(int dt, long n, int nb, int b) {
+  const long tiles = dt == BF16 ? (long)nb * ((b + 127) / 128) * (b >= 256 ? b / 256 : 1)
+                                : (long)nb * ((b + 63) / 64) * ((b + 63) / 64);
+  const long kt = dt == BF16 ? (n + 63) / 64 : (n + 15) / 16;
+  long s = std::max<long>(1, kNumSms / std::max<long>(1, tiles));
+  s = std::min<long>(s, std::max<long>(1, kt / 4));
+  return (int)std::max<long>(1, std::min<long>(s, 64));
+}
+
+poetx_status block_grads(int dt, long n, int d, int b, const void* lhs, const void* rhs, float* part, int splits,
+                         cudaStream_t st) {
+  GemmDesc g;
+  g.M = b; g.N = b; g.K = (int)n; g.batch = d / b; g.splits = splits;
+  g.A = view(lhs, n, d, d, 0, b); g.a_mn = true;
+  g.B = view(rhs, n, d, d, 0, b); g.b_mn = true;
+  g.epi.d1 = part; g.epi.d1_dtype = F32; g.epi.ld1 = b; g.epi.zrow1 = b; g.epi.split_stride1 = (long)d * b;
+  return run_gemm(dt, g, st, POETX_KC_GRAD_GEMM);
+}
+
+// ------------------------------------------------------------------------- CNP forward
+size_t cnp_fwd_ws(int b, int k, int dt, long nb) {
+  if (k == 0 || nb == 0) return 0;
+  const size_t blk = (size_t)nb * b * b;
+  Plan p;
+  p.take(blk * 4);                  // S (f32)
+  if (dt == BF16) p.take(blk * 2);  // S (bf16 operand)
+  if (k >= 2) { p.take(blk * esize(dt)); p.take(blk * esize(dt)); }  // M_j ping-pong
+  return p.total;
+}
+
+// Q = (I + S)(I + S + ... + S^k) by the Horner recursion on M_j = N_j - I:
+//   M_1 = S;  M_j = S + S.M_{j-1};  Q = I + S + S.M_k  (k >= 1);  Q = I + S (k = 0).
+// Keeping M_j = N_j - I (small) instead of N_j keeps the bf16 intermediates accurate; the
+// exact I + S part is added in fp32 in the epilogue (replication review, "Summary": the fused
+// CNP reuses the lower powers across terms).
+poetx_status cnp_fwd_run(int b, int k, int dt, long nb, const float* theta, void* Q, char* ws, cudaStream_t st) {
+  if (nb == 0) return POETX_OK;
+  if (k == 0) return unpack(theta, nb, b, Q, dt, b, nullptr, dt, 0, nullptr, true, st);
+  const size_t blk = (size_t)nb * b * b;
+  Plan p;
+  float* S32 = reinterpret_cast<float*>(ws + p.take(blk * 4));
+  void* Sop = dt == BF16 ? static_cast<void*>(ws + p.take(blk * 2)) : static_cast<void*>(S32);
+  void* Mbuf[2] = {nullptr, nullptr};
+  if (k >= 2) { Mbuf[0] = ws + p.take(blk * esize(dt)); Mbuf[1] = ws + p.take(blk * esize(dt)); }
+  POETX_TRY(unpack(theta, nb, b, dt == BF16 ? Sop : nullptr, dt, b, nullptr, dt, 0, S32, false, st));
+  const void* Mprev = Sop;
+  for (int j = 2; j <= k + 1; ++j) {
+    const bool last = (j == k + 1);
+    void* dst = last ? Q : Mbuf[j & 1];
+    GemmDesc g;
+    g.M = b; g.N = b; g.K = b; g.batch = (int)nb;
+    g.A = view(Sop, nb * b, b, b, b, 0);
+    g.B = view(Mprev, nb * b, b, b, b, 0); g.b_mn = true;
+    g.epi.d1 = dst; g.epi.d1_dtype = dt; g.epi.ld1 = b; g.epi.zrow1 = b;
+    g.epi.alpha1 = 1.f; g.epi.beta1 = 1.f; g.epi.diag1 = last ? 1 : 0;
+    g.epi.c = S32; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+    Mprev = dst;
+  }
+  return POETX_OK;
+}
+
+// ------------------------------------------------------------------------- CNP backward
+size_t cnp_bwd_ws(int b, int k, int dt, long nb) {
+  if (nb == 0) return 0;
+  const size_t blk = (size_t)nb * b * b;
+  Plan p;
+  p.take(blk * 4);  // G (f32)
+  if (k >= 1) {
+    p.take(blk * 4);                               // E (f32), then G_S
+    p.take(blk * 4);                               // S (f32)
+    if (dt == BF16) p.take(blk * 2);               // S (bf16 operand)
+    p.take(blk * (size_t)k * esize(dt));           // A-stack [G | Gbar_k | ... | Gbar_2]
+    p.take(blk * (size_t)k * esize(dt));           // B-stack [M_k | ... | M_1]
+  }
+  return p.total;
+}
+
+// Packed gradient from G = dL/dQ (split-K partials) by the adjoint of the Horner recursion
+// N_0 = I, N_j = I + S.N_{j-1}, Q = (I + S).N_k:
+//   G_S = G.N_k^T + sum_{j=1..k} Gbar_j.N_{j-1}^T,  Gbar_k = (I + S^T).G,  Gbar_{j-1} = S^T.Gbar_j,
+// then g[p(i,j)] = G_S[i][j] - G_S[j][i].  With N_j = I + M_j and S^T = -S this is
+//   G_S = E + [G | Gbar_k | ... | Gbar_2] . [M_k | ... | M_1]^T,   E = G + sum_{j=1..k} Gbar_j,
+// one long-K product plus an fp32 running sum E (the dominant 2G term never rounds to bf16).
+poetx_status cnp_bwd_run(int b, int k, int dt, long nb, const float* theta, const float* part, int splits,
+                         float* grad, char* ws, cudaStream_t st) {
+  if (nb == 0) return POETX_OK;
+  const size_t blk = (size_t)nb * b * b;
+  const long rows = nb * b;
+  Plan p;
+  float* G32 = reinterpret_cast<float*>(ws + p.take(blk * 4));
+  if (k == 0) {
+    POETX_TRY(reduce_splits(part, splits, rows, b, G32, nullptr, F32, 0, st));
+    return pack(G32, nb, b, grad, st);
+  }
+  float* E = reinterpret_cast<float*>(ws + p.take(blk * 4));
+  float* S32 = reinterpret_cast<float*>(ws + p.take(blk * 4));
+  void* Sop = dt == BF16 ? static_cast<void*>(ws + p.take(blk * 2)) : static_cast<void*>(S32);
+  char* Ast = ws + p.take(blk * (size_t)k * esize(dt));
+  char* Bst = ws + p.take(blk * (size_t)k * esize(dt));
+  const long kb = (long)k * b;
+  const int es = esize(dt);
+  auto aslot = [&](int t) { return static_cast<void*>(Ast + (size_t)t * b * es); };
+  auto bslot = [&](int t) { return static_cast<void*>(Bst + (size_t)t * b * es); };
+
+  POETX_TRY(reduce_splits(part, splits, rows, b, G32, aslot(0), dt, kb, st));
+  POETX_TRY(unpack(theta, nb, b, dt == BF16 ? Sop : nullptr, dt, b, bslot(k - 1), dt, kb, S32, false, st));
+
+  auto chain_gemm = [&](const void* Bsrc) {
+    GemmDesc g;
+    g.M = b; g.N = b; g.K = b; g.batch = (int)nb;
+    g.A = view(Sop, rows, b, b, b, 0);
+    g.B = view(Bsrc, rows, b, kb, b, 0); g.b_mn = true;
+    return g;
+  };
+  // M_j = S + S.M_{j-1} into B-slot k-j.
+  for (int j = 2; j <= k; ++j) {
+    GemmDesc g = chain_gemm(bslot(k - j + 1));
+    g.epi.d1 = bslot(k - j); g.epi.d1_dtype = dt; g.epi.ld1 = kb; g.epi.zrow1 = b;
+    g.epi.alpha1 = 1.f; g.epi.beta1 = 1.f;
+    g.epi.c = S32; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+  }
+  // Gbar_k = G - S.G into A-slot 1 (k >= 2);  E = 2G - S.G.
+  {
+    GemmDesc g = chain_gemm(aslot(0));
+    if (k >= 2) {
+      g.epi.d1 = aslot(1); g.epi.d1_dtype = dt; g.epi.ld1 = kb; g.epi.zrow1 = b;
+      g.epi.alpha1 = -1.f; g.epi.beta1 = 1.f;
+    }
+    g.epi.c = G32; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
+    g.epi.d2 = E; g.epi.ld2 = b; g.epi.zrow2 = b; g.epi.alpha2 = -1.f; g.epi.beta2 = 2.f; g.epi.accum2 = 0;
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+  }
+  // Gbar_j = -S.Gbar_{j+1} (Gbar_{j+1} in A-slot k-j) into A-slot k-j+1 (j >= 2);  E += Gbar_j.
+  for (int j = k - 1; j >= 1; --j) {
+    GemmDesc g = chain_gemm(aslot(k - j));
+    if (j >= 2) {
+      g.epi.d1 = aslot(k - j + 1); g.epi.d1_dtype = dt; g.epi.ld1 = kb; g.epi.zrow1 = b;
+      g.epi.alpha1 = -1.f; g.epi.beta1 = 0.f;
+    }
+    g.epi.d2 = E; g.epi.ld2 = b; g.epi.zrow2 = b; g.epi.alpha2 = -1.f; g.epi.beta2 = 0.f; g.epi.accum2 = 1;
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+  }
+  // G_S = E + A-stack . B-stack^T  (K = k.b), written over E.
+  {
+    GemmDesc g;
+    g.M = b; g.N = b; g.K = (int)kb; g.batch = (int)nb;
+    g.A = view(Ast, rows, kb, kb, b, 0);
+    g.B = view(Bst, rows, kb, kb, b, 0);
+    g.epi.d1 = E; g.epi.d1_dtype = F32; g.epi.ld1 = b; g.epi.zrow1 = b; g.epi.alpha1 = 1.f; g.epi.beta1 = 1.f;
+    g.epi.c = E; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+  }
+  return pack(E, nb, b, grad, st);
+}
+
+// ------------------------------------------------------------------------- layer plans
+struct FwdPlan {
+  size_t U, V, Yp, Z, total;
+};
+FwdPlan fwd_plan(const poetx_desc* d, long n) {
+  const size_t e = esize(d->dtype);
+  Plan p;
+  FwdPlan f;
+  f.U = p.take(n * d->d_in * e);
+  f.V = p.take(n * d->d_in * e);
+  f.Yp = p.take(n * d->d_out * e);
+  f.Z = d->mode == POETX_MEM ? p.take(n * d->d_out * e) : 0;
+  f.total = p.total;
+  return f;
+}
+
+struct BwdPlan {
+  size_t dYp, dZ, dV, U, dU, V, Z, GpR, GpP, cnp, total;
+  int sR, sP;
+};
+BwdPlan bwd_plan(const poetx_desc* d, long n) {
+  const size_t e = esize(d->dtype);
+  const int b = d->b, nbo = d->d_out / b, nbi = d->d_in / b;
+  BwdPlan w;
+  Plan p;
+  w.dYp = p.take(n * d->d_out * e);
+  w.dZ = p.take(n * d->d_out * e);
+  w.dV = p.take(n * d->d_in * e);
+  w.U = p.take(n * d->d_in * e);
+  w.dU = p.take(n * d->d_in * e);
+  w.V = d->mode == POETX_MEM ? p.take(n * d->d_in * e) : 0;
+  w.Z = d->mode == POETX_MEM ? p.take(n * d->d_out * e) : 0;
+  w.sR = grad_splits(d->dtype, n, nbo, b);
+  w.sP = grad_splits(d->dtype, n, nbi, b);
+  w.GpR = p.take((size_t)w.sR * nbo * b * b * 4);
+  w.GpP = p.take((size_t)w.sP * nbi * b * b * 4);
+  w.cnp = p.take(std::max(cnp_bwd_ws(b, d->k, d->dtype, nbo), cnp_bwd_ws(b, d->k, d->dtype, nbi)));
+  w.total = p.total;
+  return w;
+}
+
+size_t cnp_layer_ws(const poetx_desc* d) {
+  return std::max(cnp_fwd_ws(d->b, d->k, d->dtype, d->d_out / d->b), cnp_fwd_ws(d->b, d->k, d->dtype, d->d_in / d->b));
+}
+
+struct MergePlan {
+  size_t T, M2, inv, sigL, sigR, total;
+};
+MergePlan merge_plan(const poetx_desc* d) {
+  const size_t e = esize(d->dtype);
+  MergePlan m;
+  Plan p;
+  m.T = p.take((size_t)d->d_out * d->d_in * e);
+  m.M2 = p.take((size_t)d->d_out * d->d_in * e);
+  m.inv = p.take((size_t)std::max(d->d_in, d->d_out) * 4);
+  m.sigL = p.take((size_t)d->d_out * 4);
+  m.sigR = p.take((size_t)d->d_in * 4);
+  m.total = p.total;
+  return m;
+}
+
+poetx_status check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (p == nullptr) return POETX_ERR_INVALID_ARG;
+    if (!aligned16(p)) return POETX_ERR_ALIGNMENT;
+  }
+  return POETX_OK;
+}
+
+poetx_status check_ws(const void* ws, size_t have, size_t need) {
+  if (need == 0) return POETX_OK;
+  if (ws == nullptr || have < need) return POETX_ERR_WORKSPACE;
+  if (!aligned16(ws)) return POETX_ERR_ALIGNMENT;
+  return POETX_OK;
+}
+
+// Forward chain into caller buffers; `Z` receives the W0'-GEMM output.
+poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const void* W0p, const int32_t* pL,
+                           const int32_t* pR, const void* QR, const void* QP, void* Y, void* Z, char* U, char* V,
+                           char* Yp, cudaStream_t st) {
+  const int dt = d->dtype, b = d->b;
+  POETX_TRY(permute_cols(dt, X, d->d_in, U, d->d_in, n, d->d_in, pR, nullptr, false, st));
+  POETX_TRY(bd_forward(dt, n, d->d_in, b, U, QP, V, st));
+  {
+    GemmDesc g;
+    g.M = (int)n; g.N = d->d_out; g.K = d->d_in;
+    g.A = view(V, n, d->d_in, d->d_in);
+    g.B = view(W0p, d->d_out, d->d_in, d->d_in);
+    g.epi.d1 = Z; g.epi.d1_dtype = dt; g.epi.ld1 = d->d_out;
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_W_GEMM));
+  }
+  if (Y == nullptr) return POETX_OK;  // recompute only (mem-mode backward)
+  POETX_TRY(bd_forward(dt, n, d->d_out, b, Z, QR, Yp, st));
+  return permute_cols(dt, Yp, d->d_out, Y, d->d_out, n, d->d_out, pL, nullptr, true, st);
+}
+
+}  // namespace
+
+// =============================================================================== C ABI
+extern "C" {
+
+const char* poetx_status_string(poetx_status s) {
+  switch (s) {
+    case POETX_OK: return "POETX_OK";
+    case POETX_ERR_INVALID_ARG: return "POETX_ERR_INVALID_ARG";
+    case POETX_ERR_UNSUPPORTED_SHAPE: return "POETX_ERR_UNSUPPORTED_SHAPE";
+    case POETX_ERR_ALIGNMENT: return "POETX_ERR_ALIGNMENT";
+    case POETX_ERR_WORKSPACE: return "POETX_ERR_WORKSPACE";
+    case POETX_ERR_CUDA: return "POETX_ERR_CUDA";
+    case POETX_ERR_DEVICE_TIMEOUT: return "POETX_ERR_DEVICE_TIMEOUT";
+  }
+  return "POETX_ERR_UNKNOWN";
+}
+
+size_t poetx_workspace_size(const poetx_desc* desc, int n_tokens) {
+  if (check_desc(desc) != POETX_OK || n_tokens < 0) return 0;
+  size_t w = cnp_layer_ws(desc);
+  w = std::max(w, fwd_plan(desc, n_tokens).total);
+  w = std::max(w, bwd_plan(desc, n_tokens).total);
+  w = std::max(w, merge_plan(desc).total);
+  return w;
+}
+
+size_t poetx_cnp_blocks_workspace_size(const poetx_desc* desc, int n_blocks) {
+  if (check_desc(desc) != POETX_OK || n_blocks < 0) return 0;
+  return cnp_fwd_ws(desc->b, desc->k, desc->dtype, n_blocks);
+}
+
+poetx_status poetx_cnp_blocks(const poetx_desc* desc, int n_blocks, const float* theta, void* Q, void* workspace,
+                              size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_blocks < 0) return POETX_ERR_INVALID_ARG;
+  if (n_blocks == 0) return POETX_OK;
+  POETX_TRY(check_ptrs({theta, Q}));
+  POETX_TRY(check_ws(workspace, ws_bytes, cnp_fwd_ws(desc->b, desc->k, desc->dtype, n_blocks)));
+  return cnp_fwd_run(desc->b, desc->k, desc->dtype, n_blocks, theta, Q, static_cast<char*>(workspace), stream);
+}
+
+poetx_status poetx_cnp(const poetx_desc* desc, const float* theta_R, const float* theta_P, void* Q_R, void* Q_P,
+                       void* workspace, size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  POETX_TRY(check_ptrs({theta_R, theta_P, Q_R, Q_P}));
+  POETX_TRY(check_ws(workspace, ws_bytes, cnp_layer_ws(desc)));
+  char* ws = static_cast<char*>(workspace);
+  const int b = desc->b;
+  POETX_TRY(cnp_fwd_run(b, desc->k, desc->dtype, desc->d_out / b, theta_R, Q_R, ws, stream));
+  return cnp_fwd_run(b, desc->k, desc->dtype, desc->d_in / b, theta_P, Q_P, ws, stream);
+}
+
+poetx_status poetx_absorb(const poetx_desc* desc, const void* W0, const int32_t* perm_L, const int32_t* perm_R,
+                          void* W0p, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  POETX_TRY(check_ptrs({W0, perm_L, perm_R, W0p}));
+  if (W0 == W0p) return POETX_ERR_INVALID_ARG;
+  return permute_cols(desc->dtype, W0, desc->d_in, W0p, desc->d_in, desc->d_out, desc->d_in, perm_R, perm_L, false,
+                      stream);
+}
+
+poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                           const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P, void* Y,
+                           void* Z_saved, void* workspace, size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
+  if (n_tokens == 0) return POETX_OK;
+  if (desc->mode == POETX_FAST && Z_saved == nullptr) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_MEM && Z_saved != nullptr) return POETX_ERR_INVALID_ARG;
+  POETX_TRY(check_ptrs({X, W0p, perm_L, perm_R, Q_R, Q_P, Y}));
+  if (Z_saved != nullptr && !aligned16(Z_saved)) return POETX_ERR_ALIGNMENT;
+  const FwdPlan f = fwd_plan(desc, n_tokens);
+  POETX_TRY(check_ws(workspace, ws_bytes, f.total));
+  char* ws = static_cast<char*>(workspace);
+  void* Z = desc->mode == POETX_FAST ? Z_saved : ws + f.Z;
+  return forward_chain(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, Z, ws + f.U, ws + f.V, ws + f.Yp, stream);
+}
+
+poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X, const void* W0p,
+                            const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
+                            const float* theta_R, const float* theta_P, const void* Z_saved, void* dX,
+                            float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
+                            poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_FAST && Z_saved == nullptr && n_tokens > 0) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_MEM && Z_saved != nullptr) return POETX_ERR_INVALID_ARG;
+  POETX_TRY(check_ptrs({theta_R, theta_P, grad_theta_R, grad_theta_P}));
+  const int b = desc->b, dt = desc->dtype, nbo = desc->d_out / b, nbi = desc->d_in / b;
+  const size_t P = (size_t)b * (b - 1) / 2;
+  if (n_tokens == 0) {
+    if (cudaMemsetAsync(grad_theta_R, 0, nbo * P * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
+    if (cudaMemsetAsync(grad_theta_P, 0, nbi * P * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
+    return POETX_OK;
+  }
+  POETX_TRY(check_ptrs({dY, X, W0p, perm_L, perm_R, Q_R, Q_P, dX}));
+  if (Z_saved != nullptr && !aligned16(Z_saved)) return POETX_ERR_ALIGNMENT;
+  const BwdPlan w = bwd_plan(desc, n_tokens);
+  POETX_TRY(check_ws(workspace, ws_bytes, w.total));
+  char* ws = static_cast<char*>(workspace);
+  const long n = n_tokens;
+  const int din = desc->d_in, dout = desc->d_out;
+
+  const void* Z = Z_saved;
+  if (desc->mode == POETX_MEM) {
+    // POET-Xmem: recompute U = X[:, pi_R], V = BD_P.U and Z = V.W0'^T from X.
+    POETX_TRY(forward_chain(desc, n, X, W0p, perm_L, perm_R, Q_R, Q_P, nullptr, ws + w.Z, ws + w.U, ws + w.V,
+                            nullptr, stream));
+    Z = ws + w.Z;
+  }
+  // Output side: dY' = dY[:, pi_L]; G_R partials; dZ = BD_R^T-adjoint.
+  POETX_TRY(permute_cols(dt, dY, dout, ws + w.dYp, dout, n, dout, perm_L, nullptr, false, stream));
+  POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, stream));
+  POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
+  // dV = dZ . W0'
+  {
+    GemmDesc g;
+    g.M = (int)n; g.N = din; g.K = dout;
+    g.A = view(ws + w.dZ, n, dout, dout);
+    g.B = view(W0p, dout, din, din); g.b_mn = true;
+    g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM));
+  }
+  // Input side: U = X[:, pi_R] (already there in mem mode); G_P partials; dU; dX[:, pi_R] = dU.
+  if (desc->mode == POETX_FAST)
+    POETX_TRY(permute_cols(dt, X, din, ws + w.U, din, n, din, perm_R, nullptr, false, stream));
+  POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, ws + w.U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
+  POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
+  POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, stream));
+  // CNP adjoint, packed gradients only.
+  POETX_TRY(cnp_bwd_run(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + w.GpR), w.sR,
+                        grad_theta_R, ws + w.cnp, stream));
+  return cnp_bwd_run(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + w.GpP), w.sP, grad_theta_P,
+                     ws + w.cnp, stream);
+}
+
+poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, const void* Q_P,
+                         const int32_t* perm_L_old, const int32_t* perm_R_old, const int32_t* perm_L_new,
+                         const int32_t* perm_R_new, float* theta_R, float* theta_P, void* workspace, size_t ws_bytes,
+                         poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  POETX_TRY(check_ptrs({W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P}));
+  const MergePlan m = merge_plan(desc);
+  POETX_TRY(check_ws(workspace, ws_bytes, m.total));
+  char* ws = static_cast<char*>(workspace);
+  const int dt = desc->dtype, b = desc->b, din = desc->d_in, dout = desc->d_out;
+  // T = W0' . BD_P   (column blocks: T[:, blk z] = W0'[:, blk z] . Q_P,z)
+  {
+    GemmDesc g;
+    g.M = dout; g.N = b; g.K = b; g.batch = din / b;
+    g.A = view(W0p, dout, din, din, 0, b);
+    g.B = view(Q_P, din, b, b, b, 0); g.b_mn = true;
+    g.epi.d1 = ws + m.T; g.epi.d1_dtype = dt; g.epi.ld1 = din; g.epi.zcol1 = b;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_MERGE_GEMM));
+  }
+  // M2 = BD_R . T   (row blocks: M2[blk z, :] = Q_R,z . T[blk z, :])
+  {
+    GemmDesc g;
+    g.M = b; g.N = din; g.K = b; g.batch = dout / b;
+    g.A = view(Q_R, dout, b, b, b, 0);
+    g.B = view(ws + m.T, dout, din, din, b, 0); g.b_mn = true;
+    g.epi.d1 = ws + m.M2; g.epi.d1_dtype = dt; g.epi.ld1 = din; g.epi.zrow1 = b;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_MERGE_GEMM));
+  }
+  // sigma_L = pi_L_old^-1 o pi_L_new, sigma_R likewise; W0'_new[i][j] = M2[sigma_L(i)][sigma_R(j)].
+  int32_t* inv = reinterpret_cast<int32_t*>(ws + m.inv);
+  int32_t* sL = reinterpret_cast<int32_t*>(ws + m.sigL);
+  int32_t* sR = reinterpret_cast<int32_t*>(ws + m.sigR);
+  {
+    LaunchScope ls(POETX_KC_ELEMENTWISE, stream);
+    perm_inverse_kernel<<<ew_grid(dout), 256, 0, stream>>>(perm_L_old, dout, inv);
+  }
+  {
+    LaunchScope ls(POETX_KC_ELEMENTWISE, stream);
+    perm_compose_kernel<<<ew_grid(dout), 256, 0, stream>>>(inv, perm_L_new, dout, sL);
+  }
+  {
+    LaunchScope ls(POETX_KC_ELEMENTWISE, stream);
+    perm_inverse_kernel<<<ew_grid(din), 256, 0, stream>>>(perm_R_old, din, inv);
+  }
+  {
+    LaunchScope ls(POETX_KC_ELEMENTWISE, stream);
+    perm_compose_kernel<<<ew_grid(din), 256, 0, stream>>>(inv, perm_R_new, din, sR);
+  }
+  POETX_TRY(last_launch());
+  POETX_TRY(permute_cols(dt, ws + m.M2, din, W0p, din, dout, din, sR, sL, false, stream));
+  const size_t P = (size_t)b * (b - 1) / 2;
+  if (cudaMemsetAsync(theta_R, 0, (size_t)(dout / b) * P * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
+  if (cudaMemsetAsync(theta_P, 0, (size_t)(din / b) * P * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
+  return POETX_OK;
+}
+
+poetx_status poetx_device_status(int* detail) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return POETX_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return POETX_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return POETX_ERR_CUDA;
+  if (detail) *detail = v;
+  return v ? POETX_ERR_DEVICE_TIMEOUT : POETX_OK;
+}
+
+poetx_status poetx_test_gemm(int dtype, int M, int N, int K, int batch, int splits, const void* a, long long a_rows,
+                             long long a_cols, long long a_ld, long long a_zrow, long long a_zcol, int a_mn,
+                             const void* b, long long b_rows, long long b_cols, long long b_ld, long long b_zrow,
+                             long long b_zcol, int b_mn, void* d, int d_dtype, long long d_ld, long long d_zrow,
+                             long long d_zcol, long long d_split_stride, float alpha, float beta, const float* c,
+                             long long c_ld, long long c_zrow, long long c_zcol, int diag, poetx_stream stream) {
+  if (dtype != F32 && dtype != BF16) return POETX_ERR_INVALID_ARG;
+  if (d_dtype != F32 && d_dtype != BF16) return POETX_ERR_INVALID_ARG;
+  if (d == nullptr) return POETX_ERR_INVALID_ARG;
+  GemmDesc g;
+  g.M = M; g.N = N; g.K = K; g.batch = batch; g.splits = splits;
+  g.A = view(a, a_rows, a_cols, a_ld, a_zrow, a_zcol); g.a_mn = a_mn != 0;
+  g.B = view(b, b_rows, b_cols, b_ld, b_zrow, b_zcol); g.b_mn = b_mn != 0;
+  g.epi.d1 = d; g.epi.d1_dtype = d_dtype; g.epi.ld1 = d_ld; g.epi.zrow1 = d_zrow; g.epi.zcol1 = d_zcol;
+  g.epi.split_stride1 = d_split_stride; g.epi.alpha1 = alpha; g.epi.beta1 = beta; g.epi.diag1 = diag;
+  g.epi.c = c; g.epi.c_dtype = F32; g.epi.ldc = c_ld; g.epi.zrowc = c_zrow; g.epi.zcolc = c_zcol;
+  return run_gemm(dtype, g, stream, POETX_KC_TEST_GEMM);
+}
+
+unsigned long long poetx_launch_count(void) { return prof().launches.load(); }
+
+poetx_status poetx_profile_enable(int on) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (on) {
+    p.recs.clear();
+    p.used = 0;
+  }
+  p.on = on != 0;
+  return POETX_OK;
+}
+
+poetx_status poetx_profile_summary(int* counts, float* total_ms) {
+  if (counts == nullptr || total_ms == nullptr) return POETX_ERR_INVALID_ARG;
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  for (int c = 0; c < POETX_KC_COUNT; ++c) { counts[c] = 0; total_ms[c] = 0.f; }
+  for (auto& r : p.recs) {
+    if (cudaEventSynchronize(r.second.second) != cudaSuccess) return POETX_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.second.first, r.second.second) != cudaSuccess) return POETX_ERR_CUDA;
+    if (r.first >= 0 && r.first < POETX_KC_COUNT) { counts[r.first] += 1; total_ms[r.first] += ms; }
+  }
+  return POETX_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,88 @@
+"""Device buffers of one POET-X layer and the call sequence of one training step.
+
+Plumbing only: torch provides device memory and the stream; every step of the layer runs in
+libpoetx's kernels through the C ABI (see the package __init__).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_backward, poetx_cnp,
+               poetx_desc, poetx_forward, poetx_merge, poetx_workspace_size)
+
+TORCH_DTYPE = {POETX_F32: torch.float32, POETX_BF16: torch.bfloat16}
+
+
+def make_desc(d_in: int, d_out: int, b: int, k: int, dtype: str, mode: str) -> poetx_desc:
+    return poetx_desc(d_in, d_out, b, k, POETX_BF16 if dtype == "bf16" else POETX_F32,
+                      POETX_MEM if mode == "mem" else POETX_FAST)
+
+
+class PoetxLayer:
+    """Holds W0', theta, permutations, Q and scratch of one layer on one device."""
+
+    def __init__(self, desc: poetx_desc, n_tokens: int, device="cuda"):
+        self.desc = desc
+        self.n = int(n_tokens)
+        self.device = torch.device(device)
+        dt = TORCH_DTYPE[desc.dtype]
+        self.dtype = dt
+        b, din, dout = desc.b, desc.d_in, desc.d_out
+        P = b * (b - 1) // 2
+        dev = self.device
+        self.W0p = torch.empty(dout, din, dtype=dt, device=dev)
+        self.theta_R = torch.zeros(dout // b, P, dtype=torch.float32, device=dev)
+        self.theta_P = torch.zeros(din // b, P, dtype=torch.float32, device=dev)
+        self.perm_L = torch.arange(dout, dtype=torch.int32, device=dev)
+        self.perm_R = torch.arange(din, dtype=torch.int32, device=dev)
+        self.Q_R = torch.empty(dout // b, b, b, dtype=dt, device=dev)
+        self.Q_P = torch.empty(din // b, b, b, dtype=dt, device=dev)
+        self.Y = torch.empty(self.n, dout, dtype=dt, device=dev)
+        self.Z = torch.empty(self.n, dout, dtype=dt, device=dev) if desc.mode == POETX_FAST else None
+        self.dX = torch.empty(self.n, din, dtype=dt, device=dev)
+        self.g_R = torch.empty_like(self.theta_R)
+        self.g_P = torch.empty_like(self.theta_P)
+        ws = poetx_workspace_size(desc, self.n)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    # ------------------------------------------------------------------ state upload helpers
+    def to_dev(self, a: np.ndarray, dtype=None) -> torch.Tensor:
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return t.to(device=self.device, dtype=dtype or self.dtype)
+
+    def load_state(self, W0: np.ndarray, theta_R, theta_P, pi_L, pi_R):
+        """Uploads the original-basis W0 and absorbs the two permutations on the device."""
+        self.perm_L.copy_(torch.from_numpy(np.asarray(pi_L, np.int32)))
+        self.perm_R.copy_(torch.from_numpy(np.asarray(pi_R, np.int32)))
+        self.theta_R.copy_(torch.from_numpy(np.asarray(theta_R, np.float32)))
+        self.theta_P.copy_(torch.from_numpy(np.asarray(theta_P, np.float32)))
+        W0_dev = self.to_dev(W0)
+        poetx_absorb(self.desc, W0_dev, self.perm_L, self.perm_R, self.W0p)
+
+    # ------------------------------------------------------------------------- the step
+    def cnp(self):
+        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.ws)
+
+    def forward(self, X: torch.Tensor):
+        poetx_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
+                      self.Z, self.ws)
+        return self.Y
+
+    def backward(self, dY: torch.Tensor, X: torch.Tensor):
+        poetx_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
+                       self.theta_R, self.theta_P, self.Z, self.dX, self.g_R, self.g_P, self.ws)
+        return self.dX, self.g_R, self.g_P
+
+    def step(self, X: torch.Tensor, dY: torch.Tensor):
+        """CNP forward + layer forward + layer backward (incl. the CNP adjoint)."""
+        self.cnp()
+        self.forward(X)
+        self.backward(dY, X)
+
+    def merge(self, pi_L_new: torch.Tensor, pi_R_new: torch.Tensor):
+        """Folds R and P into W0', absorbs the new permutations and resets theta (Q must be current)."""
+        poetx_merge(self.desc, self.W0p, self.Q_R, self.Q_P, self.perm_L, self.perm_R, pi_L_new, pi_R_new,
+                    self.theta_R, self.theta_P, self.ws)
+        self.perm_L.copy_(pi_L_new)
+        self.perm_R.copy_(pi_R_new)

@@ -1,0 +1,99 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, and rejects bad calls
+on the host before launching anything."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import orthogonal_equivalence_cnp_b200 as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+char\s*\*|poetx_status|size_t|unsigned\s+long\s+long)\s+(poetx_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_symbols()
+    assert len(declared) >= 11, declared
+    so = ctypes.CDLL(P.library_path())
+    for name in declared:
+        assert hasattr(so, name), name
+    assert set(declared) <= set(P.exported_symbols())
+
+
+def test_status_strings():
+    for code, name in P.STATUS.items():
+        assert P.poetx_status_string(code) == name
+
+
+def _desc(**kw):
+    base = dict(d_in=256, d_out=256, b=32, k=3, dtype=P.POETX_F32, mode=P.POETX_FAST)
+    base.update(kw)
+    return P.poetx_desc(base["d_in"], base["d_out"], base["b"], base["k"], base["dtype"], base["mode"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(b=48), 2), (dict(b=32, dtype=P.POETX_BF16), 2), (dict(d_in=250), 2), (dict(k=9), 2),
+    (dict(k=-1), 1), (dict(dtype=7), 1), (dict(mode=3), 1), (dict(d_out=0), 1),
+])
+def test_invalid_descriptors_rejected(kw, code):
+    d = _desc(**kw)
+    assert P.poetx_workspace_size(d, 64) == 0
+    L = P.lib()
+    fake = 1 << 20  # aligned, never dereferenced: validation fails first
+    st = L.poetx_cnp(ctypes.byref(d), fake, fake, fake, fake, fake, 1 << 30, None)
+    assert st == code
+
+
+def test_null_misaligned_and_workspace_errors():
+    L = P.lib()
+    d = _desc()
+    ws = P.poetx_workspace_size(d, 64)
+    assert ws > 0
+    A = 1 << 20
+    # NULL output
+    assert L.poetx_forward(ctypes.byref(d), 64, A, A, A, A, A, A, None, A, A, ws, None) == 1
+    # misaligned input
+    assert L.poetx_forward(ctypes.byref(d), 64, A + 4, A, A, A, A, A, A, A, A, ws, None) == 3
+    # workspace too small / missing
+    assert L.poetx_forward(ctypes.byref(d), 64, A, A, A, A, A, A, A, A, A, 1024, None) == 4
+    assert L.poetx_forward(ctypes.byref(d), 64, A, A, A, A, A, A, A, A, None, ws, None) == 4
+    # mode / Z_saved mismatch
+    assert L.poetx_forward(ctypes.byref(d), 64, A, A, A, A, A, A, A, None, A, ws, None) == 1
+    dm = _desc(mode=P.POETX_MEM)
+    assert L.poetx_forward(ctypes.byref(dm), 64, A, A, A, A, A, A, A, A, A, ws, None) == 1
+    # negative token count
+    assert L.poetx_forward(ctypes.byref(d), -1, A, A, A, A, A, A, A, A, A, ws, None) == 1
+    # zero tokens: valid, nothing launched
+    assert L.poetx_forward(ctypes.byref(d), 0, A, A, A, A, A, A, A, A, A, ws, None) == 0
+    # absorb must not alias
+    assert L.poetx_absorb(ctypes.byref(d), A, A, A, A, None) == 1
+    # merge with a NULL permutation
+    assert L.poetx_merge(ctypes.byref(d), A, A, A, None, A, A, A, A, A, A, 1 << 30, None) == 1
+
+
+def test_workspace_grows_with_tokens_and_mem_mode():
+    d = _desc(d_in=4096, d_out=4096, b=256, dtype=P.POETX_BF16)
+    a, b = P.poetx_workspace_size(d, 1024), P.poetx_workspace_size(d, 2048)
+    assert 0 < a < b
+    dm = _desc(d_in=4096, d_out=4096, b=256, dtype=P.POETX_BF16, mode=P.POETX_MEM)
+    assert P.poetx_workspace_size(dm, 2048) > b
+    assert P.poetx_cnp_blocks_workspace_size(d, 10240) > 0
+
+
+def test_gemm_hook_rejects_out_of_range_views():
+    # A view that would read past its array is refused on the host.
+    st = P.lib().poetx_test_gemm(0, 64, 64, 64, 2, 1, 1 << 20, 64, 64, 64, 64, 0, 0,
+                                 1 << 20, 64, 64, 64, 0, 0, 0, 1 << 20, 0, 64, 0, 0, 0,
+                                 1.0, 0.0, None, 0, 0, 0, 0, None)
+    assert st == 1

@@ -376,3 +376,11 @@ def test_planted_mistakes_are_caught():
     ]
     for old, new in mistakes:
         assert not _pins_pass(variant(old, new)), new
+
+
+def test_absorb_equals_permutation_matrix_product():
+    rng = np.random.default_rng(12)
+    W = rng.standard_normal((6, 10))
+    pl, pr = rng.permutation(6), rng.permutation(10)
+    assert np.array_equal(O.absorb(W, pl, pr), O.perm_matrix(pl) @ W @ O.perm_matrix(pr).T)
+    assert np.array_equal(O.unabsorb(O.absorb(W, pl, pr), pl, pr), W)
