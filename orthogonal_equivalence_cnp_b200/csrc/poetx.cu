@@ -335,15 +335,20 @@ size_t cnp_fwd_ws(int b, int k, int dt, long nb) {
   Plan p;
   p.take(blk * 4);                  // S (f32)
   if (dt == BF16) p.take(blk * 2);  // S (bf16 operand)
-  if (k >= 2) { p.take(blk * esize(dt)); p.take(blk * esize(dt)); }  // M_j ping-pong
+  if (k >= 2) {
+    p.take(blk * esize(dt));        // M_j ping-pong
+    p.take(blk * esize(dt));
+    p.take(blk * 4);                // T = S + M_k (f32)
+  }
   return p.total;
 }
 
-// Q = (I + S)(I + S + ... + S^k) by the Horner recursion on M_j = N_j - I:
-//   M_1 = S;  M_j = S + S.M_{j-1};  Q = I + S + S.M_k  (k >= 1);  Q = I + S (k = 0).
-// Keeping M_j = N_j - I (small) instead of N_j keeps the bf16 intermediates accurate; the
-// exact I + S part is added in fp32 in the epilogue (replication review, "Summary": the fused
-// CNP reuses the lower powers across terms).
+// Q = (I + S)(I + S + ... + S^k) by the Horner recursion N_1 = I + S, N_j = I + S.N_{j-1},
+// Q = N_k + S.N_k, carried on M_j = N_j - I (small, so bf16 intermediates stay accurate):
+//   M_1 = S;  M_j = S + S.M_{j-1};  Q = I + (S + M_k) + S.M_k.
+// The product that yields M_k also writes T = S + M_k = 2S + S.M_{k-1} in fp32, and the exact
+// I + T part of Q is added in fp32 in the last epilogue (replication review, "Summary": the
+// fused CNP reuses the lower powers across terms).
 poetx_status cnp_fwd_run(int b, int k, int dt, long nb, const float* theta, void* Q, char* ws, cudaStream_t st) {
   if (nb == 0) return POETX_OK;
   if (k == 0) return unpack(theta, nb, b, Q, dt, b, nullptr, dt, 0, nullptr, true, st);
@@ -352,23 +357,38 @@ poetx_status cnp_fwd_run(int b, int k, int dt, long nb, const float* theta, void
   float* S32 = reinterpret_cast<float*>(ws + p.take(blk * 4));
   void* Sop = dt == BF16 ? static_cast<void*>(ws + p.take(blk * 2)) : static_cast<void*>(S32);
   void* Mbuf[2] = {nullptr, nullptr};
-  if (k >= 2) { Mbuf[0] = ws + p.take(blk * esize(dt)); Mbuf[1] = ws + p.take(blk * esize(dt)); }
+  float* T32 = nullptr;
+  if (k >= 2) {
+    Mbuf[0] = ws + p.take(blk * esize(dt));
+    Mbuf[1] = ws + p.take(blk * esize(dt));
+    T32 = reinterpret_cast<float*>(ws + p.take(blk * 4));
+  }
   POETX_TRY(unpack(theta, nb, b, dt == BF16 ? Sop : nullptr, dt, b, nullptr, dt, 0, S32, false, st));
-  const void* Mprev = Sop;
-  for (int j = 2; j <= k + 1; ++j) {
-    const bool last = (j == k + 1);
-    void* dst = last ? Q : Mbuf[j & 1];
+  auto chain = [&](const void* Mprev) {
     GemmDesc g;
     g.M = b; g.N = b; g.K = b; g.batch = (int)nb;
     g.A = view(Sop, nb * b, b, b, b, 0);
     g.B = view(Mprev, nb * b, b, b, b, 0); g.b_mn = true;
-    g.epi.d1 = dst; g.epi.d1_dtype = dt; g.epi.ld1 = b; g.epi.zrow1 = b;
-    g.epi.alpha1 = 1.f; g.epi.beta1 = 1.f; g.epi.diag1 = last ? 1 : 0;
-    g.epi.c = S32; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
+    g.epi.d1_dtype = dt; g.epi.ld1 = b; g.epi.zrow1 = b;
+    g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
+    return g;
+  };
+  const void* Mprev = Sop;  // M_1 = S
+  for (int j = 2; j <= k; ++j) {
+    GemmDesc g = chain(Mprev);
+    g.epi.d1 = Mbuf[j & 1];
+    g.epi.alpha1 = 1.f; g.epi.beta1 = 1.f; g.epi.c = S32;   // M_j = S.M_{j-1} + S
+    if (j == k) {                                            // T = S + M_k = S.M_{k-1} + 2S
+      g.epi.d2 = T32; g.epi.ld2 = b; g.epi.zrow2 = b; g.epi.alpha2 = 1.f; g.epi.beta2 = 2.f;
+    }
     POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
-    Mprev = dst;
+    Mprev = Mbuf[j & 1];
   }
-  return POETX_OK;
+  GemmDesc g = chain(Mprev);                                 // Q = I + T + S.M_k
+  g.epi.d1 = Q; g.epi.alpha1 = 1.f; g.epi.diag1 = 1;
+  if (k == 1) { g.epi.c = S32; g.epi.beta1 = 2.f; }          // T = S + M_1 = 2S
+  else { g.epi.c = T32; g.epi.beta1 = 1.f; }
+  return run_gemm(dt, g, st, POETX_KC_CNP_GEMM);
 }
 
 // ------------------------------------------------------------------------- CNP backward
