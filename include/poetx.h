@@ -100,6 +100,25 @@ size_t poetx_cnp_blocks_workspace_size(const poetx_desc* desc, int n_blocks);
 poetx_status poetx_cnp_blocks(const poetx_desc* desc, int n_blocks, const float* theta, void* Q,
                               void* workspace, size_t ws_bytes, poetx_stream stream);
 
+/* Allocation-free variant of poetx_cnp_blocks.  The paper has no counterpart: this entry point
+ * exists for callers that cannot supply device scratch, such as a plugin inside a host
+ * framework that owns all device memory and offers it no allocator, or a latency-critical loop
+ * that must not call cudaMalloc.  Its scratch is a fixed array of POETX_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) compiled into the library; every GPU that loads the library holds it until the
+ * process exits.  The call itself allocates nothing.
+ *   theta float32 [n_blocks, b(b-1)/2] (in); Q dtype [n_blocks, b, b] (out), caller-owned.
+ * Limit: poetx_cnp_blocks_workspace_size(desc, n_blocks) must not exceed 32 MiB (e.g. bf16,
+ * b = 256, k = 3: at most 36 blocks; b = 128: 146; b = 512: 9); larger requests return
+ * POETX_ERR_WORKSPACE and launch nothing.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All calls on a device
+ * share the one array: calls that may run at the same time on the GPU (unordered streams)
+ * race on it and must be serialised by the caller.  No part of the array needs clearing: each
+ * call writes all the scratch it reads. */
+#define POETX_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+poetx_status poetx_cnp_blocks_noalloc(const poetx_desc* desc, int n_blocks, const float* theta,
+                                      void* Q, poetx_stream stream);
+
 /* Absorb two of the four permutations into the base weight in advance (replication review,
  * "Summary": permutation reduction): W0'[i][j] = W0[perm_L[i]][perm_R[j]].
  *   W0 dtype [d_out, d_in] (in); perm_L int32 [d_out], perm_R int32 [d_in] bijections (in);

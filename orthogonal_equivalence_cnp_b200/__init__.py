@@ -17,6 +17,7 @@ __all__ = [
     "poetx_cnp_blocks_workspace_size", "poetx_absorb", "poetx_forward", "poetx_backward",
     "poetx_merge", "poetx_status_string", "poetx_device_status", "poetx_test_gemm",
     "poetx_launch_count", "poetx_profile_enable", "poetx_profile_summary", "KERNEL_CLASSES",
+    "poetx_cnp_blocks_noalloc",
 ]
 
 POETX_F32, POETX_BF16 = 0, 1
@@ -61,6 +62,7 @@ _SIGNATURES = {
     "poetx_cnp_blocks_workspace_size": (_SZ, [_D, _I]),
     "poetx_cnp": (_I, [_D, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_cnp_blocks": (_I, [_D, _I, _P, _P, _P, _SZ, _P]),
+    "poetx_cnp_blocks_noalloc": (_I, [_D, _I, _P, _P, _P]),
     "poetx_absorb": (_I, [_D, _P, _P, _P, _P, _P]),
     "poetx_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -214,3 +216,9 @@ def poetx_profile_summary():
     ms = (ctypes.c_float * n)()
     _check(lib().poetx_profile_summary(counts, ms), "poetx_profile_summary")
     return {KERNEL_CLASSES[i]: (counts[i], ms[i]) for i in range(n)}
+
+
+def poetx_cnp_blocks_noalloc(desc, n_blocks, theta, Q, stream=None):
+    """CNP forward that takes no workspace (built-in 32 MiB device scratch; see include/poetx.h)."""
+    _check(lib().poetx_cnp_blocks_noalloc(ctypes.byref(desc), n_blocks, _ptr(theta), _ptr(Q), _stream(stream)),
+           "poetx_cnp_blocks_noalloc")

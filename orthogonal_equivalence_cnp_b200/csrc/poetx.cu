@@ -582,6 +582,37 @@ poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const voi
   return permute_cols(dt, Yp, d->d_out, Y, d->d_out, n, d->d_out, pL, nullptr, true, st);
 }
 
+// ------------------------------------------------------------ allocation-free CNP forward
+// Built-in scratch for poetx_cnp_blocks_noalloc.  Some callers cannot hand the library a
+// workspace: a plugin living inside a host framework that owns every device allocation and
+// exposes no allocator to it, or a latency-critical loop that must never pay for cudaMalloc
+// (which can synchronise the device).  For them the CNP forward runs out of this fixed array,
+// which every GPU that loads the library keeps until the process exits.  All calls on a device
+// share it, so calls that overlap in time on the GPU (different streams, no ordering) race on
+// it.  Nothing in it has to start at zero: the CNP forward writes every scratch element it
+// reads in the same call.
+constexpr size_t kNoAllocScratchBytes = POETX_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_cnp_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the built-in scratch on the current device.  In host code the array's
+// name is only a host-side stand-in; the real address comes from cudaGetSymbolAddress, looked
+// up once per device (with that device current) and cached.
+poetx_status noalloc_scratch(char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return POETX_ERR_CUDA;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_cnp_noalloc_scratch) != cudaSuccess || p == nullptr) return POETX_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<char*>(g_noalloc_addr[dev]);
+  return POETX_OK;
+}
+
 }  // namespace
 
 // =============================================================================== C ABI
@@ -828,6 +859,18 @@ poetx_status poetx_profile_summary(int* counts, float* total_ms) {
     if (r.first >= 0 && r.first < POETX_KC_COUNT) { counts[r.first] += 1; total_ms[r.first] += ms; }
   }
   return POETX_OK;
+}
+
+poetx_status poetx_cnp_blocks_noalloc(const poetx_desc* desc, int n_blocks, const float* theta, void* Q,
+                                      poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_blocks < 0) return POETX_ERR_INVALID_ARG;
+  if (n_blocks == 0) return POETX_OK;
+  POETX_TRY(check_ptrs({theta, Q}));
+  if (cnp_fwd_ws(desc->b, desc->k, desc->dtype, n_blocks) > kNoAllocScratchBytes) return POETX_ERR_WORKSPACE;
+  char* ws = nullptr;
+  POETX_TRY(noalloc_scratch(&ws));
+  return cnp_fwd_run(desc->b, desc->k, desc->dtype, n_blocks, theta, Q, ws, stream);
 }
 
 }  // extern "C"
