@@ -108,7 +108,7 @@ poetx_status poetx_cnp_blocks(const poetx_desc* desc, int n_blocks, const float*
  * process exits.  The call itself allocates nothing.
  *   theta float32 [n_blocks, b(b-1)/2] (in); Q dtype [n_blocks, b, b] (out), caller-owned.
  * Limit: poetx_cnp_blocks_workspace_size(desc, n_blocks) must not exceed 32 MiB (e.g. bf16,
- * b = 256, k = 3: at most 36 blocks; b = 128: 146; b = 512: 9); larger requests return
+ * k = 3: at most 85 blocks of b = 256, 341 of b = 128, 9 of b = 512); larger requests return
  * POETX_ERR_WORKSPACE and launch nothing.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
  * that device current; make that first call before any stream capture.  All calls on a device

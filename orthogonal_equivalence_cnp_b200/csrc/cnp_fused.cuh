@@ -1,0 +1,322 @@
+// Fused Cayley–Neumann kernels: the whole CNP forward (or its adjoint) of every block in one
+// launch (replication review of POET-X, "Summary": a fused kernel for the Cayley–Neumann
+// series that reuses the lower powers; "Reproducibility & code": forward and grad-Q kernels).
+//
+// Each b x b block (b <= 256) is owned by one thread-block cluster of (b/BN) x ceil(b/128) CTAs;
+// CTA (n-tile, m-tile) owns the same 128 x BN tile of every intermediate of its block.  The
+// kernel runs a short program of stages:
+//   GEMM stage  — tile of D = A . B^T on tcgen05 (A: S or the stacked adjoint terms, K-major;
+//                 B: the previous power / adjoint term, streamed from L2 by TMA);
+//   UNPACK      — packed theta -> S;
+//   REDUCE      — split-K partial sum of G = dL/dQ, fused with UNPACK;
+//   PACK        — g[p(i,j)] = G_S[i][j] - G_S[j][i].
+// Per-row state that only the owning CTA reads back (S, T = S + M_k, G, the running sum E)
+// stays in TMEM beside the accumulator: four regions of BN fp32 columns (ACC, R1, R2, R3), one
+// TMEM lane per tile row, read and written by the thread that owns the row.  Only operands
+// that peer CTAs consume (bf16 S, M_j, adjoint terms), the f32 G_S needed by PACK and the final
+// outputs go through global memory.  Between stages each CTA publishes its tile (stores, proxy
+// fence for the peers' TMA reads) and meets the others at a cluster barrier; every CTA executes
+// every barrier of the program, whatever happens to its bounded waits.
+#pragma once
+
+#include "common.cuh"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+#include "sm100.cuh"
+
+namespace poetx {
+
+constexpr int CNP_MAX_STAGES = 20;
+constexpr int CNP_THREADS = 256;  // 8 warps: warp w owns TMEM lane quarter w%4, column half w/4
+enum CnpStageKind : int { CNP_GEMM = 0, CNP_UNPACK = 1, CNP_REDUCE_UNPACK = 2, CNP_PACK = 3 };
+enum CnpReg : int { CNP_NONE = -1, CNP_ACC = 0, CNP_R1 = 1, CNP_R2 = 2, CNP_R3 = 3 };
+enum : int { KID_CNP_FUSED = 2 };
+
+// Stage description shared by the segments (register-form epilogue):
+//   out1 = alpha1*acc + beta1*REG[c_reg] (+ I if diag1)  -> global g1 (g1_dtype) and/or REG[r1]
+//   out2 = alpha2*acc + beta2*REG[c_reg] (+ REG[r2] if accum2) -> REG[r2]
+struct CnpStageDesc {
+  int kind;
+  int b_mn;
+  int c_reg;
+  float alpha1, beta1;
+  int diag1;
+  int r1;
+  int g1_dtype;  // BF16 or F32 (g1 may be null per segment)
+  int r2;
+  float alpha2, beta2;
+  int accum2;
+};
+
+struct CnpSegStage {
+  CUtensorMap tmA;  // K-major A operand map (box 64 x 128)
+  CUtensorMap tmB;  // B operand map (K-major box 64 x BN, or MN-major box 64 x 64)
+  int K;
+  int a_zrow, b_zrow, b_zcol;
+  void* g1;         // global out1: element (z*b+i, j) at g1[(z*b+i)*g1_ld + j]
+  long g1_ld;
+};
+
+struct CnpSegment {
+  int nb;
+  const float* theta;  // [nb, b(b-1)/2]
+  // UNPACK: S -> R1 (unless no_sreg), two optional bf16 global copies, optional identity.
+  int no_sreg;
+  void* Sb0;
+  long ld0;
+  void* Sb1;
+  long ld1;
+  int add_identity;
+  // REDUCE: G = sum of split-K partials -> R2, optional bf16 copy Gb, optional f32 copy G32.
+  const float* part;  // [splits][nb*b][b]
+  int splits;
+  void* Gb;
+  long ldg;
+  float* G32;
+  // PACK
+  const float* GS;    // [nb*b][b] f32
+  float* grad;        // [nb, b(b-1)/2]
+};
+
+struct CnpProgram {
+  int b;
+  int nstages;
+  int nseg;
+  CnpStageDesc st[CNP_MAX_STAGES];
+  CnpSegment seg[2];
+  CnpSegStage g[CNP_MAX_STAGES][2];
+};
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __grid_constant__ CnpProgram prog) {
+  constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
+  constexpr uint32_t B_BYTES = BN * TC_BK * 2;
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t TMEM_COLS = 4 * BN;  // ACC, R1, R2, R3
+  constexpr int HALF = BN / 2;            // columns per warp (two warps share a lane quarter)
+  static_assert(HALF % 32 == 0, "tile half must be whole 32-column chunks");
+  using namespace sm100;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  const uint32_t smem0 = smem_u32(smem);
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int b = prog.b;
+  const int zg = blockIdx.z;
+  const int seg = (prog.nseg > 1 && zg >= prog.seg[0].nb) ? 1 : 0;
+  const int z = seg ? zg - prog.seg[0].nb : zg;
+  const CnpSegment& S = prog.seg[seg];
+  const int m0 = blockIdx.y * TC_BM, n0 = blockIdx.x * BN;
+  const long P = (long)b * (b - 1) / 2;
+  const float* th = S.theta + (long)z * P;
+  const int i = m0 + quarter * 32 + lane;  // the tile row this thread owns
+  const bool row_ok = i < b;
+  const long grow = (long)z * b + i;       // row in the [nb*b, *] scratch arrays
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(accum_bar, 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem0 = *tmem_holder;
+  const uint32_t tlane = tmem0 + ((uint32_t)(quarter * 32) << 16);
+  auto treg = [&](int reg, int col) { return tlane + (uint32_t)(reg * BN + col); };
+
+  uint32_t it = 0;
+  uint32_t acc_phase = 0;
+
+  for (int s = 0; s < prog.nstages; ++s) {
+    const CnpStageDesc& D = prog.st[s];
+    bool wrote_global = false, wrote_tmem = false;
+    if (D.kind == CNP_GEMM) {
+      const CnpSegStage& G = prog.g[s][seg];
+      const bool b_mn = D.b_mn != 0;
+      const int nkt = (G.K + TC_BK - 1) / TC_BK;
+      const uint32_t idesc = idesc_bf16_f32(TC_BM, BN, false, b_mn);
+      if (warp == 0 && lane == 0) {
+        for (int k = 0; k < nkt; ++k) {
+          const uint32_t q = it + k;
+          const int stg = q % STAGES;
+          const uint32_t ph = (q / STAGES) & 1u;
+          if (!mbar_wait(empty_bar(stg), ph ^ 1u, KID_CNP_FUSED, 1)) break;
+          mbar_arrive_expect_tx(full_bar(stg), STAGE_BYTES);
+          const int k0 = k * TC_BK;
+          const uint32_t sa = smem0 + stg * STAGE_BYTES, sb = sa + A_BYTES;
+          tma_load_2d(sa, &G.tmA, full_bar(stg), k0, z * G.a_zrow + m0);
+          if (!b_mn) {
+            tma_load_2d(sb, &G.tmB, full_bar(stg), z * G.b_zcol + k0, z * G.b_zrow + n0);
+          } else {
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h)
+              tma_load_2d(sb + h * 8192, &G.tmB, full_bar(stg), z * G.b_zcol + n0 + 64 * h, z * G.b_zrow + k0);
+          }
+        }
+      } else if (warp == 1 && lane == 0) {
+        for (int k = 0; k < nkt; ++k) {
+          const uint32_t q = it + k;
+          const int stg = q % STAGES;
+          const uint32_t ph = (q / STAGES) & 1u;
+          if (!mbar_wait(full_bar(stg), ph, KID_CNP_FUSED, 2)) break;
+          tc_fence_after();
+          const uint32_t sa = smem0 + stg * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = b_mn ? smem_desc_sw128(sb + kk * 2048, 8192, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            mma_bf16(tmem0, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(empty_bar(stg));
+        }
+        mma_commit(accum_bar);
+      }
+      __syncwarp();
+      it += nkt;
+      bool ok = mbar_wait(accum_bar, acc_phase, KID_CNP_FUSED, 3);
+      acc_phase ^= 1u;
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      if (ok) {
+#pragma unroll 1
+        for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
+          uint32_t ra[32], rc[32], re[32];
+          tmem_ld_32x32b_x32(treg(CNP_ACC, c), ra);
+          if (D.c_reg >= 0) tmem_ld_32x32b_x32(treg(D.c_reg, c), rc);
+          if (D.r2 >= 0 && D.accum2) tmem_ld_32x32b_x32(treg(D.r2, c), re);
+          tmem_wait_ld();
+          const int n = n0 + c;
+          if (D.r2 >= 0) {  // out2 first, in place in re (it needs acc and the addend only)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              float v = D.alpha2 * __uint_as_float(ra[j]);
+              if (D.c_reg >= 0) v += D.beta2 * __uint_as_float(rc[j]);
+              if (D.accum2) v += __uint_as_float(re[j]);
+              re[j] = __float_as_uint(v);
+            }
+            tmem_st_32x32b_x32(treg(D.r2, c), re);
+            wrote_tmem = true;
+          }
+          float o1[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float v = D.alpha1 * __uint_as_float(ra[j]);
+            if (D.c_reg >= 0) v += D.beta1 * __uint_as_float(rc[j]);
+            if (D.diag1 && i == n + j) v += 1.f;
+            o1[j] = v;
+          }
+          if (D.r1 >= 0) {
+            tmem_st_32x32b_x32(treg(D.r1, c), reinterpret_cast<const uint32_t (&)[32]>(o1));
+            wrote_tmem = true;
+          }
+          if (G.g1 != nullptr && row_ok) {
+            store32(G.g1, grow * G.g1_ld + n, D.g1_dtype, o1);
+            wrote_global = true;
+          }
+        }
+      }
+    } else if (D.kind == CNP_UNPACK || D.kind == CNP_REDUCE_UNPACK) {
+      const long sstride = (long)S.nb * b * b;
+#pragma unroll 1
+      for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
+        const int n = n0 + c;
+        // S[i][n..n+31]: above the diagonal a contiguous run of theta's row i; below it,
+        // theta[p(j, i)] for consecutive rows i of the warp, i.e. coalesced across lanes.
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int jj = n + j;
+          float x = 0.f;
+          if (row_ok) {
+            if (i < jj) x = __ldg(th + packed_pos(i, jj, b));
+            else if (i > jj) x = -__ldg(th + packed_pos(jj, i, b));
+            else if (S.add_identity) x = 1.f;
+          }
+          v[j] = x;
+        }
+        float gsum[32];
+        if (D.kind == CNP_REDUCE_UNPACK) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) gsum[j] = 0.f;
+          if (row_ok)
+            for (int sp = 0; sp < S.splits; ++sp) {
+              float t[32];
+              load32(S.part + sp * sstride, grow * b + n, F32, t);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) gsum[j] += t[j];
+            }
+        }
+        if (!S.no_sreg) {
+          uint32_t w[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+          tmem_st_32x32b_x32(treg(CNP_R1, c), w);
+          wrote_tmem = true;
+        }
+        if (row_ok) {
+          if (S.Sb0) store32(S.Sb0, grow * S.ld0 + n, BF16, v);
+          if (S.Sb1) store32(S.Sb1, grow * S.ld1 + n, BF16, v);
+          wrote_global = true;
+        }
+        if (D.kind == CNP_REDUCE_UNPACK) {
+          uint32_t w[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(gsum[j]);
+          tmem_st_32x32b_x32(treg(CNP_R2, c), w);
+          wrote_tmem = true;
+          if (row_ok) {
+            if (S.Gb) store32(S.Gb, grow * S.ldg + n, BF16, gsum);
+            if (S.G32) store32(S.G32, grow * b + n, F32, gsum);
+          }
+        }
+      }
+    } else if (D.kind == CNP_PACK) {
+#pragma unroll 1
+      for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
+        const int n = n0 + c;
+        if (!row_ok || n + 31 <= i) continue;
+        float a[32], t[32];
+        load32(S.GS, grow * b + n, F32, a);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) t[j] = (i < n + j) ? S.GS[((long)z * b + n + j) * b + i] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (i < n + j) S.grad[(long)z * P + packed_pos(i, n + j, b)] = a[j] - t[j];
+      }
+    }
+    if (wrote_tmem) tmem_wait_st();
+    if (wrote_global) fence_proxy_async_global();
+    tc_fence_before();
+    cluster_sync_all();
+    fence_proxy_async_global();  // the next stage's TMA reads see the peers' generic-proxy writes
+    tc_fence_after();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem0, TMEM_COLS);
+}
+
+}  // namespace poetx

@@ -15,10 +15,14 @@ __host__ __device__ __forceinline__ long packed_pos(int i, int j, int b) {
 // (replication review of POET-X, "Summary": permutations applied by index, never as a matmul;
 // Table 1 of the paper measures such a kernel).  A block stages `rb` whole rows in shared
 // memory with 16-byte coalesced loads, permutes inside shared memory and writes 16-byte
-// coalesced stores, so HBM sees one read and one write of each row.
+// coalesced stores, so HBM sees one read and one write of each element.  Each thread keeps
+// PERM_VPT independent 16-byte loads in flight (registers first, then shared memory), which is
+// what it takes to cover HBM latency at ~16 resident warps per SM.
 //   gather (scatter == 0): out[r][j] = in[rowmap ? rowmap[r] : r][colmap[j]]
 //   scatter (scatter == 1): out[r][colmap[j]] = in[r][j]
-// Requires cols % (16 / sizeof(T)) == 0, 16-byte aligned rows.
+// Requires cols % (16 / sizeof(T)) == 0 and 16-byte aligned rows.
+constexpr int PERM_VPT = 8;
+
 template <typename T>
 __global__ void __launch_bounds__(256)
     permute_cols_kernel(const T* __restrict__ in, long ld_in, T* __restrict__ out, long ld_out, long rows,
@@ -28,38 +32,62 @@ __global__ void __launch_bounds__(256)
   T* buf = reinterpret_cast<T*>(smem_perm);
   constexpr int VEC = 16 / sizeof(T);
   const int nvec = cols / VEC;
+  const int nthr = blockDim.x;
   for (long r0 = (long)blockIdx.x * rb; r0 < rows; r0 += (long)gridDim.x * rb) {
     const int nr = (int)min((long)rb, rows - r0);
     const int total = nr * nvec;
-    if (!scatter) {
-      for (int t = threadIdx.x; t < total; t += blockDim.x) {
-        const int rr = t / nvec, v = t - rr * nvec;
-        const long rin = rowmap ? (long)__ldg(rowmap + r0 + rr) : r0 + rr;
-        reinterpret_cast<uint4*>(buf + (long)rr * cols)[v] = __ldg(reinterpret_cast<const uint4*>(in + rin * ld_in) + v);
+    // Phase 1: rows -> registers -> shared memory (gather: as is; scatter: permuted).
+    for (int base = threadIdx.x; base < total; base += nthr * PERM_VPT) {
+      uint4 v[PERM_VPT];
+#pragma unroll
+      for (int u = 0; u < PERM_VPT; ++u) {
+        const int t = base + u * nthr;
+        if (t < total) {
+          const int rr = t / nvec, c = t - rr * nvec;
+          const long rin = (!scatter && rowmap) ? (long)__ldg(rowmap + r0 + rr) : r0 + rr;
+          v[u] = __ldg(reinterpret_cast<const uint4*>(in + rin * ld_in) + c);
+        }
       }
-      __syncthreads();
-      for (int t = threadIdx.x; t < total; t += blockDim.x) {
-        const int rr = t / nvec, v = t - rr * nvec;
-        const T* srow = buf + (long)rr * cols;
+#pragma unroll
+      for (int u = 0; u < PERM_VPT; ++u) {
+        const int t = base + u * nthr;
+        if (t < total) {
+          const int rr = t / nvec, c = t - rr * nvec;
+          T* row = buf + (long)rr * cols;
+          if (!scatter) {
+            reinterpret_cast<uint4*>(row)[c] = v[u];
+          } else {
+            const T* vals = reinterpret_cast<const T*>(&v[u]);
+            int idx[VEC];
+#pragma unroll
+            for (int q = 0; q < VEC; q += 4) {
+              const int4 m4 = __ldg(reinterpret_cast<const int4*>(colmap + c * VEC + q));
+              idx[q] = m4.x; idx[q + 1] = m4.y; idx[q + 2] = m4.z; idx[q + 3] = m4.w;
+            }
+#pragma unroll
+            for (int q = 0; q < VEC; ++q) row[idx[q]] = vals[q];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // Phase 2: shared memory -> 16-byte coalesced stores (gather: permuted read).
+    for (int t = threadIdx.x; t < total; t += nthr) {
+      const int rr = t / nvec, c = t - rr * nvec;
+      const T* row = buf + (long)rr * cols;
+      uint4 o;
+      if (!scatter) {
         T vals[VEC];
 #pragma unroll
-        for (int q = 0; q < VEC; ++q) vals[q] = srow[__ldg(colmap + v * VEC + q)];
-        reinterpret_cast<uint4*>(out + (r0 + rr) * ld_out)[v] = *reinterpret_cast<const uint4*>(vals);
+        for (int q = 0; q < VEC; q += 4) {
+          const int4 m4 = __ldg(reinterpret_cast<const int4*>(colmap + c * VEC + q));
+          vals[q] = row[m4.x]; vals[q + 1] = row[m4.y]; vals[q + 2] = row[m4.z]; vals[q + 3] = row[m4.w];
+        }
+        o = *reinterpret_cast<const uint4*>(vals);
+      } else {
+        o = reinterpret_cast<const uint4*>(row)[c];
       }
-    } else {
-      for (int t = threadIdx.x; t < total; t += blockDim.x) {
-        const int rr = t / nvec, v = t - rr * nvec;
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(in + (r0 + rr) * ld_in) + v);
-        const T* vals = reinterpret_cast<const T*>(&u);
-        T* drow = buf + (long)rr * cols;
-#pragma unroll
-        for (int q = 0; q < VEC; ++q) drow[__ldg(colmap + v * VEC + q)] = vals[q];
-      }
-      __syncthreads();
-      for (int t = threadIdx.x; t < total; t += blockDim.x) {
-        const int rr = t / nvec, v = t - rr * nvec;
-        reinterpret_cast<uint4*>(out + (r0 + rr) * ld_out)[v] = reinterpret_cast<const uint4*>(buf + (long)rr * cols)[v];
-      }
+      reinterpret_cast<uint4*>(out + (r0 + rr) * ld_out)[c] = o;
     }
     __syncthreads();
   }

@@ -99,12 +99,16 @@ __device__ __forceinline__ void store32(void* base, long off, int dt, const floa
   }
 }
 
-// Applies the epilogue to 32 consecutive columns n..n+31 of row m (batch z, split `split`).
-__device__ __forceinline__ void epilogue32(const Epilogue& e, int z, int split, int m, int n,
-                                           const float (&acc)[32]) {
-  float cv[32];
+// Loads the 32 addend values of row m, columns n..n+31 (batch z).
+__device__ __forceinline__ void epilogue_load_c(const Epilogue& e, int z, int m, int n, float (&cv)[32]) {
+  if (e.c != nullptr) load32(e.c, ((long)z * e.zrowc + m) * e.ldc + (long)z * e.zcolc + n, e.c_dtype, cv);
+}
+
+// Applies the epilogue to 32 consecutive columns n..n+31 of row m (batch z, split `split`),
+// with the addend values already in cv.
+__device__ __forceinline__ void epilogue32c(const Epilogue& e, int z, int split, int m, int n,
+                                            const float (&acc)[32], const float (&cv)[32]) {
   const bool has_c = e.c != nullptr;
-  if (has_c) load32(e.c, (long)z * e.zrowc * e.ldc + (long)m * e.ldc + (long)z * e.zcolc + n, e.c_dtype, cv);
   if (e.d1 != nullptr) {
     float o[32];
 #pragma unroll
@@ -128,6 +132,35 @@ __device__ __forceinline__ void epilogue32(const Epilogue& e, int z, int split, 
       o[j] = e.accum2 ? o[j] + v : v;
     }
     store32(e.d2, off, F32, o);
+  }
+}
+
+__device__ __forceinline__ void epilogue32(const Epilogue& e, int z, int split, int m, int n,
+                                           const float (&acc)[32]) {
+  float cv[32];
+  epilogue_load_c(e, z, m, n, cv);
+  epilogue32c(e, z, split, m, n, acc, cv);
+}
+
+// Drains a BN-column TMEM accumulator (this thread's lane = tile row m) through the epilogue,
+// loading the addend of the next 32-column chunk before storing the current one.
+template <int BN>
+__device__ __forceinline__ void drain_tile(uint32_t taddr, const Epilogue& e, int z, int split, int m, bool row_ok,
+                                           int n0, bool zero_acc) {
+  float cv[32], cn[32];
+  if (row_ok) epilogue_load_c(e, z, m, n0, cv);
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t r[32];
+    sm100::tmem_ld_32x32b_x32(taddr + (uint32_t)c, r);
+    sm100::tmem_wait_ld();
+    if (row_ok && c + 32 < BN) epilogue_load_c(e, z, m, n0 + c + 32, cn);
+    float acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = zero_acc ? 0.f : __uint_as_float(r[j]);
+    if (row_ok) epilogue32c(e, z, split, m, n0 + c, acc, cv);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) cv[j] = cn[j];
   }
 }
 
@@ -168,7 +201,7 @@ __host__ __device__ constexpr size_t tc_smem_bytes() {
 // epilogue.  Every wait is bounded (kWaitLimitNs); on a timeout the CTA records the error,
 // skips the rest of its work and still releases its TMEM.
 template <int BN, int STAGES, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128)
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const TcArgs args) {
   constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
@@ -264,16 +297,7 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   if (ok) {
     const int m = m0 + warp * 32 + lane;
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, r);
-      tmem_wait_ld();
-      float acc[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = nkt > 0 ? __uint_as_float(r[j]) : 0.f;
-      if (m < args.M) epilogue32(args.epi, z, split, m, n0 + c, acc);
-    }
+    drain_tile<BN>(tmem_d + ((uint32_t)(warp * 32) << 16), args.epi, z, split, m, m < args.M, n0, nkt == 0);
   }
   tc_fence_before();
   __syncthreads();

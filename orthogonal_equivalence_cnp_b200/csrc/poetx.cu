@@ -15,6 +15,7 @@
 #include "elementwise.cuh"
 #include "gemm.cuh"
 #include "sm100.cuh"
+#include "cnp_fused.cuh"
 
 using namespace poetx;
 
@@ -210,9 +211,19 @@ poetx_status launch_tc_major(const GemmDesc& g, cudaStream_t st, int cls) {
 poetx_status run_gemm(int dt, const GemmDesc& g, cudaStream_t st, int cls) {
   POETX_TRY(check_gemm(g, dt));
   if (dt == BF16) {
-    if (g.N % 256 == 0) return launch_tc_major<256, 4>(g, st, cls);
-    if (g.N % 128 == 0) return launch_tc_major<128, 6>(g, st, cls);
-    return launch_tc_major<64, 8>(g, st, cls);
+    // Long K (>= 16 k-tiles per CTA): deep ring, one CTA per SM, widest tile.  Short K: a
+    // 96 KiB ring so two CTAs share an SM (one's epilogue overlaps the other's loads), and the
+    // widest tile that still gives at least two CTAs per SM.
+    const long kt = ((long)(g.K + TC_BK - 1) / TC_BK) / g.splits;
+    const long base = (long)((g.M + TC_BM - 1) / TC_BM) * g.batch * g.splits;
+    if (kt >= 16) {
+      if (g.N % 256 == 0) return launch_tc_major<256, 4>(g, st, cls);
+      if (g.N % 128 == 0) return launch_tc_major<128, 6>(g, st, cls);
+      return launch_tc_major<64, 8>(g, st, cls);
+    }
+    if (g.N % 256 == 0 && base * (g.N / 256) >= 2 * kNumSms) return launch_tc_major<256, 2>(g, st, cls);
+    if (g.N % 128 == 0 && base * (g.N / 128) >= 2 * kNumSms) return launch_tc_major<128, 3>(g, st, cls);
+    return launch_tc_major<64, 4>(g, st, cls);
   }
   SimtArgs p;
   p.M = g.M; p.N = g.N; p.K = g.K; p.splits = g.splits;
@@ -329,7 +340,7 @@ poetx_status block_grads(int dt, long n, int d, int b, const void* lhs, const vo
 }
 
 // ------------------------------------------------------------------------- CNP forward
-size_t cnp_fwd_ws(int b, int k, int dt, long nb) {
+size_t cnp_fwd_generic_ws(int b, int k, int dt, long nb) {
   if (k == 0 || nb == 0) return 0;
   const size_t blk = (size_t)nb * b * b;
   Plan p;
@@ -349,7 +360,7 @@ size_t cnp_fwd_ws(int b, int k, int dt, long nb) {
 // The product that yields M_k also writes T = S + M_k = 2S + S.M_{k-1} in fp32, and the exact
 // I + T part of Q is added in fp32 in the last epilogue (replication review, "Summary": the
 // fused CNP reuses the lower powers across terms).
-poetx_status cnp_fwd_run(int b, int k, int dt, long nb, const float* theta, void* Q, char* ws, cudaStream_t st) {
+poetx_status cnp_fwd_generic(int b, int k, int dt, long nb, const float* theta, void* Q, char* ws, cudaStream_t st) {
   if (nb == 0) return POETX_OK;
   if (k == 0) return unpack(theta, nb, b, Q, dt, b, nullptr, dt, 0, nullptr, true, st);
   const size_t blk = (size_t)nb * b * b;
@@ -392,7 +403,7 @@ poetx_status cnp_fwd_run(int b, int k, int dt, long nb, const float* theta, void
 }
 
 // ------------------------------------------------------------------------- CNP backward
-size_t cnp_bwd_ws(int b, int k, int dt, long nb) {
+size_t cnp_bwd_generic_ws(int b, int k, int dt, long nb) {
   if (nb == 0) return 0;
   const size_t blk = (size_t)nb * b * b;
   Plan p;
@@ -413,8 +424,8 @@ size_t cnp_bwd_ws(int b, int k, int dt, long nb) {
 // then g[p(i,j)] = G_S[i][j] - G_S[j][i].  With N_j = I + M_j and S^T = -S this is
 //   G_S = E + [G | Gbar_k | ... | Gbar_2] . [M_k | ... | M_1]^T,   E = G + sum_{j=1..k} Gbar_j,
 // one long-K product plus an fp32 running sum E (the dominant 2G term never rounds to bf16).
-poetx_status cnp_bwd_run(int b, int k, int dt, long nb, const float* theta, const float* part, int splits,
-                         float* grad, char* ws, cudaStream_t st) {
+poetx_status cnp_bwd_generic(int b, int k, int dt, long nb, const float* theta, const float* part, int splits,
+                             float* grad, char* ws, cudaStream_t st) {
   if (nb == 0) return POETX_OK;
   const size_t blk = (size_t)nb * b * b;
   const long rows = nb * b;
@@ -486,6 +497,258 @@ poetx_status cnp_bwd_run(int b, int k, int dt, long nb, const float* theta, cons
   return pack(E, nb, b, grad, st);
 }
 
+// ----------------------------------------------------------------- fused CNP (bf16 path)
+// One launch runs the whole CNP forward (or adjoint) of up to two block sets (the R and P sides
+// of a layer) as a cluster program; see cnp_fused.cuh.  Used for bf16 and b <= 256.
+bool cnp_fused_ok(int b, int dt) { return dt == BF16 && b >= 64 && b <= 256; }
+int cnp_bn(int b) { return b >= 128 ? 128 : 64; }
+
+// Global scratch of the fused programs (per side): the bf16 operands the peer CTAs read.
+size_t cnp_fwd_fused_ws(int b, int k, long nb) {
+  if (k == 0 || nb == 0) return 0;
+  const size_t blk = (size_t)nb * b * b;
+  Plan p;
+  p.take(blk * 2);                                  // S (bf16)
+  if (k >= 2) { p.take(blk * 2); p.take(blk * 2); }  // M_j ping-pong (bf16)
+  return p.total;
+}
+size_t cnp_bwd_fused_ws(int b, int k, long nb) {
+  if (nb == 0) return 0;
+  const size_t blk = (size_t)nb * b * b;
+  Plan p;
+  p.take(blk * 4);  // E = G_S (f32), read transposed by PACK (G itself when k = 0)
+  if (k >= 1) {
+    p.take(blk * 2);               // S (bf16)
+    p.take(blk * (size_t)k * 2);   // A-stack [G | Gbar_k | ... | Gbar_2]
+    p.take(blk * (size_t)k * 2);   // B-stack [M_k | ... | M_1]
+  }
+  return p.total;
+}
+
+struct CnpSide {
+  long nb = 0;
+  const float* theta = nullptr;
+  void* Q = nullptr;                // forward output
+  const float* part = nullptr;      // adjoint: split-K partials of G
+  int splits = 1;
+  float* grad = nullptr;            // adjoint output
+  char* ws = nullptr;               // this side's scratch
+};
+
+CnpStageDesc stage_desc(int kind) {
+  CnpStageDesc d;
+  d.kind = kind; d.b_mn = 0; d.c_reg = CNP_NONE; d.alpha1 = 1.f; d.beta1 = 0.f; d.diag1 = 0; d.r1 = CNP_NONE;
+  d.g1_dtype = BF16; d.r2 = CNP_NONE; d.alpha2 = 1.f; d.beta2 = 0.f; d.accum2 = 0;
+  return d;
+}
+
+// Operand maps, K and global output of GEMM stage s for one segment.  A is K-major [rows, lda]
+// (block z at row z*b); B is MN-major (B[n][k] = mem[z*b+k][n]) or K-major (B[n][k] = mem[z*b+n][k]).
+poetx_status set_seg_gemm(CnpProgram& pr, int s, int q, long nb, const void* A, long lda, const void* B, long ldb,
+                          bool b_mn, int K, void* g1, long g1_ld) {
+  const int b = pr.b, BN = cnp_bn(b);
+  GemmDesc g;
+  g.M = b; g.N = b; g.K = K; g.batch = (int)nb;
+  g.A = view(A, nb * b, K, lda, b, 0);
+  g.B = view(B, nb * b, b_mn ? b : K, ldb, b, 0); g.b_mn = b_mn;
+  POETX_TRY(check_gemm(g, BF16));
+  CnpSegStage& G = pr.g[s][q];
+  if (!make_tmap(&G.tmA, g.A, 64, TC_BM)) return POETX_ERR_CUDA;
+  if (!make_tmap(&G.tmB, g.B, 64, b_mn ? 64 : BN)) return POETX_ERR_CUDA;
+  G.K = K; G.a_zrow = b; G.b_zrow = b; G.b_zcol = 0;
+  G.g1 = g1; G.g1_ld = g1_ld;
+  if (g1 && (!aligned16(g1) || g1_ld % 8)) return POETX_ERR_ALIGNMENT;
+  pr.st[s].b_mn = b_mn ? 1 : 0;
+  return POETX_OK;
+}
+
+template <int BN>
+poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_t st) {
+  constexpr int ST = 4;
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
+  constexpr size_t smem = tc_smem_bytes<BN, ST>();
+  auto kern = cnp_program_kernel<BN, ST>;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return POETX_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  if (nb_total > 65535) return POETX_ERR_UNSUPPORTED_SHAPE;
+  const int b = pr.b, nt = b / BN, mt = (b + TC_BM - 1) / TC_BM;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nt, mt, (unsigned)nb_total);
+  cfg.blockDim = dim3(CNP_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nt;
+  attr[0].val.clusterDim.y = mt;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LaunchScope ls(POETX_KC_CNP_GEMM, st);
+  if (cudaLaunchKernelEx(&cfg, kern, pr) != cudaSuccess) return POETX_ERR_CUDA;
+  return last_launch();
+}
+
+poetx_status run_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_t st) {
+  return cnp_bn(pr.b) == 128 ? launch_cnp_program<128>(pr, nb_total, st) : launch_cnp_program<64>(pr, nb_total, st);
+}
+
+std::mutex g_cnp_prog_mu;
+CnpProgram g_cnp_prog;  // large; rebuilt on the host for every launch (guarded by the mutex)
+
+// Forward: Q = (I + S)(I + S + ... + S^k) per block by the Horner recursion on M_j = N_j - I:
+//   R1 = S;  M_j = S.M_{j-1} + R1 (bf16 to global);  at j = k also R2 = T = S.M_{k-1} + 2 R1;
+//   Q = S.M_k + R2 + I   (k = 1: Q = S.S + 2 R1 + I;  k = 0: Q = I + S directly).
+poetx_status cnp_fwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaStream_t st) {
+  std::lock_guard<std::mutex> lock(g_cnp_prog_mu);
+  CnpProgram& pr = g_cnp_prog;
+  pr = CnpProgram();
+  pr.b = b;
+  pr.nseg = nsides;
+  long nb_total = 0;
+  for (int q = 0; q < nsides; ++q) nb_total += sides[q].nb;
+  if (nb_total == 0) return POETX_OK;
+  pr.st[0] = stage_desc(CNP_UNPACK);
+  int ns = 1;
+  if (k >= 1) {
+    for (int j = 2; j <= k + 1; ++j, ++ns) {
+      CnpStageDesc d = stage_desc(CNP_GEMM);
+      d.c_reg = CNP_R1;
+      d.beta1 = 1.f;
+      if (j == k && j <= k) { d.r2 = CNP_R2; d.alpha2 = 1.f; d.beta2 = 2.f; }
+      if (j == k + 1) {
+        d.diag1 = 1;
+        if (k == 1) d.beta1 = 2.f; else d.c_reg = CNP_R2;
+      }
+      pr.st[ns] = d;
+    }
+  }
+  pr.nstages = ns;
+  for (int q = 0; q < nsides; ++q) {
+    const CnpSide& sd = sides[q];
+    CnpSegment& S = pr.seg[q];
+    S.nb = (int)sd.nb;
+    S.theta = sd.theta;
+    S.splits = 1;
+    if (k == 0) {
+      S.no_sreg = 1; S.Sb0 = sd.Q; S.ld0 = b; S.add_identity = 1;
+      continue;
+    }
+    const size_t blk = (size_t)sd.nb * b * b;
+    Plan p;
+    char* Sop = sd.ws + p.take(blk * 2);
+    char* Mbuf[2] = {nullptr, nullptr};
+    if (k >= 2) { Mbuf[0] = sd.ws + p.take(blk * 2); Mbuf[1] = sd.ws + p.take(blk * 2); }
+    S.Sb0 = Sop; S.ld0 = b;
+    const void* Mprev = Sop;
+    int s = 1;
+    for (int j = 2; j <= k + 1; ++j, ++s) {
+      const bool last = (j == k + 1);
+      void* out = last ? sd.Q : Mbuf[j & 1];
+      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, Mprev, b, true, b, out, b));
+      Mprev = out;
+    }
+  }
+  return run_cnp_program(pr, nb_total, st);
+}
+
+// Adjoint (packed gradients) from the split-K partials of G = dL/dQ, by the Horner adjoint:
+//   G_S = G.N_k^T + sum_{j=1..k} Gbar_j.N_{j-1}^T,  Gbar_k = (I + S^T).G,  Gbar_{j-1} = S^T.Gbar_j,
+//   = E + [G | Gbar_k | ... | Gbar_2] . [M_k | ... | M_1]^T,  E = G + sum_j Gbar_j (f32, in TMEM R3).
+poetx_status cnp_bwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaStream_t st) {
+  std::lock_guard<std::mutex> lock(g_cnp_prog_mu);
+  CnpProgram& pr = g_cnp_prog;
+  pr = CnpProgram();
+  pr.b = b;
+  pr.nseg = nsides;
+  long nb_total = 0;
+  for (int q = 0; q < nsides; ++q) nb_total += sides[q].nb;
+  if (nb_total == 0) return POETX_OK;
+  const long kb = (long)k * b;
+  // stage list (same for both segments)
+  int ns = 0;
+  pr.st[ns++] = stage_desc(CNP_REDUCE_UNPACK);
+  if (k >= 1) {
+    for (int j = 2; j <= k; ++j) {  // M_j = S.M_{j-1} + S
+      CnpStageDesc d = stage_desc(CNP_GEMM);
+      d.c_reg = CNP_R1; d.beta1 = 1.f;
+      pr.st[ns++] = d;
+    }
+    {  // Gbar_k = G - S.G (bf16 out, k >= 2);  E = 2G - S.G
+      CnpStageDesc d = stage_desc(CNP_GEMM);
+      d.c_reg = CNP_R2; d.alpha1 = -1.f; d.beta1 = 1.f;
+      d.r2 = CNP_R3; d.alpha2 = -1.f; d.beta2 = 2.f;
+      pr.st[ns++] = d;
+    }
+    for (int j = k - 1; j >= 1; --j) {  // Gbar_j = -S.Gbar_{j+1};  E += Gbar_j
+      CnpStageDesc d = stage_desc(CNP_GEMM);
+      d.alpha1 = -1.f;
+      d.r2 = CNP_R3; d.alpha2 = -1.f; d.accum2 = 1;
+      pr.st[ns++] = d;
+    }
+    {  // G_S = E + A-stack . B-stack^T  -> global f32
+      CnpStageDesc d = stage_desc(CNP_GEMM);
+      d.c_reg = CNP_R3; d.beta1 = 1.f; d.g1_dtype = F32;
+      pr.st[ns++] = d;
+    }
+  }
+  pr.st[ns++] = stage_desc(CNP_PACK);
+  pr.nstages = ns;
+  for (int q = 0; q < nsides; ++q) {
+    const CnpSide& sd = sides[q];
+    CnpSegment& S = pr.seg[q];
+    S.nb = (int)sd.nb;
+    S.theta = sd.theta;
+    S.part = sd.part;
+    S.splits = sd.splits;
+    S.grad = sd.grad;
+    const size_t blk = (size_t)sd.nb * b * b;
+    Plan p;
+    float* E = reinterpret_cast<float*>(sd.ws + p.take(blk * 4));
+    S.GS = E;
+    if (k == 0) {
+      S.no_sreg = 1; S.G32 = E;
+      continue;
+    }
+    char* Sop = sd.ws + p.take(blk * 2);
+    char* Ast = sd.ws + p.take(blk * (size_t)k * 2);
+    char* Bst = sd.ws + p.take(blk * (size_t)k * 2);
+    auto aslot = [&](int t) { return static_cast<void*>(Ast + (size_t)t * b * 2); };
+    auto bslot = [&](int t) { return static_cast<void*>(Bst + (size_t)t * b * 2); };
+    S.Sb0 = Sop; S.ld0 = b; S.Sb1 = bslot(k - 1); S.ld1 = kb;
+    S.Gb = aslot(0); S.ldg = kb;
+    int s = 1;
+    for (int j = 2; j <= k; ++j, ++s)
+      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, bslot(k - j + 1), kb, true, b, bslot(k - j), kb));
+    POETX_TRY(set_seg_gemm(pr, s++, q, sd.nb, Sop, b, aslot(0), kb, true, b, k >= 2 ? aslot(1) : nullptr, kb));
+    for (int j = k - 1; j >= 1; --j, ++s)
+      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, aslot(k - j), kb, true, b, j >= 2 ? aslot(k - j + 1) : nullptr,
+                             kb));
+    POETX_TRY(set_seg_gemm(pr, s++, q, sd.nb, Ast, kb, Bst, kb, false, (int)kb, E, b));
+  }
+  return run_cnp_program(pr, nb_total, st);
+}
+
+// Scratch of the CNP forward / adjoint for nb blocks (fused path for bf16 and b <= 256).
+size_t cnp_fwd_ws(int b, int k, int dt, long nb) {
+  return cnp_fused_ok(b, dt) ? cnp_fwd_fused_ws(b, k, nb) : cnp_fwd_generic_ws(b, k, dt, nb);
+}
+size_t cnp_bwd_ws(int b, int k, int dt, long nb) {
+  return cnp_fused_ok(b, dt) ? cnp_bwd_fused_ws(b, k, nb) : cnp_bwd_generic_ws(b, k, dt, nb);
+}
+
+poetx_status cnp_fwd_run(int b, int k, int dt, long nb, const float* theta, void* Q, char* ws, cudaStream_t st) {
+  if (!cnp_fused_ok(b, dt)) return cnp_fwd_generic(b, k, dt, nb, theta, Q, ws, st);
+  CnpSide sd;
+  sd.nb = nb; sd.theta = theta; sd.Q = Q; sd.ws = ws;
+  return cnp_fwd_fused(b, k, &sd, 1, st);
+}
+
 // ------------------------------------------------------------------------- layer plans
 struct FwdPlan {
   size_t U, V, Yp, Z, total;
@@ -503,7 +766,7 @@ FwdPlan fwd_plan(const poetx_desc* d, long n) {
 }
 
 struct BwdPlan {
-  size_t dYp, dZ, dV, U, dU, V, Z, GpR, GpP, cnp, total;
+  size_t dYp, dZ, dV, U, dU, V, Z, GpR, GpP, cnpR, cnpP, total;
   int sR, sP;
 };
 BwdPlan bwd_plan(const poetx_desc* d, long n) {
@@ -522,13 +785,16 @@ BwdPlan bwd_plan(const poetx_desc* d, long n) {
   w.sP = grad_splits(d->dtype, n, nbi, b);
   w.GpR = p.take((size_t)w.sR * nbo * b * b * 4);
   w.GpP = p.take((size_t)w.sP * nbi * b * b * 4);
-  w.cnp = p.take(std::max(cnp_bwd_ws(b, d->k, d->dtype, nbo), cnp_bwd_ws(b, d->k, d->dtype, nbi)));
+  w.cnpR = p.take(cnp_bwd_ws(b, d->k, d->dtype, nbo));
+  w.cnpP = p.take(cnp_bwd_ws(b, d->k, d->dtype, nbi));
   w.total = p.total;
   return w;
 }
 
+// Scratch of poetx_cnp: the two sides run concurrently and need disjoint regions.
 size_t cnp_layer_ws(const poetx_desc* d) {
-  return std::max(cnp_fwd_ws(d->b, d->k, d->dtype, d->d_out / d->b), cnp_fwd_ws(d->b, d->k, d->dtype, d->d_in / d->b));
+  return align256(cnp_fwd_ws(d->b, d->k, d->dtype, d->d_out / d->b)) +
+         align256(cnp_fwd_ws(d->b, d->k, d->dtype, d->d_in / d->b));
 }
 
 struct MergePlan {
@@ -662,8 +928,15 @@ poetx_status poetx_cnp(const poetx_desc* desc, const float* theta_R, const float
   POETX_TRY(check_ws(workspace, ws_bytes, cnp_layer_ws(desc)));
   char* ws = static_cast<char*>(workspace);
   const int b = desc->b;
-  POETX_TRY(cnp_fwd_run(b, desc->k, desc->dtype, desc->d_out / b, theta_R, Q_R, ws, stream));
-  return cnp_fwd_run(b, desc->k, desc->dtype, desc->d_in / b, theta_P, Q_P, ws, stream);
+  const size_t offP = align256(cnp_fwd_ws(b, desc->k, desc->dtype, desc->d_out / b));
+  if (cnp_fused_ok(b, desc->dtype)) {
+    CnpSide sides[2];
+    sides[0].nb = desc->d_out / b; sides[0].theta = theta_R; sides[0].Q = Q_R; sides[0].ws = ws;
+    sides[1].nb = desc->d_in / b; sides[1].theta = theta_P; sides[1].Q = Q_P; sides[1].ws = ws + offP;
+    return cnp_fwd_fused(b, desc->k, sides, 2, stream);
+  }
+  POETX_TRY(cnp_fwd_generic(b, desc->k, desc->dtype, desc->d_out / b, theta_R, Q_R, ws, stream));
+  return cnp_fwd_generic(b, desc->k, desc->dtype, desc->d_in / b, theta_P, Q_P, ws + offP, stream);
 }
 
 poetx_status poetx_absorb(const poetx_desc* desc, const void* W0, const int32_t* perm_L, const int32_t* perm_R,
@@ -744,10 +1017,18 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
   POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
   POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, stream));
   // CNP adjoint, packed gradients only.
-  POETX_TRY(cnp_bwd_run(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + w.GpR), w.sR,
-                        grad_theta_R, ws + w.cnp, stream));
-  return cnp_bwd_run(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + w.GpP), w.sP, grad_theta_P,
-                     ws + w.cnp, stream);
+  if (cnp_fused_ok(b, dt)) {
+    CnpSide sides[2];
+    sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + w.GpR);
+    sides[0].splits = w.sR; sides[0].grad = grad_theta_R; sides[0].ws = ws + w.cnpR;
+    sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + w.GpP);
+    sides[1].splits = w.sP; sides[1].grad = grad_theta_P; sides[1].ws = ws + w.cnpP;
+    return cnp_bwd_fused(b, desc->k, sides, 2, stream);
+  }
+  POETX_TRY(cnp_bwd_generic(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + w.GpR), w.sR,
+                            grad_theta_R, ws + w.cnpR, stream));
+  return cnp_bwd_generic(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + w.GpP), w.sP,
+                         grad_theta_P, ws + w.cnpP, stream);
 }
 
 poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, const void* Q_P,

@@ -19,7 +19,7 @@ from orthogonal_equivalence_cnp_b200.layer import make_desc
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("dtype,b,nblocks", [("bf16", 256, 36), ("bf16", 128, 20), ("f32", 32, 24)])
+@pytest.mark.parametrize("dtype,b,nblocks", [("bf16", 256, 85), ("bf16", 128, 20), ("bf16", 512, 9), ("f32", 32, 24)])
 def test_noalloc_matches_workspace_entry_point_twice(dtype, b, nblocks):
     desc = make_desc(b, b, b, 3, dtype, "fast")
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -40,9 +40,9 @@ def test_noalloc_matches_workspace_entry_point_twice(dtype, b, nblocks):
 
 def test_noalloc_rejects_more_than_its_scratch():
     desc = make_desc(256, 256, 256, 3, "bf16", "fast")
-    assert P.poetx_cnp_blocks_workspace_size(desc, 36) <= 32 << 20 < P.poetx_cnp_blocks_workspace_size(desc, 37)
-    theta = torch.zeros(37, 256 * 255 // 2, dtype=torch.float32, device="cuda")
-    Q = torch.empty(37, 256, 256, dtype=torch.bfloat16, device="cuda")
-    st = P.lib().poetx_cnp_blocks_noalloc(ctypes.byref(desc), 37, theta.data_ptr(), Q.data_ptr(),
+    assert P.poetx_cnp_blocks_workspace_size(desc, 85) <= 32 << 20 < P.poetx_cnp_blocks_workspace_size(desc, 86)
+    theta = torch.zeros(86, 256 * 255 // 2, dtype=torch.float32, device="cuda")
+    Q = torch.empty(86, 256, 256, dtype=torch.bfloat16, device="cuda")
+    st = P.lib().poetx_cnp_blocks_noalloc(ctypes.byref(desc), 86, theta.data_ptr(), Q.data_ptr(),
                                            torch.cuda.current_stream().cuda_stream)
     assert st == 4  # POETX_ERR_WORKSPACE: beyond the built-in 32 MiB, nothing launched
