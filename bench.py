@@ -125,6 +125,15 @@ def gpu_uuid(dev) -> str:
         return ""
 
 
+def count_step_launches(P, layer, X, dY) -> int:
+    """Kernels the library launches in one step (counted on a directly launched step)."""
+    import torch
+    n0 = P.poetx_launch_count()
+    layer.step(X, dY)
+    torch.cuda.synchronize()
+    return P.poetx_launch_count() - n0
+
+
 # ---------------------------------------------------------------------------- distributed
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
@@ -223,6 +232,22 @@ def run_poetx(args):
         raise RuntimeError(f"device-side timeout during warm-up ({det:#x})")
 
     K = args.steps
+    # One step captured into a CUDA graph and replayed: launch-bound sequences of short kernels
+    # run without host overhead between them (every kernel of the step is one of ours).
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer.step(X, dY)
+        graph.replay()
+        torch.cuda.synchronize()
+
+    def run_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            layer.step(X, dY)
+
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     clocks = ClockSampler()
@@ -231,14 +256,15 @@ def run_poetx(args):
     barrier()
     torch.cuda.synchronize()
     launches0 = P.poetx_launch_count()
+    step_launches = count_step_launches(P, layer, X, dY) if graph is not None else None
     for i in range(K):
         flush.zero_()
         ev0[i].record(stream)
-        layer.step(X, dY)
+        run_step()
         ev1[i].record(stream)
     torch.cuda.synchronize()
     barrier()
-    launches = P.poetx_launch_count() - launches0
+    launches = P.poetx_launch_count() - launches0 if graph is None else step_launches * K
     clk = clocks.stop(gpu_uuid(dev))
     times = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
     t_ms = max_over_ranks(sum(times), world, dev)
@@ -246,15 +272,30 @@ def run_poetx(args):
     if st != 0:
         raise RuntimeError(f"device-side timeout in the timed region ({det:#x})")
 
-    # Live per-kernel durations: the same K steps again with the library's event pairs around
-    # every launch (separate pass, so the headline timing carries no bookkeeping).
+    # Live per-kernel durations: a graph of one step captured with the library's CUDA-event pair
+    # around every launch, replayed K times (separate pass, so the headline timing carries no
+    # bookkeeping); per-class device time is read back after each replay.
     P.poetx_profile_enable(True)
+    if graph is not None:
+        pgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pgraph):
+            layer.step(X, dY)
+    P.poetx_profile_enable(False)
+    prof = {}
     for i in range(K):
         flush.zero_()
-        layer.step(X, dY)
-    torch.cuda.synchronize()
-    prof = P.poetx_profile_summary()
-    P.poetx_profile_enable(False)
+        if graph is not None:
+            pgraph.replay()
+        else:
+            P.poetx_profile_enable(True)
+            layer.step(X, dY)
+            P.poetx_profile_enable(False)
+        torch.cuda.synchronize()
+        for k, (n, ms) in P.poetx_profile_summary().items():
+            c = prof.get(k, (0, 0.0))
+            prof[k] = (c[0] + n, c[1] + ms)
+    if graph is not None:
+        del pgraph
 
     # End to end through the public API with host buffers: H2D of X and dY from pinned memory,
     # the step, D2H of dX and the packed gradients, all inside the timed interval.
@@ -312,6 +353,7 @@ def run_poetx(args):
                    "n_tokens_per_gpu": s.n_tokens, "mode": s.mode,
                    "step": "CNP fwd (R,P) + forward + backward incl. CNP adjoint",
                    "l2": "flushed between steps (256 MiB write outside the timed intervals)",
+                   "launch": "CUDA graph of one step, replayed" if graph is not None else "direct launches",
                    "parallelism": f"replicas x{world} (data parallel over tokens, no collective on the path)",
                    "algorithmic_gflop_per_step": round(fl["total"] / 1e9, 2)},
         "roofline": {"bound": "tensor", "kernel": "w0_gemm (Z = V W0'^T, dV = dZ W0')",
@@ -398,6 +440,7 @@ def main():
     ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
     ap.add_argument("--workload", choices=sorted(I.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every step directly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

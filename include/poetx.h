@@ -62,15 +62,15 @@ typedef enum {
 
 typedef enum { POETX_F32 = 0, POETX_BF16 = 1 } poetx_dtype;
 
-/* POET-Xfast keeps the W0'-GEMM output Z for the backward pass; POET-Xmem keeps only X and
- * recomputes Π_R·x, BD_P·(·) and Z in the backward pass (replication review, "Summary":
+/* POET-Xfast keeps the W0'-GEMM output Z and the permuted input Π_R·x for the backward pass;
+ * POET-Xmem keeps only X and recomputes Π_R·x, BD_P·(·) and Z in the backward pass (replication review, "Summary":
  * POET-Xfast and checkpointed POET-Xmem; agidaily.cc article: the mem variant recomputes part
  * of the activations). */
 typedef enum { POETX_FAST = 0, POETX_MEM = 1 } poetx_mode;
 
 typedef struct {
-  int d_in;          /* input features, multiple of b                                     */
-  int d_out;         /* output features, multiple of b                                    */
+  int d_in;          /* input features, multiple of b; at most 32768 (BF16) / 16384 (F32) */
+  int d_out;         /* output features, same rules as d_in                               */
   int b;             /* block size: 32, 64, 128, 256 or 512 (BF16: 64..512)              */
   int k;             /* Neumann order, 0 <= k <= 8 (the pages use k = 3)                  */
   poetx_dtype dtype; /* storage type of activations, W0', Q                               */
@@ -133,27 +133,28 @@ poetx_status poetx_absorb(const poetx_desc* desc, const void* W0, const int32_t*
  *   perm_L  int32 [d_out], perm_R int32 [d_in] (in)
  *   Q_R     dtype [d_out/b, b, b], Q_P dtype [d_in/b, b, b] (in, from poetx_cnp)
  *   Y       dtype [N, d_out] (out)
- *   Z_saved dtype [N, d_out] (out) in POETX_FAST mode — pass it back to poetx_backward;
- *           must be NULL in POETX_MEM mode.
+ *   saved   dtype [N*(d_out + d_in)] (out) in POETX_FAST mode: Z = V . W0'^T [N, d_out]
+ *           followed by U = X[:, π_R] [N, d_in]; pass it back to poetx_backward.  Must be
+ *           NULL in POETX_MEM mode (nothing is kept; the backward pass recomputes both).
  * n_tokens == 0 is valid and launches nothing. */
 poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
                            const int32_t* perm_L, const int32_t* perm_R, const void* Q_R,
-                           const void* Q_P, void* Y, void* Z_saved, void* workspace,
+                           const void* Q_P, void* Y, void* saved, void* workspace,
                            size_t ws_bytes, poetx_stream stream);
 
 /* Backward pass: dX and the gradients w.r.t. the PACKED skew parameters (only the packed form
  * is written; replication review, "Summary": compact skew storage; W0 is frozen, so there is
- * no dW0).  In POETX_MEM mode Z_saved must be NULL and Z is recomputed from X.
+ * no dW0).  In POETX_MEM mode `saved` must be NULL and U, V, Z are recomputed from X.
  *   dY dtype [N, d_out], X dtype [N, d_in], W0p, perm_L, perm_R, Q_R, Q_P as in forward (in)
  *   theta_R, theta_P float32 packed (in; the CNP adjoint needs S)
- *   Z_saved dtype [N, d_out] (in, FAST) or NULL (MEM)
+ *   saved   dtype [N*(d_out + d_in)] (in, FAST: as written by poetx_forward) or NULL (MEM)
  *   dX dtype [N, d_in] (out); grad_theta_R float32 [d_out/b, b(b-1)/2] (out);
  *   grad_theta_P float32 [d_in/b, b(b-1)/2] (out).
  * n_tokens == 0 writes zero gradients. */
 poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
                             const void* W0p, const int32_t* perm_L, const int32_t* perm_R,
                             const void* Q_R, const void* Q_P, const float* theta_R,
-                            const float* theta_P, const void* Z_saved, void* dX,
+                            const float* theta_P, const void* saved, void* dX,
                             float* grad_theta_R, float* grad_theta_P, void* workspace,
                             size_t ws_bytes, poetx_stream stream);
 

@@ -159,19 +159,19 @@ def poetx_absorb(desc, W0, perm_L, perm_R, W0p, stream=None):
                               _stream(stream)), "poetx_absorb")
 
 
-def poetx_forward(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, Z_saved, workspace, ws_bytes=None,
+def poetx_forward(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, saved, workspace, ws_bytes=None,
                   stream=None):
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0p), _ptr(perm_L), _ptr(perm_R),
-                               _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(Z_saved), _ptr(workspace), ws_bytes,
+                               _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(saved), _ptr(workspace), ws_bytes,
                                _stream(stream)), "poetx_forward")
 
 
-def poetx_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, Z_saved, dX,
+def poetx_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved, dX,
                    grad_theta_R, grad_theta_P, workspace, ws_bytes=None, stream=None):
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_backward(ctypes.byref(desc), n_tokens, _ptr(dY), _ptr(X), _ptr(W0p), _ptr(perm_L),
-                                _ptr(perm_R), _ptr(Q_R), _ptr(Q_P), _ptr(theta_R), _ptr(theta_P), _ptr(Z_saved),
+                                _ptr(perm_R), _ptr(Q_R), _ptr(Q_P), _ptr(theta_R), _ptr(theta_P), _ptr(saved),
                                 _ptr(dX), _ptr(grad_theta_R), _ptr(grad_theta_P), _ptr(workspace), ws_bytes,
                                 _stream(stream)), "poetx_backward")
 

@@ -31,6 +31,9 @@ constexpr int CNP_THREADS = 256;  // 8 warps: warp w owns TMEM lane quarter w%4,
 enum CnpStageKind : int { CNP_GEMM = 0, CNP_UNPACK = 1, CNP_REDUCE_UNPACK = 2, CNP_PACK = 3 };
 enum CnpReg : int { CNP_NONE = -1, CNP_ACC = 0, CNP_R1 = 1, CNP_R2 = 2, CNP_R3 = 3 };
 enum : int { KID_CNP_FUSED = 2 };
+// Rows (or columns) per lane batch in the elementwise stages: all loads of a batch are issued
+// before the first shared-memory store.
+template <int BN> struct EwBatch { static constexpr int value = 8; };
 
 // Stage description shared by the segments (register-form epilogue):
 //   out1 = alpha1*acc + beta1*REG[c_reg] (+ I if diag1)  -> global g1 (g1_dtype) and/or REG[r1]
@@ -94,6 +97,19 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Shared memory of the program kernel: the TMA ring, or two padded 128 x BN f32 staging tiles
+// (whichever is larger), then the barriers.
+template <int BN, int STAGES>
+__host__ __device__ constexpr size_t cnp_data_bytes() {
+  return (size_t)STAGES * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) > (size_t)2 * TC_BM * (BN + 4) * 4
+             ? (size_t)STAGES * (TC_BM * TC_BK * 2 + BN * TC_BK * 2)
+             : ((size_t)2 * TC_BM * (BN + 4) * 4 + 1023) / 1024 * 1024;
+}
+template <int BN, int STAGES>
+__host__ __device__ constexpr size_t cnp_smem_bytes() {
+  return cnp_data_bytes<BN, STAGES>() + 1024 /*align*/ + 256 /*barriers*/;
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __grid_constant__ CnpProgram prog) {
   constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
@@ -106,7 +122,7 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + cnp_data_bytes<BN, STAGES>());
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
   const uint32_t smem0 = smem_u32(smem);
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -146,7 +162,31 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
   const uint32_t tmem0 = *tmem_holder;
   const uint32_t tlane = tmem0 + ((uint32_t)(quarter * 32) << 16);
   auto treg = [&](int reg, int col) { return tlane + (uint32_t)(reg * BN + col); };
-
+  // Two 128 x BN f32 staging tiles (padded row stride), overlaid on the TMA ring, which is idle
+  // whenever they are in use (between the last MMA of a stage and the first TMA load of the next).
+  constexpr int TS = BN + 4;  // padded row stride (16-byte aligned rows for float4 access)
+  constexpr int EW_B = EwBatch<BN>::value;
+  float* T0 = reinterpret_cast<float*>(smem);
+  float* T1 = T0 + TC_BM * TS;
+  // Coalesced write of a staged tile to global: warps over rows, lanes along columns.
+  auto tile_store = [&](const float* T, void* dst, long ld, int dt) {
+    for (int r = warp; r < TC_BM; r += CNP_THREADS / 32) {
+      const int ii = m0 + r;
+      if (ii >= b) break;
+      const long base = ((long)z * b + ii) * ld + n0;
+      for (int cc = lane * 4; cc < BN; cc += 128) {
+        const float4 f = *reinterpret_cast<const float4*>(T + r * TS + cc);
+        if (dt == BF16) {
+          uint2 u;
+          u.x = pack_bf16x2(f.x, f.y);
+          u.y = pack_bf16x2(f.z, f.w);
+          *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dst) + base + cc) = u;
+        } else {
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(dst) + base + cc) = f;
+        }
+      }
+    }
+  };
   uint32_t it = 0;
   uint32_t acc_phase = 0;
 
@@ -239,72 +279,160 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         }
       }
     } else if (D.kind == CNP_UNPACK || D.kind == CNP_REDUCE_UNPACK) {
-      const long sstride = (long)S.nb * b * b;
+      // theta -> T0 with coalesced, batched loads: above the diagonal warps walk rows (theta's
+      // packed row i is contiguous in j), below it warps walk columns (packed row j is
+      // contiguous in i).  Each lane issues EW_B loads before its first shared-memory store.
+      constexpr int RW = TC_BM / (CNP_THREADS / 32);  // rows (or columns) per warp
+      constexpr int CPL = BN / 32;                    // columns (or rows / 32) per lane
+#pragma unroll 1
+      for (int t0 = 0; t0 < RW; t0 += EW_B) {
+        float v[EW_B][CPL];
+#pragma unroll
+        for (int t = 0; t < EW_B; ++t)
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) {
+            const int ii = m0 + warp + 8 * (t0 + t), jj = n0 + lane + 32 * q;
+            v[t][q] = (ii < b && jj > ii) ? __ldg(th + packed_pos(ii, jj, b)) : 0.f;
+          }
+#pragma unroll
+        for (int t = 0; t < EW_B; ++t)
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) {
+            const int r = warp + 8 * (t0 + t), cc = lane + 32 * q, ii = m0 + r, jj = n0 + cc;
+            if (jj > ii) T0[r * TS + cc] = v[t][q];
+            else if (jj == ii) T0[r * TS + cc] = S.add_identity ? 1.f : 0.f;
+          }
+      }
+      constexpr int RPL = TC_BM / 32;  // rows per lane in the column walk
+#pragma unroll 1
+      for (int t0 = 0; t0 < BN / 8; t0 += EW_B) {
+        float v[EW_B][RPL];
+#pragma unroll
+        for (int t = 0; t < EW_B; ++t)
+#pragma unroll
+          for (int q = 0; q < RPL; ++q) {
+            const int jj = n0 + warp + 8 * (t0 + t), ii = m0 + lane + 32 * q;
+            v[t][q] = (ii < b && ii > jj) ? -__ldg(th + packed_pos(jj, ii, b)) : 0.f;
+          }
+#pragma unroll
+        for (int t = 0; t < EW_B; ++t)
+#pragma unroll
+          for (int q = 0; q < RPL; ++q) {
+            const int cc = warp + 8 * (t0 + t), r = lane + 32 * q;
+            if (m0 + r > n0 + cc) T0[r * TS + cc] = v[t][q];
+          }
+      }
+      if (D.kind == CNP_REDUCE_UNPACK) {
+        // G = sum of split-K partials -> T1, row walk with one float4 per lane per row.
+        const long sstride = (long)S.nb * b * b;
+        constexpr int RB = 4;
+#pragma unroll 1
+        for (int t0 = 0; t0 < RW; t0 += RB) {
+          float4 acc4[RB];
+#pragma unroll
+          for (int t = 0; t < RB; ++t) acc4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int sp0 = 0; sp0 < S.splits; sp0 += 4) {  // four splits' loads in flight at once
+            float4 ld4[4][RB];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int t = 0; t < RB; ++t) {
+                const int ii = m0 + warp + 8 * (t0 + t), sp = sp0 + u;
+                ld4[u][t] = (sp < S.splits && ii < b && lane * 4 < BN)
+                                ? __ldg(reinterpret_cast<const float4*>(S.part + sp * sstride + ((long)z * b + ii) * b + n0) + lane)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int t = 0; t < RB; ++t) {
+                acc4[t].x += ld4[u][t].x; acc4[t].y += ld4[u][t].y; acc4[t].z += ld4[u][t].z; acc4[t].w += ld4[u][t].w;
+              }
+          }
+#pragma unroll
+          for (int t = 0; t < RB; ++t)
+            if (lane * 4 < BN) *reinterpret_cast<float4*>(T1 + (warp + 8 * (t0 + t)) * TS + lane * 4) = acc4[t];
+        }
+      }
+      __syncthreads();
+      // Coalesced global copies from the tiles; then each thread moves its row into TMEM.
+      if (S.Sb0) tile_store(T0, S.Sb0, S.ld0, BF16);
+      if (S.Sb1) tile_store(T0, S.Sb1, S.ld1, BF16);
+      if (D.kind == CNP_REDUCE_UNPACK) {
+        if (S.Gb) tile_store(T1, S.Gb, S.ldg, BF16);
+        if (S.G32) tile_store(T1, S.G32, b, F32);
+      }
+      wrote_global = true;
 #pragma unroll 1
       for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
-        const int n = n0 + c;
-        // S[i][n..n+31]: above the diagonal a contiguous run of theta's row i; below it,
-        // theta[p(j, i)] for consecutive rows i of the warp, i.e. coalesced across lanes.
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int jj = n + j;
-          float x = 0.f;
-          if (row_ok) {
-            if (i < jj) x = __ldg(th + packed_pos(i, jj, b));
-            else if (i > jj) x = -__ldg(th + packed_pos(jj, i, b));
-            else if (S.add_identity) x = 1.f;
-          }
-          v[j] = x;
-        }
-        float gsum[32];
-        if (D.kind == CNP_REDUCE_UNPACK) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) gsum[j] = 0.f;
-          if (row_ok)
-            for (int sp = 0; sp < S.splits; ++sp) {
-              float t[32];
-              load32(S.part + sp * sstride, grow * b + n, F32, t);
-#pragma unroll
-              for (int j = 0; j < 32; ++j) gsum[j] += t[j];
-            }
-        }
+        uint32_t w[32];
         if (!S.no_sreg) {
-          uint32_t w[32];
+          const float4* trow = reinterpret_cast<const float4*>(T0 + (quarter * 32 + lane) * TS + c);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+          for (int j = 0; j < 8; ++j) {
+            const float4 f = trow[j];
+            w[4 * j] = __float_as_uint(f.x); w[4 * j + 1] = __float_as_uint(f.y);
+            w[4 * j + 2] = __float_as_uint(f.z); w[4 * j + 3] = __float_as_uint(f.w);
+          }
           tmem_st_32x32b_x32(treg(CNP_R1, c), w);
           wrote_tmem = true;
         }
-        if (row_ok) {
-          if (S.Sb0) store32(S.Sb0, grow * S.ld0 + n, BF16, v);
-          if (S.Sb1) store32(S.Sb1, grow * S.ld1 + n, BF16, v);
-          wrote_global = true;
-        }
         if (D.kind == CNP_REDUCE_UNPACK) {
-          uint32_t w[32];
+          const float4* grow4 = reinterpret_cast<const float4*>(T1 + (quarter * 32 + lane) * TS + c);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(gsum[j]);
+          for (int j = 0; j < 8; ++j) {
+            const float4 f = grow4[j];
+            w[4 * j] = __float_as_uint(f.x); w[4 * j + 1] = __float_as_uint(f.y);
+            w[4 * j + 2] = __float_as_uint(f.z); w[4 * j + 3] = __float_as_uint(f.w);
+          }
           tmem_st_32x32b_x32(treg(CNP_R2, c), w);
           wrote_tmem = true;
-          if (row_ok) {
-            if (S.Gb) store32(S.Gb, grow * S.ldg + n, BF16, gsum);
-            if (S.G32) store32(S.G32, grow * b + n, F32, gsum);
-          }
         }
       }
     } else if (D.kind == CNP_PACK) {
+      // T0 = own tile of G_S (row walk), T1[i][j] = G_S[j][i] (column walk, contiguous in i);
+      // then g[p(i,j)] = T0 - T1 with lanes along j (contiguous in p).
+      constexpr int RW = TC_BM / (CNP_THREADS / 32);
+      constexpr int CPL = BN / 32;
+      constexpr int RPL = TC_BM / 32;
 #pragma unroll 1
-      for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
-        const int n = n0 + c;
-        if (!row_ok || n + 31 <= i) continue;
-        float a[32], t[32];
-        load32(S.GS, grow * b + n, F32, a);
+      for (int t0 = 0; t0 < RW; t0 += EW_B) {
+        float v[EW_B][CPL];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) t[j] = (i < n + j) ? S.GS[((long)z * b + n + j) * b + i] : 0.f;
+        for (int t = 0; t < EW_B; ++t)
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (i < n + j) S.grad[(long)z * P + packed_pos(i, n + j, b)] = a[j] - t[j];
+          for (int q = 0; q < CPL; ++q) {
+            const int ii = m0 + warp + 8 * (t0 + t);
+            v[t][q] = ii < b ? S.GS[((long)z * b + ii) * b + n0 + lane + 32 * q] : 0.f;
+          }
+#pragma unroll
+        for (int t = 0; t < EW_B; ++t)
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) T0[(warp + 8 * (t0 + t)) * TS + lane + 32 * q] = v[t][q];
+      }
+#pragma unroll 1
+      for (int t0 = 0; t0 < BN / 8; t0 += EW_B) {
+        float v[EW_B][RPL];
+#pragma unroll
+        for (int t = 0; t < EW_B; ++t)
+#pragma unroll
+          for (int q = 0; q < RPL; ++q) {
+            const int jj = n0 + warp + 8 * (t0 + t), ii = m0 + lane + 32 * q;
+            v[t][q] = ii < b ? S.GS[((long)z * b + jj) * b + ii] : 0.f;
+          }
+#pragma unroll
+        for (int t = 0; t < EW_B; ++t)
+#pragma unroll
+          for (int q = 0; q < RPL; ++q) T1[(lane + 32 * q) * TS + warp + 8 * (t0 + t)] = v[t][q];
+      }
+      __syncthreads();
+      for (int r = warp; r < TC_BM; r += CNP_THREADS / 32) {
+        const int ii = m0 + r;
+        if (ii >= b) break;
+        for (int cc = lane; cc < BN; cc += 32) {
+          const int jj = n0 + cc;
+          if (ii < jj) S.grad[(long)z * P + packed_pos(ii, jj, b)] = T0[r * TS + cc] - T1[r * TS + cc];
+        }
       }
     }
     if (wrote_tmem) tmem_wait_st();

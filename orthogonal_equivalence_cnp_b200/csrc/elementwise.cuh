@@ -2,7 +2,10 @@
 // unpack / packed-gradient pack, split-K reduction, permutation inverse and composition.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace poetx {
 
@@ -13,82 +16,107 @@ __host__ __device__ __forceinline__ long packed_pos(int i, int j, int b) {
 
 // Index-based permutation of the feature (column) dimension of a row-major [rows, cols] array
 // (replication review of POET-X, "Summary": permutations applied by index, never as a matmul;
-// Table 1 of the paper measures such a kernel).  A block stages `rb` whole rows in shared
-// memory with 16-byte coalesced loads, permutes inside shared memory and writes 16-byte
-// coalesced stores, so HBM sees one read and one write of each element.  Each thread keeps
-// PERM_VPT independent 16-byte loads in flight (registers first, then shared memory), which is
-// what it takes to cover HBM latency at ~16 resident warps per SM.
+// Table 1 of the paper measures such a kernel).  HBM sees one read and one write per element.
+// ROWS rows (4, or 2 for very wide rows) are processed together and stored in shared memory
+// interleaved: one word (ROWS x 16 bit) holds element c of all of them, so one random word
+// access moves ROWS elements.  The word of column c sits at (c & 7) * (cols / 8) + (c >> 3),
+// which lets the loading lanes write consecutive words (no bank conflicts).  Rows are read with
+// coalesced 16-byte loads straight into registers and written back with 16-byte coalesced
+// stores; the 16-bit source map (for a scatter: the inverse map, built in shared memory)
+// is cached per block.
 //   gather (scatter == 0): out[r][j] = in[rowmap ? rowmap[r] : r][colmap[j]]
 //   scatter (scatter == 1): out[r][colmap[j]] = in[r][j]
-// Requires cols % (16 / sizeof(T)) == 0 and 16-byte aligned rows.
-constexpr int PERM_VPT = 8;
+// bf16 (16-bit) elements; requires cols <= 65536, cols % 8 == 0, 16-byte aligned rows.
+template <int ROWS>
+__host__ __device__ constexpr size_t permute_smem_bytes(int cols) {
+  return ((size_t)cols * 2 + 15) / 16 * 16 + (size_t)cols * 2 * ROWS;
+}
 
-template <typename T>
+template <int ROWS>
 __global__ void __launch_bounds__(256)
-    permute_cols_kernel(const T* __restrict__ in, long ld_in, T* __restrict__ out, long ld_out, long rows,
-                        int cols, const int32_t* __restrict__ colmap, const int32_t* __restrict__ rowmap,
-                        int scatter, int rb) {
+    permute_cols_bf16_kernel(const uint16_t* __restrict__ in, long ld_in, uint16_t* __restrict__ out, long ld_out,
+                             long rows, int cols, const int32_t* __restrict__ colmap,
+                             const int32_t* __restrict__ rowmap, int scatter) {
+  using Word = typename std::conditional<ROWS == 4, uint64_t, uint32_t>::type;
   extern __shared__ __align__(16) uint8_t smem_perm[];
-  T* buf = reinterpret_cast<T*>(smem_perm);
-  constexpr int VEC = 16 / sizeof(T);
-  const int nvec = cols / VEC;
-  const int nthr = blockDim.x;
-  for (long r0 = (long)blockIdx.x * rb; r0 < rows; r0 += (long)gridDim.x * rb) {
-    const int nr = (int)min((long)rb, rows - r0);
-    const int total = nr * nvec;
-    // Phase 1: rows -> registers -> shared memory (gather: as is; scatter: permuted).
-    for (int base = threadIdx.x; base < total; base += nthr * PERM_VPT) {
-      uint4 v[PERM_VPT];
+  uint16_t* src_of = reinterpret_cast<uint16_t*>(smem_perm);  // output column j reads source column src_of[j]
+  Word* W = reinterpret_cast<Word*>(smem_perm + ((size_t)cols * 2 + 15) / 16 * 16);
+  const int nvec = cols / 8;
+  for (int j = threadIdx.x; j < cols; j += blockDim.x) {
+    const int m = __ldg(colmap + j);
+    if (scatter) src_of[m] = (uint16_t)j; else src_of[j] = (uint16_t)m;
+  }
+  __syncthreads();
+  const long ngroups = (rows + ROWS - 1) / ROWS;
+  for (long g = blockIdx.x; g < ngroups; g += gridDim.x) {
+    const long r0 = g * ROWS;
+    const int nr = (int)min((long)ROWS, rows - r0);
+    long src_row[ROWS];
 #pragma unroll
-      for (int u = 0; u < PERM_VPT; ++u) {
-        const int t = base + u * nthr;
-        if (t < total) {
-          const int rr = t / nvec, c = t - rr * nvec;
-          const long rin = (!scatter && rowmap) ? (long)__ldg(rowmap + r0 + rr) : r0 + rr;
-          v[u] = __ldg(reinterpret_cast<const uint4*>(in + rin * ld_in) + c);
+    for (int r = 0; r < ROWS; ++r) {
+      const long rr = r0 + min(r, nr - 1);  // a short group repeats its last row
+      src_row[r] = (!scatter && rowmap) ? (long)__ldg(rowmap + rr) : rr;
+    }
+    // Load: 8 columns of each row per thread, two column vectors in flight per thread.
+    for (int c0 = threadIdx.x; c0 < nvec; c0 += blockDim.x * 2) {
+      uint4 v[2][ROWS];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          const int c = c0 + u * blockDim.x;
+          if (c < nvec) v[u][r] = __ldg(reinterpret_cast<const uint4*>(in + src_row[r] * ld_in) + c);
         }
-      }
 #pragma unroll
-      for (int u = 0; u < PERM_VPT; ++u) {
-        const int t = base + u * nthr;
-        if (t < total) {
-          const int rr = t / nvec, c = t - rr * nvec;
-          T* row = buf + (long)rr * cols;
-          if (!scatter) {
-            reinterpret_cast<uint4*>(row)[c] = v[u];
-          } else {
-            const T* vals = reinterpret_cast<const T*>(&v[u]);
-            int idx[VEC];
+      for (int u = 0; u < 2; ++u) {
+        const int c = c0 + u * blockDim.x;
+        if (c >= nvec) continue;
 #pragma unroll
-            for (int q = 0; q < VEC; q += 4) {
-              const int4 m4 = __ldg(reinterpret_cast<const int4*>(colmap + c * VEC + q));
-              idx[q] = m4.x; idx[q + 1] = m4.y; idx[q + 2] = m4.z; idx[q + 3] = m4.w;
-            }
+        for (int q = 0; q < 8; ++q) {
+          Word w = 0;
 #pragma unroll
-            for (int q = 0; q < VEC; ++q) row[idx[q]] = vals[q];
-          }
+          for (int r = 0; r < ROWS; ++r) w |= (Word)reinterpret_cast<const uint16_t*>(&v[u][r])[q] << (16 * r);
+          W[q * nvec + c] = w;
         }
       }
     }
     __syncthreads();
-    // Phase 2: shared memory -> 16-byte coalesced stores (gather: permuted read).
-    for (int t = threadIdx.x; t < total; t += nthr) {
-      const int rr = t / nvec, c = t - rr * nvec;
-      const T* row = buf + (long)rr * cols;
-      uint4 o;
-      if (!scatter) {
-        T vals[VEC];
+    // Store: column vector c of the output rows, each element read through the source map.
+    for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+      const uint4 ix4 = reinterpret_cast<const uint4*>(src_of)[c];
+      const uint16_t* ix = reinterpret_cast<const uint16_t*>(&ix4);
+      Word w[8];
 #pragma unroll
-        for (int q = 0; q < VEC; q += 4) {
-          const int4 m4 = __ldg(reinterpret_cast<const int4*>(colmap + c * VEC + q));
-          vals[q] = row[m4.x]; vals[q + 1] = row[m4.y]; vals[q + 2] = row[m4.z]; vals[q + 3] = row[m4.w];
-        }
-        o = *reinterpret_cast<const uint4*>(vals);
-      } else {
-        o = reinterpret_cast<const uint4*>(row)[c];
+      for (int q = 0; q < 8; ++q) w[q] = W[(ix[q] & 7) * nvec + (ix[q] >> 3)];
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        if (r >= nr) break;
+        uint16_t e[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) e[q] = (uint16_t)(w[q] >> (16 * r));
+        reinterpret_cast<uint4*>(out + (r0 + r) * ld_out)[c] = *reinterpret_cast<const uint4*>(e);
       }
-      reinterpret_cast<uint4*>(out + (r0 + rr) * ld_out)[c] = o;
     }
+    __syncthreads();
+  }
+}
+
+// fp32 variant for the fp32 path (small layers): one row at a time, staged in shared memory.
+__global__ void __launch_bounds__(256)
+    permute_cols_f32_kernel(const float* __restrict__ in, long ld_in, float* __restrict__ out, long ld_out, long rows,
+                            int cols, const int32_t* __restrict__ colmap, const int32_t* __restrict__ rowmap,
+                            int scatter) {
+  extern __shared__ __align__(16) uint8_t smem_perm[];
+  float* row = reinterpret_cast<float*>(smem_perm);
+  for (long r = blockIdx.x; r < rows; r += gridDim.x) {
+    const long rin = (!scatter && rowmap) ? (long)__ldg(rowmap + r) : r;
+    for (int j = threadIdx.x; j < cols; j += blockDim.x) {
+      const float x = __ldg(in + rin * ld_in + j);
+      if (scatter) row[__ldg(colmap + j)] = x; else row[j] = x;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < cols; j += blockDim.x)
+      out[r * ld_out + j] = scatter ? row[j] : row[__ldg(colmap + j)];
     __syncthreads();
   }
 }

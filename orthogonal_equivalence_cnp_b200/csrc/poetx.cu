@@ -76,6 +76,7 @@ struct LaunchScope {
   int cls;
   cudaStream_t st;
   cudaEvent_t e0 = nullptr, e1 = nullptr;
+  unsigned int flags = cudaEventRecordDefault;
   LaunchScope(int c, cudaStream_t s) : cls(c), st(s) {
     Profiler& p = prof();
     p.launches.fetch_add(1, std::memory_order_relaxed);
@@ -83,13 +84,17 @@ struct LaunchScope {
       std::lock_guard<std::mutex> g(p.mu);
       e0 = p.take();
       e1 = p.take();
-      if (e0 && e1) cudaEventRecord(e0, st);
+      // Under stream capture the records must be external so that they become event nodes.
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      cudaStreamIsCapturing(st, &cs);
+      flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+      if (e0 && e1) cudaEventRecordWithFlags(e0, st, flags);
     }
   }
   ~LaunchScope() {
     if (e0 && e1) {
       Profiler& p = prof();
-      cudaEventRecord(e1, st);
+      cudaEventRecordWithFlags(e1, st, flags);
       std::lock_guard<std::mutex> g(p.mu);
       p.recs.push_back({cls, {e0, e1}});
     }
@@ -106,9 +111,9 @@ poetx_status check_desc(const poetx_desc* d) {
   if (d->dtype == POETX_BF16 && b < 64) return POETX_ERR_UNSUPPORTED_SHAPE;
   if (d->k > 8) return POETX_ERR_UNSUPPORTED_SHAPE;
   if (d->d_in % b != 0 || d->d_out % b != 0) return POETX_ERR_UNSUPPORTED_SHAPE;
-  // One feature row (d * element size) must fit in a block's shared memory for the
-  // permutation kernel: at most 128 KiB.
-  const int dmax = d->dtype == POETX_BF16 ? 65536 : 32768;
+  // The permutation kernel stages up to three feature rows (d * element size each) in one
+  // block's shared memory: at most 64 KiB per row.
+  const int dmax = d->dtype == POETX_BF16 ? 32768 : 16384;
   if (d->d_in > dmax || d->d_out > dmax) return POETX_ERR_UNSUPPORTED_SHAPE;
   return POETX_OK;
 }
@@ -242,24 +247,31 @@ int ew_grid(long n) { return (int)std::min<long>((n + 255) / 256, (long)kNumSms 
 poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld_out, long rows, int cols,
                           const int32_t* colmap, const int32_t* rowmap, bool scatter, cudaStream_t st) {
   if (rows <= 0) return POETX_OK;
-  const size_t row_bytes = (size_t)cols * esize(dt);
-  int rb = (int)std::max<size_t>(1, std::min<size_t>(4, (96 * 1024) / row_bytes));
-  const size_t smem = rb * row_bytes;
-  const int grid = (int)std::min<long>((rows + rb - 1) / rb, (long)kNumSms * 8);
+  if (cols > 65536) return POETX_ERR_UNSUPPORTED_SHAPE;
   if (dt == BF16) {
-    auto k = permute_cols_kernel<__nv_bfloat16>;
-    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    // Groups of four rows (two for very wide rows); as many blocks as fit.
+    const bool four = permute_smem_bytes<4>(cols) <= 160 * 1024;
+    const size_t smem = four ? permute_smem_bytes<4>(cols) : permute_smem_bytes<2>(cols);
+    if (smem > 200 * 1024) return POETX_ERR_UNSUPPORTED_SHAPE;
+    const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (224 * 1024) / (smem + 1024)));
+    const long groups = (rows + (four ? 4 : 2) - 1) / (four ? 4 : 2);
+    const int grid = (int)std::min<long>(groups, (long)kNumSms * per_sm);
+    auto k = four ? permute_cols_bf16_kernel<4> : permute_cols_bf16_kernel<2>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return POETX_ERR_CUDA;
     LaunchScope ls(POETX_KC_PERMUTE, st);
-    k<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(in), ld_in, static_cast<__nv_bfloat16*>(out), ld_out,
-                               rows, cols, colmap, rowmap, scatter ? 1 : 0, rb);
+    k<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(in), ld_in, static_cast<uint16_t*>(out), ld_out, rows,
+                               cols, colmap, rowmap, scatter ? 1 : 0);
   } else {
-    auto k = permute_cols_kernel<float>;
-    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    const size_t smem = (size_t)cols * 4;
+    if (smem > 200 * 1024) return POETX_ERR_UNSUPPORTED_SHAPE;
+    auto k = permute_cols_f32_kernel;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return POETX_ERR_CUDA;
+    const int grid = (int)std::min<long>(rows, (long)kNumSms * 4);
     LaunchScope ls(POETX_KC_PERMUTE, st);
     k<<<grid, 256, smem, st>>>(static_cast<const float*>(in), ld_in, static_cast<float*>(out), ld_out, rows, cols,
-                               colmap, rowmap, scatter ? 1 : 0, rb);
+                               colmap, rowmap, scatter ? 1 : 0);
   }
   return last_launch();
 }
@@ -568,7 +580,7 @@ poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
-  constexpr size_t smem = tc_smem_bytes<BN, ST>();
+  constexpr size_t smem = cnp_smem_bytes<BN, ST>();
   auto kern = cnp_program_kernel<BN, ST>;
   if (!attr_done[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -757,7 +769,7 @@ FwdPlan fwd_plan(const poetx_desc* d, long n) {
   const size_t e = esize(d->dtype);
   Plan p;
   FwdPlan f;
-  f.U = p.take(n * d->d_in * e);
+  f.U = d->mode == POETX_MEM ? p.take(n * d->d_in * e) : 0;
   f.V = p.take(n * d->d_in * e);
   f.Yp = p.take(n * d->d_out * e);
   f.Z = d->mode == POETX_MEM ? p.take(n * d->d_out * e) : 0;
@@ -777,7 +789,7 @@ BwdPlan bwd_plan(const poetx_desc* d, long n) {
   w.dYp = p.take(n * d->d_out * e);
   w.dZ = p.take(n * d->d_out * e);
   w.dV = p.take(n * d->d_in * e);
-  w.U = p.take(n * d->d_in * e);
+  w.U = d->mode == POETX_MEM ? p.take(n * d->d_in * e) : 0;
   w.dU = p.take(n * d->d_in * e);
   w.V = d->mode == POETX_MEM ? p.take(n * d->d_in * e) : 0;
   w.Z = d->mode == POETX_MEM ? p.take(n * d->d_out * e) : 0;
@@ -950,30 +962,33 @@ poetx_status poetx_absorb(const poetx_desc* desc, const void* W0, const int32_t*
 
 poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
                            const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P, void* Y,
-                           void* Z_saved, void* workspace, size_t ws_bytes, poetx_stream stream) {
+                           void* saved, void* workspace, size_t ws_bytes, poetx_stream stream) {
   POETX_TRY(check_desc(desc));
   if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
   if (n_tokens == 0) return POETX_OK;
-  if (desc->mode == POETX_FAST && Z_saved == nullptr) return POETX_ERR_INVALID_ARG;
-  if (desc->mode == POETX_MEM && Z_saved != nullptr) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_FAST && saved == nullptr) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_MEM && saved != nullptr) return POETX_ERR_INVALID_ARG;
   POETX_TRY(check_ptrs({X, W0p, perm_L, perm_R, Q_R, Q_P, Y}));
-  if (Z_saved != nullptr && !aligned16(Z_saved)) return POETX_ERR_ALIGNMENT;
+  if (saved != nullptr && !aligned16(saved)) return POETX_ERR_ALIGNMENT;
   const FwdPlan f = fwd_plan(desc, n_tokens);
   POETX_TRY(check_ws(workspace, ws_bytes, f.total));
   char* ws = static_cast<char*>(workspace);
-  void* Z = desc->mode == POETX_FAST ? Z_saved : ws + f.Z;
-  return forward_chain(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, Z, ws + f.U, ws + f.V, ws + f.Yp, stream);
+  // POET-Xfast keeps Z = V.W0'^T and U = X[:, pi_R] for the backward pass (in `saved`).
+  const size_t zbytes = (size_t)n_tokens * desc->d_out * esize(desc->dtype);
+  void* Z = desc->mode == POETX_FAST ? saved : ws + f.Z;
+  char* U = desc->mode == POETX_FAST ? static_cast<char*>(saved) + zbytes : ws + f.U;
+  return forward_chain(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, Z, U, ws + f.V, ws + f.Yp, stream);
 }
 
 poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X, const void* W0p,
                             const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
-                            const float* theta_R, const float* theta_P, const void* Z_saved, void* dX,
+                            const float* theta_R, const float* theta_P, const void* saved, void* dX,
                             float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
                             poetx_stream stream) {
   POETX_TRY(check_desc(desc));
   if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
-  if (desc->mode == POETX_FAST && Z_saved == nullptr && n_tokens > 0) return POETX_ERR_INVALID_ARG;
-  if (desc->mode == POETX_MEM && Z_saved != nullptr) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_FAST && saved == nullptr && n_tokens > 0) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_MEM && saved != nullptr) return POETX_ERR_INVALID_ARG;
   POETX_TRY(check_ptrs({theta_R, theta_P, grad_theta_R, grad_theta_P}));
   const int b = desc->b, dt = desc->dtype, nbo = desc->d_out / b, nbi = desc->d_in / b;
   const size_t P = (size_t)b * (b - 1) / 2;
@@ -983,14 +998,15 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
     return POETX_OK;
   }
   POETX_TRY(check_ptrs({dY, X, W0p, perm_L, perm_R, Q_R, Q_P, dX}));
-  if (Z_saved != nullptr && !aligned16(Z_saved)) return POETX_ERR_ALIGNMENT;
+  if (saved != nullptr && !aligned16(saved)) return POETX_ERR_ALIGNMENT;
   const BwdPlan w = bwd_plan(desc, n_tokens);
   POETX_TRY(check_ws(workspace, ws_bytes, w.total));
   char* ws = static_cast<char*>(workspace);
   const long n = n_tokens;
   const int din = desc->d_in, dout = desc->d_out;
 
-  const void* Z = Z_saved;
+  const void* Z = saved;  // fast mode: Z then U = X[:, pi_R], both kept by the forward pass
+  const char* U = desc->mode == POETX_FAST ? static_cast<const char*>(saved) + (size_t)n * dout * esize(dt) : ws + w.U;
   if (desc->mode == POETX_MEM) {
     // POET-Xmem: recompute U = X[:, pi_R], V = BD_P.U and Z = V.W0'^T from X.
     POETX_TRY(forward_chain(desc, n, X, W0p, perm_L, perm_R, Q_R, Q_P, nullptr, ws + w.Z, ws + w.U, ws + w.V,
@@ -1010,10 +1026,8 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
     g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
     POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM));
   }
-  // Input side: U = X[:, pi_R] (already there in mem mode); G_P partials; dU; dX[:, pi_R] = dU.
-  if (desc->mode == POETX_FAST)
-    POETX_TRY(permute_cols(dt, X, din, ws + w.U, din, n, din, perm_R, nullptr, false, stream));
-  POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, ws + w.U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
+  // Input side: G_P partials (U saved or recomputed); dU; dX[:, pi_R] = dU.
+  POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
   POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
   POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, stream));
   // CNP adjoint, packed gradients only.

@@ -39,7 +39,8 @@ class PoetxLayer:
         self.Q_R = torch.empty(dout // b, b, b, dtype=dt, device=dev)
         self.Q_P = torch.empty(din // b, b, b, dtype=dt, device=dev)
         self.Y = torch.empty(self.n, dout, dtype=dt, device=dev)
-        self.Z = torch.empty(self.n, dout, dtype=dt, device=dev) if desc.mode == POETX_FAST else None
+        # POET-Xfast keeps Z [N, d_out] and U = X[:, pi_R] [N, d_in] for the backward pass.
+        self.saved = torch.empty(self.n * (dout + din), dtype=dt, device=dev) if desc.mode == POETX_FAST else None
         self.dX = torch.empty(self.n, din, dtype=dt, device=dev)
         self.g_R = torch.empty_like(self.theta_R)
         self.g_P = torch.empty_like(self.theta_P)
@@ -66,12 +67,12 @@ class PoetxLayer:
 
     def forward(self, X: torch.Tensor):
         poetx_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
-                      self.Z, self.ws)
+                      self.saved, self.ws)
         return self.Y
 
     def backward(self, dY: torch.Tensor, X: torch.Tensor):
         poetx_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
-                       self.theta_R, self.theta_P, self.Z, self.dX, self.g_R, self.g_P, self.ws)
+                       self.theta_R, self.theta_P, self.saved, self.dX, self.g_R, self.g_P, self.ws)
         return self.dX, self.g_R, self.g_P
 
     def step(self, X: torch.Tensor, dY: torch.Tensor):

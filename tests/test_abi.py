@@ -68,7 +68,7 @@ def test_null_misaligned_and_workspace_errors():
     # workspace too small / missing
     assert L.poetx_forward(ctypes.byref(d), 64, A, A, A, A, A, A, A, A, A, 1024, None) == 4
     assert L.poetx_forward(ctypes.byref(d), 64, A, A, A, A, A, A, A, A, None, ws, None) == 4
-    # mode / Z_saved mismatch
+    # mode / saved-buffer mismatch
     assert L.poetx_forward(ctypes.byref(d), 64, A, A, A, A, A, A, A, None, A, ws, None) == 1
     dm = _desc(mode=P.POETX_MEM)
     assert L.poetx_forward(ctypes.byref(dm), 64, A, A, A, A, A, A, A, A, A, ws, None) == 1
