@@ -326,8 +326,22 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         // G = sum of split-K partials -> T1, row walk with one float4 per lane per row.
         const long sstride = (long)S.nb * b * b;
         constexpr int RB = 4;
+        if (S.splits == 1) {
+          // One partial (the gradient GEMM did not split K): all of a warp's rows in flight.
+          float4 ld4[RW];
+#pragma unroll
+          for (int t = 0; t < RW; ++t) {
+            const int ii = m0 + warp + 8 * t;
+            ld4[t] = (ii < b && lane * 4 < BN)
+                         ? __ldg(reinterpret_cast<const float4*>(S.part + ((long)z * b + ii) * b + n0) + lane)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int t = 0; t < RW; ++t)
+            if (lane * 4 < BN) *reinterpret_cast<float4*>(T1 + (warp + 8 * t) * TS + lane * 4) = ld4[t];
+        }
 #pragma unroll 1
-        for (int t0 = 0; t0 < RW; t0 += RB) {
+        for (int t0 = 0; t0 < (S.splits == 1 ? 0 : RW); t0 += RB) {
           float4 acc4[RB];
 #pragma unroll
           for (int t = 0; t < RB; ++t) acc4[t] = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -304,6 +304,199 @@ __global__ void __launch_bounds__(128)
   if (warp == 0) tmem_dealloc(tmem_d, BN);
 }
 
+// ------------------------------------------------- W0' GEMM fused with a block-diagonal factor
+// One 128 x 256 output tile of D = A . B^T (A K-major, B K- or MN-major) where the 256 columns
+// are exactly one b = 256 block; after the K loop the tile is (a) stored (bf16, optional) and
+// (b) written as bf16 into the idle TMA ring in the 128-byte-swizzled K-major layout, where it
+// is the A operand of a second tcgen05 product with that block's Q (K-major: out2 = D . Q^T,
+// forward BD_R; MN-major: out2 = D . Q, adjoint of BD_P).  Two accumulators share TMEM
+// (columns 0..255 and 256..511).  This removes a separate block-diagonal launch and its read
+// of D.  All waits bounded; every thread reaches every barrier.
+struct FuseArgs {
+  int M, N, K;
+  void* d1;       // bf16 [M, N] store of D (may be null)
+  long ld1;
+  void* out2;     // bf16 [M, N] result of the block-diagonal factor
+  long ld2;
+};
+
+template <bool B_MN, bool Q_MN>
+__global__ void __launch_bounds__(128, 1)
+    gemm_bd_fused_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmQ, const FuseArgs args) {
+  constexpr int BN = 256, STAGES = 4;
+  constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
+  constexpr uint32_t B_BYTES = BN * TC_BK * 2;
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t IDESC = sm100::idesc_bf16_f32(TC_BM, BN, false, B_MN);
+  constexpr uint32_t IDESC2 = sm100::idesc_bf16_f32(TC_BM, BN, false, Q_MN);
+  using namespace sm100;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  const uint32_t smem0 = smem_u32(smem);
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
+  const uint32_t q_full = smem_u32(bars + 2 * STAGES + 1);
+  const uint32_t acc2_bar = smem_u32(bars + 2 * STAGES + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * TC_BM, n0 = blockIdx.x * BN;
+  const int zq = blockIdx.x;  // the b = 256 block this tile's columns form
+  const int nkt = (args.K + TC_BK - 1) / TC_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(accum_bar, 1);
+    mbar_init(q_full, 1);
+    mbar_init(acc2_bar, 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmQ);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer: the K loop, then this block's Q into the ring's B halves.
+    bool ok = true;
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 5)) { ok = false; break; }
+      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+      const int k0 = i * TC_BK;
+      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+      tma_load_2d(sa, &tmA, full_bar(s), k0, m0);
+      if (!B_MN) {
+        tma_load_2d(sb, &tmB, full_bar(s), k0, n0);
+      } else {
+#pragma unroll
+        for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmB, full_bar(s), n0 + 64 * h, k0);
+      }
+    }
+    // The ring is free once every MMA of the K loop has completed.
+    if (ok && mbar_wait(accum_bar, 0, KID_GEMM_TC, 6)) {
+      mbar_arrive_expect_tx(q_full, STAGES * B_BYTES);
+#pragma unroll
+      for (int t = 0; t < STAGES; ++t) {
+        const uint32_t sb = smem0 + t * STAGE_BYTES + A_BYTES;
+        if (!Q_MN) {
+          tma_load_2d(sb, &tmQ, q_full, 64 * t, zq * BN);
+        } else {
+#pragma unroll
+          for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmQ, q_full, 64 * h, zq * BN + 64 * t);
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer: the K loop
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (!mbar_wait(full_bar(s), ph, KID_GEMM_TC, 7)) break;
+      tc_fence_after();
+      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk) {
+        const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+        const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+        mma_bf16(tmem_d, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(empty_bar(s));
+    }
+    mma_commit(accum_bar);
+  }
+  __syncwarp();
+
+  // ---------------- phase 1: D (TMEM) -> bf16 -> global d1 and the swizzled A tiles in the ring
+  bool ok = mbar_wait(accum_bar, 0, KID_GEMM_TC, 8);
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after();
+  const int r = warp * 32 + lane;  // tile row
+  const int m = m0 + r;
+  if (ok) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+      tmem_wait_ld();
+      uint4 q[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        q[u] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1])),
+                          pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+                          pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+                          pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+      if (args.d1 != nullptr && m < args.M) {
+        uint4* g = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(args.d1) + (long)m * args.ld1 + n0 + c);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) g[u] = q[u];
+      }
+      // K-major 128-byte swizzle: 16-byte chunk ch of row r sits at chunk position ch ^ (r % 8).
+      uint8_t* tileA = smem + (c / 64) * STAGE_BYTES + r * 128;
+      const int ch0 = (c % 64) / 8;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(tileA + (((ch0 + u) ^ (r & 7)) * 16)) = q[u];
+    }
+  }
+  fence_proxy_async_smem();  // the tensor core reads what the threads just wrote
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---------------- phase 2: out2 = D_tile . Q_block (second accumulator, TMEM columns 256..511)
+  if (warp == 1 && lane == 0 && ok) {
+    if (mbar_wait(q_full, 0, KID_GEMM_TC, 9)) {
+      tc_fence_after();
+#pragma unroll
+      for (int t = 0; t < STAGES; ++t) {
+        const uint32_t sa = smem0 + t * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < TC_BK / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+          const uint64_t bd = Q_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+          mma_bf16(tmem_d + BN, ad, bd, IDESC2, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+    }
+    mma_commit(acc2_bar);
+  }
+  __syncwarp();
+  bool ok2 = ok && mbar_wait(acc2_bar, 0, KID_GEMM_TC, 10);
+  ok2 = __all_sync(0xffffffffu, ok2);
+  tc_fence_after();
+  if (ok2) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(warp * 32) << 16) + (uint32_t)(BN + c), v);
+      tmem_wait_ld();
+      float f[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+      if (m < args.M) store32(args.out2, (long)m * args.ld2 + n0 + c, BF16, f);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem_d, 2 * BN);
+}
+
 // ---------------------------------------------------------------------------- f32 SIMT kernel
 struct SimtArgs {
   int M, N, K, splits;

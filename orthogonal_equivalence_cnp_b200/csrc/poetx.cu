@@ -44,6 +44,15 @@ struct Plan {
     if (_s != POETX_OK) return _s;       \
   } while (0)
 
+// Opts a kernel into `smem` bytes of dynamic shared memory and the largest shared-memory carveout
+// (the default carveout can leave room for fewer resident blocks than the shared memory allows).
+template <typename K>
+inline bool set_smem(K kern, size_t smem) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess &&
+         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+}
+
 inline poetx_status last_launch() {
   return cudaGetLastError() == cudaSuccess ? POETX_OK : POETX_ERR_CUDA;
 }
@@ -188,8 +197,7 @@ poetx_status launch_tc(const GemmDesc& g, cudaStream_t st, int cls) {
   constexpr size_t smem = tc_smem_bytes<BN, ST>();
   auto kern = gemm_bf16_tc<BN, ST, AMN, BMN>;
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return POETX_ERR_CUDA;
+    if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
   CUtensorMap ta, tb;
@@ -217,16 +225,17 @@ poetx_status run_gemm(int dt, const GemmDesc& g, cudaStream_t st, int cls) {
   POETX_TRY(check_gemm(g, dt));
   if (dt == BF16) {
     // Long K (>= 16 k-tiles per CTA): deep ring, one CTA per SM, widest tile.  Short K: a
-    // 96 KiB ring so two CTAs share an SM (one's epilogue overlaps the other's loads), and the
-    // widest tile that still gives at least two CTAs per SM.
+    // 96 KiB ring so two CTAs share an SM (one's epilogue overlaps the other's loads); the
+    // full 256-column tile (A read once) as long as it still fills 1.5 CTAs per SM.
     const long kt = ((long)(g.K + TC_BK - 1) / TC_BK) / g.splits;
     const long base = (long)((g.M + TC_BM - 1) / TC_BM) * g.batch * g.splits;
     if (kt >= 16) {
-      if (g.N % 256 == 0) return launch_tc_major<256, 4>(g, st, cls);
-      if (g.N % 128 == 0) return launch_tc_major<128, 6>(g, st, cls);
+      // The widest tile that still occupies three quarters of the SMs.
+      if (g.N % 256 == 0 && 4 * base * (g.N / 256) >= 3 * kNumSms) return launch_tc_major<256, 4>(g, st, cls);
+      if (g.N % 128 == 0 && 4 * base * (g.N / 128) >= 3 * kNumSms) return launch_tc_major<128, 6>(g, st, cls);
       return launch_tc_major<64, 8>(g, st, cls);
     }
-    if (g.N % 256 == 0 && base * (g.N / 256) >= 2 * kNumSms) return launch_tc_major<256, 2>(g, st, cls);
+    if (g.N % 256 == 0 && 2 * base * (g.N / 256) >= 3 * kNumSms) return launch_tc_major<256, 2>(g, st, cls);
     if (g.N % 128 == 0 && base * (g.N / 128) >= 2 * kNumSms) return launch_tc_major<128, 3>(g, st, cls);
     return launch_tc_major<64, 4>(g, st, cls);
   }
@@ -248,17 +257,19 @@ poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld
                           const int32_t* colmap, const int32_t* rowmap, bool scatter, cudaStream_t st) {
   if (rows <= 0) return POETX_OK;
   if (cols > 65536) return POETX_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(colmap)) return POETX_ERR_ALIGNMENT;
   if (dt == BF16) {
     // Groups of four rows (two for very wide rows); as many blocks as fit.
     const bool four = permute_smem_bytes<4>(cols) <= 160 * 1024;
     const size_t smem = four ? permute_smem_bytes<4>(cols) : permute_smem_bytes<2>(cols);
     if (smem > 200 * 1024) return POETX_ERR_UNSUPPORTED_SHAPE;
-    const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (224 * 1024) / (smem + 1024)));
     const long groups = (rows + (four ? 4 : 2) - 1) / (four ? 4 : 2);
-    const int grid = (int)std::min<long>(groups, (long)kNumSms * per_sm);
     auto k = four ? permute_cols_bf16_kernel<4> : permute_cols_bf16_kernel<2>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (!set_smem(k, smem)) return POETX_ERR_CUDA;
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, smem) != cudaSuccess || per_sm < 1)
       return POETX_ERR_CUDA;
+    const int grid = (int)std::min<long>(groups, (long)kNumSms * per_sm);
     LaunchScope ls(POETX_KC_PERMUTE, st);
     k<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(in), ld_in, static_cast<uint16_t*>(out), ld_out, rows,
                                cols, colmap, rowmap, scatter ? 1 : 0);
@@ -266,8 +277,7 @@ poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld
     const size_t smem = (size_t)cols * 4;
     if (smem > 200 * 1024) return POETX_ERR_UNSUPPORTED_SHAPE;
     auto k = permute_cols_f32_kernel;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return POETX_ERR_CUDA;
+    if (!set_smem(k, smem)) return POETX_ERR_CUDA;
     const int grid = (int)std::min<long>(rows, (long)kNumSms * 4);
     LaunchScope ls(POETX_KC_PERMUTE, st);
     k<<<grid, 256, smem, st>>>(static_cast<const float*>(in), ld_in, static_cast<float*>(out), ld_out, rows, cols,
@@ -310,6 +320,49 @@ Operand view(const void* base, long rows, long cols, long ld, long zrow = 0, lon
   return o;
 }
 
+// W0' GEMM fused with the following block-diagonal factor (b = 256 only): out2 = D . Q^T
+// (q_mn = false, forward BD_R) or D . Q (q_mn = true, adjoint of BD_P), D also stored to d1.
+bool bd_fusable(int dt, int b, const GemmDesc& g) {
+  return dt == BF16 && b == 256 && !g.a_mn && g.N % 256 == 0 && g.batch == 1 && g.splits == 1 && g.K > 0;
+}
+
+template <bool BMN, bool QMN>
+poetx_status launch_bd_fused(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st) {
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
+  constexpr size_t smem = tc_smem_bytes<256, 4>();
+  auto kern = gemm_bd_fused_tc<BMN, QMN>;
+  if (!attr_done[dev]) {
+    if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  CUtensorMap ta, tb, tq;
+  if (!make_tmap(&ta, g.A, 64, TC_BM)) return POETX_ERR_CUDA;
+  if (!make_tmap(&tb, g.B, 64, BMN ? 64 : 256)) return POETX_ERR_CUDA;
+  if (!make_tmap(&tq, view(Q, q_rows, 256, 256), 64, QMN ? 64 : 256)) return POETX_ERR_CUDA;
+  FuseArgs a;
+  a.M = g.M; a.N = g.N; a.K = g.K;
+  a.d1 = g.epi.d1; a.ld1 = g.epi.ld1;
+  a.out2 = out2; a.ld2 = ld2;
+  dim3 grid(g.N / 256, (g.M + TC_BM - 1) / TC_BM, 1);
+  LaunchScope ls(POETX_KC_W_GEMM, st);
+  kern<<<grid, 128, smem, st>>>(ta, tb, tq, a);
+  return last_launch();
+}
+
+poetx_status run_gemm_bd_fused(const GemmDesc& g, const void* Q, long q_rows, bool q_mn, void* out2, long ld2,
+                               cudaStream_t st) {
+  POETX_TRY(check_gemm(g, BF16));
+  if (q_rows < g.N || !aligned16(Q) || !aligned16(out2) || ld2 % 8) return POETX_ERR_ALIGNMENT;
+  const Epilogue& e = g.epi;
+  if (e.d1 && (e.d1_dtype != BF16 || e.alpha1 != 1.f || e.c || e.d2 || e.diag1 || e.split_stride1)) return POETX_ERR_INVALID_ARG;
+  if (!g.b_mn && !q_mn) return launch_bd_fused<false, false>(g, Q, q_rows, out2, ld2, st);
+  if (!g.b_mn && q_mn) return launch_bd_fused<false, true>(g, Q, q_rows, out2, ld2, st);
+  if (g.b_mn && !q_mn) return launch_bd_fused<true, false>(g, Q, q_rows, out2, ld2, st);
+  return launch_bd_fused<true, true>(g, Q, q_rows, out2, ld2, st);
+}
+
 // Out[:, blk z] = In[:, blk z] . Q_z^T  (forward block-diagonal application; tokens are rows).
 poetx_status bd_forward(int dt, long n, int d, int b, const void* in, const void* Q, void* out, cudaStream_t st) {
   GemmDesc g;
@@ -332,8 +385,10 @@ poetx_status bd_backward(int dt, long n, int d, int b, const void* in, const voi
 }
 
 // Gpart[s][z] = Lhs[:, blk z]^T . Rhs[:, blk z] over split s of the tokens (f32 partials).
+// Split-K factor of the block-gradient GEMMs: enough CTAs of 128 x 64 tiles (bf16) to fill the
+// SMs, and no split at all when the tiles alone do (the CNP adjoint then reads one partial).
 int grad_splits(int dt, long n, int nb, int b) {
-  const long tiles = dt == BF16 ? (long)nb * ((b + 127) / 128) * (b >= 256 ? b / 256 : 1)
+  const long tiles = dt == BF16 ? (long)nb * ((b + 127) / 128) * ((b + 63) / 64)
                                 : (long)nb * ((b + 63) / 64) * ((b + 63) / 64);
   const long kt = dt == BF16 ? (n + 63) / 64 : (n + 15) / 16;
   long s = std::max<long>(1, kNumSms / std::max<long>(1, tiles));
@@ -583,8 +638,7 @@ poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_
   constexpr size_t smem = cnp_smem_bytes<BN, ST>();
   auto kern = cnp_program_kernel<BN, ST>;
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return POETX_ERR_CUDA;
+    if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
   if (nb_total > 65535) return POETX_ERR_UNSUPPORTED_SHAPE;
@@ -847,16 +901,19 @@ poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const voi
   const int dt = d->dtype, b = d->b;
   POETX_TRY(permute_cols(dt, X, d->d_in, U, d->d_in, n, d->d_in, pR, nullptr, false, st));
   POETX_TRY(bd_forward(dt, n, d->d_in, b, U, QP, V, st));
-  {
-    GemmDesc g;
-    g.M = (int)n; g.N = d->d_out; g.K = d->d_in;
-    g.A = view(V, n, d->d_in, d->d_in);
-    g.B = view(W0p, d->d_out, d->d_in, d->d_in);
-    g.epi.d1 = Z; g.epi.d1_dtype = dt; g.epi.ld1 = d->d_out;
+  GemmDesc g;
+  g.M = (int)n; g.N = d->d_out; g.K = d->d_in;
+  g.A = view(V, n, d->d_in, d->d_in);
+  g.B = view(W0p, d->d_out, d->d_in, d->d_in);
+  g.epi.d1 = Z; g.epi.d1_dtype = dt; g.epi.ld1 = d->d_out;
+  if (Y == nullptr) return run_gemm(dt, g, st, POETX_KC_W_GEMM);  // recompute only (mem-mode backward)
+  if (bd_fusable(dt, b, g)) {
+    // Z = V.W0'^T and Y'_i = Z_i.Q_R,i^T in one kernel.
+    POETX_TRY(run_gemm_bd_fused(g, QR, d->d_out, false, Yp, d->d_out, st));
+  } else {
     POETX_TRY(run_gemm(dt, g, st, POETX_KC_W_GEMM));
+    POETX_TRY(bd_forward(dt, n, d->d_out, b, Z, QR, Yp, st));
   }
-  if (Y == nullptr) return POETX_OK;  // recompute only (mem-mode backward)
-  POETX_TRY(bd_forward(dt, n, d->d_out, b, Z, QR, Yp, st));
   return permute_cols(dt, Yp, d->d_out, Y, d->d_out, n, d->d_out, pL, nullptr, true, st);
 }
 
@@ -1017,18 +1074,18 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
   POETX_TRY(permute_cols(dt, dY, dout, ws + w.dYp, dout, n, dout, perm_L, nullptr, false, stream));
   POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, stream));
   POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
-  // dV = dZ . W0'
-  {
-    GemmDesc g;
-    g.M = (int)n; g.N = din; g.K = dout;
-    g.A = view(ws + w.dZ, n, dout, dout);
-    g.B = view(W0p, dout, din, din); g.b_mn = true;
-    g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
-    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM));
-  }
+  // dV = dZ . W0' (and, for b = 256, dU_i = dV_i . Q_P,i in the same kernel)
+  GemmDesc g;
+  g.M = (int)n; g.N = din; g.K = dout;
+  g.A = view(ws + w.dZ, n, dout, dout);
+  g.B = view(W0p, dout, din, din); g.b_mn = true;
+  g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
+  const bool fused_du = bd_fusable(dt, b, g);
+  if (fused_du) POETX_TRY(run_gemm_bd_fused(g, Q_P, din, true, ws + w.dU, din, stream));
+  else POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM));
   // Input side: G_P partials (U saved or recomputed); dU; dX[:, pi_R] = dU.
   POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
-  POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
+  if (!fused_du) POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
   POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, stream));
   // CNP adjoint, packed gradients only.
   if (cnp_fused_ok(b, dt)) {

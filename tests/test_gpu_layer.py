@@ -107,6 +107,7 @@ def test_layer_f32_orders(k):
 
 
 @pytest.mark.parametrize("d_in,d_out,b,n", [(512, 384, 128, 300), (256, 512, 64, 130), (1024, 768, 256, 200),
+                                            (512, 1280, 256, 333), (512, 512, 256, 600),
                                             (1024, 1024, 512, 129)])
 @pytest.mark.parametrize("mode", ["fast", "mem"])
 def test_layer_bf16_small(d_in, d_out, b, n, mode):
