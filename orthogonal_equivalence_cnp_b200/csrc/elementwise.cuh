@@ -33,7 +33,7 @@ __host__ __device__ constexpr size_t permute_smem_bytes(int cols) {
 }
 
 template <int ROWS>
-__global__ void __launch_bounds__(256, ROWS == 4 ? 4 : 2)
+__global__ void __launch_bounds__(256, ROWS == 4 ? 3 : 2)
     permute_cols_bf16_kernel(const uint16_t* __restrict__ in, long ld_in, uint16_t* __restrict__ out, long ld_out,
                              long rows, int cols, const int32_t* __restrict__ colmap,
                              const int32_t* __restrict__ rowmap, int scatter) {
@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(256, ROWS == 4 ? 4 : 2)
   uint16_t* src_of = reinterpret_cast<uint16_t*>(smem_perm);  // output column j reads source column src_of[j]
   Word* W = reinterpret_cast<Word*>(smem_perm + ((size_t)cols * 2 + 15) / 16 * 16);
   const int nvec = cols / 8;
-  {
+  auto build_map = [&]() {
     // The map is read with 16-byte loads, four per thread in flight (cols % 8 == 0, 16-byte
     // aligned map), so building it costs about one L2 round trip.
     const int n4 = cols / 4;
@@ -65,43 +65,48 @@ __global__ void __launch_bounds__(256, ROWS == 4 ? 4 : 2)
         }
       }
     }
-  }
-  __syncthreads();
+  };
   const long ngroups = (rows + ROWS - 1) / ROWS;
-  for (long g = blockIdx.x; g < ngroups; g += gridDim.x) {
+  // Source rows of group g (a short last group repeats its last row; only nr rows are stored).
+  auto group_rows = [&](long g, long (&src_row)[ROWS]) {
     const long r0 = g * ROWS;
     const int nr = (int)min((long)ROWS, rows - r0);
-    long src_row[ROWS];
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
-      const long rr = r0 + min(r, nr - 1);  // a short group repeats its last row
+      const long rr = r0 + min(r, nr - 1);
       src_row[r] = (!scatter && rowmap) ? (long)__ldg(rowmap + rr) : rr;
     }
-    // Load: 8 columns of each row per thread, two column vectors in flight per thread.
-    for (int c0 = threadIdx.x; c0 < nvec; c0 += blockDim.x * 2) {
-      uint4 v[2][ROWS];
+  };
+  // 8 columns of each row per thread, column vectors c0 and c0 + blockDim.x.
+  auto load = [&](long g, int c0, uint4 (&v)[2][ROWS]) {
+    long src_row[ROWS];
+    group_rows(g, src_row);
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-          const int c = c0 + u * blockDim.x;
-          if (c < nvec) v[u][r] = __ldg(reinterpret_cast<const uint4*>(in + src_row[r] * ld_in) + c);
-        }
+      for (int r = 0; r < ROWS; ++r) {
+        const int c = c0 + u * (int)blockDim.x;
+        if (c < nvec) v[u][r] = __ldg(reinterpret_cast<const uint4*>(in + src_row[r] * ld_in) + c);
+      }
+  };
+  auto put = [&](int c0, const uint4 (&v)[2][ROWS]) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = c0 + u * blockDim.x;
-        if (c >= nvec) continue;
+    for (int u = 0; u < 2; ++u) {
+      const int c = c0 + u * (int)blockDim.x;
+      if (c >= nvec) continue;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          Word w = 0;
+      for (int q = 0; q < 8; ++q) {
+        Word w = 0;
 #pragma unroll
-          for (int r = 0; r < ROWS; ++r) w |= (Word)reinterpret_cast<const uint16_t*>(&v[u][r])[q] << (16 * r);
-          W[q * nvec + c] = w;
-        }
+        for (int r = 0; r < ROWS; ++r) w |= (Word)reinterpret_cast<const uint16_t*>(&v[u][r])[q] << (16 * r);
+        W[q * nvec + c] = w;
       }
     }
-    __syncthreads();
-    // Store: column vector c of the output rows, each element read through the source map.
+  };
+  // Column vector c of the output rows, each element read through the source map.
+  auto store = [&](long g) {
+    const long r0 = g * ROWS;
+    const int nr = (int)min((long)ROWS, rows - r0);
     for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
       const uint4 ix4 = reinterpret_cast<const uint4*>(src_of)[c];
       const uint16_t* ix = reinterpret_cast<const uint16_t*>(&ix4);
@@ -117,6 +122,35 @@ __global__ void __launch_bounds__(256, ROWS == 4 ? 4 : 2)
         reinterpret_cast<uint4*>(out + (r0 + r) * ld_out)[c] = *reinterpret_cast<const uint4*>(e);
       }
     }
+  };
+
+  if (nvec <= 2 * (int)blockDim.x) {
+    // A whole group fits in two vectors per thread: software pipeline across groups.  The first
+    // group's loads are in flight while the map is built, and each next group's loads while the
+    // current group is gathered and stored, so HBM sees reads and writes at the same time.
+    uint4 v[2][ROWS];
+    long g = blockIdx.x;
+    if (g < ngroups) load(g, threadIdx.x, v);
+    build_map();
+    for (; g < ngroups; g += gridDim.x) {
+      put(threadIdx.x, v);
+      __syncthreads();  // W (and, the first time, the map) complete
+      if (g + gridDim.x < ngroups) load(g + gridDim.x, threadIdx.x, v);
+      store(g);
+      __syncthreads();  // W free again
+    }
+    return;
+  }
+  build_map();
+  __syncthreads();
+  for (long g = blockIdx.x; g < ngroups; g += gridDim.x) {
+    for (int c0 = threadIdx.x; c0 < nvec; c0 += blockDim.x * 2) {
+      uint4 v[2][ROWS];
+      load(g, c0, v);
+      put(c0, v);
+    }
+    __syncthreads();
+    store(g);
     __syncthreads();
   }
 }

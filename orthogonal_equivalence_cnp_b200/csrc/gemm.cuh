@@ -389,12 +389,16 @@ __global__ void __launch_bounds__(128, 1)
         for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmB, full_bar(s), n0 + 64 * h, k0);
       }
     }
-    // The ring is free once every MMA of the K loop has completed.
-    if (ok && mbar_wait(accum_bar, 0, KID_GEMM_TC, 6)) {
+    // Q's four 64-wide K chunks follow the K loop through the ring as if they were iterations
+    // nkt .. nkt+3: each lands in the B half of its stage as soon as the last MMA reading that
+    // stage has completed, so the load overlaps the tail of the K loop.
+    if (ok) {
       mbar_arrive_expect_tx(q_full, STAGES * B_BYTES);
-#pragma unroll
       for (int t = 0; t < STAGES; ++t) {
-        const uint32_t sb = smem0 + t * STAGE_BYTES + A_BYTES;
+        const int v = nkt + t;
+        const int s = v % STAGES;
+        if (!mbar_wait(empty_bar(s), ((uint32_t)(v / STAGES) & 1u) ^ 1u, KID_GEMM_TC, 6)) break;
+        const uint32_t sb = smem0 + s * STAGE_BYTES + A_BYTES;
         if (!Q_MN) {
           tma_load_2d(sb, &tmQ, q_full, 64 * t, zq * BN);
         } else {
@@ -448,7 +452,8 @@ __global__ void __launch_bounds__(128, 1)
         for (int u = 0; u < 4; ++u) g[u] = q[u];
       }
       // K-major 128-byte swizzle: 16-byte chunk ch of row r sits at chunk position ch ^ (r % 8).
-      uint8_t* tileA = smem + (c / 64) * STAGE_BYTES + r * 128;
+      // K chunk t of D goes to the A half of the stage that holds Q's chunk t.
+      uint8_t* tileA = smem + ((nkt + c / 64) % STAGES) * STAGE_BYTES + r * 128;
       const int ch0 = (c % 64) / 8;
 #pragma unroll
       for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(tileA + (((ch0 + u) ^ (r & 7)) * 16)) = q[u];
@@ -465,7 +470,7 @@ __global__ void __launch_bounds__(128, 1)
       tc_fence_after();
 #pragma unroll
       for (int t = 0; t < STAGES; ++t) {
-        const uint32_t sa = smem0 + t * STAGE_BYTES, sb = sa + A_BYTES;
+        const uint32_t sa = smem0 + ((nkt + t) % STAGES) * STAGE_BYTES, sb = sa + A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < TC_BK / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
@@ -491,6 +496,231 @@ __global__ void __launch_bounds__(128, 1)
       for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
       if (m < args.M) store32(args.out2, (long)m * args.ld2 + n0 + c, BF16, f);
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem_d, 2 * BN);
+}
+
+// ----------------------------------------- W0' GEMM, 256 x 256 tiles, optional block factor
+// One CTA computes a 256 x 256 tile of D = A . B^T (A K-major, B K- or MN-major) as two M = 128
+// halves sharing every B tile: per 64-wide k step it issues eight tcgen05.mma (2 halves x 4
+// K=16 steps) into two TMEM accumulators (columns 0..255 and 256..511).  Against a 128 x 256
+// tile this halves the B bytes per FLOP and doubles the MMA time covered by each ring stage
+// (3 stages of 64 KiB), which is what keeps the tensor pipe fed from L2.  With out2 set (b = 256:
+// the tile's columns are one block) each half is then written as bf16 into the idle ring in the
+// swizzled K-major layout and multiplied by the block's Q (K-major: D . Q^T, forward BD_R;
+// MN-major: D . Q, adjoint of BD_P), reusing the half's own TMEM columns once drained.  Q's
+// four 64-wide K chunks follow the K loop through the ring (two per stage); the D half uses the
+// third stage.  All waits bounded; every thread reaches every barrier.
+struct WideArgs {
+  int M, N, K;
+  void* d1;    // bf16 [M, N] store of D (may be null when out2 is set)
+  long ld1;
+  void* out2;  // bf16 [M, N] block-factor result, or null (plain GEMM)
+  long ld2;
+};
+
+constexpr int TCW_BM = 256, TCW_BN = 256, TCW_STAGES = 3;
+__host__ __device__ constexpr size_t tcw_smem_bytes() {
+  return (size_t)TCW_STAGES * (TCW_BM * TC_BK * 2 + TCW_BN * TC_BK * 2) + 1024 + 256;
+}
+
+template <bool B_MN, bool Q_MN>
+__global__ void __launch_bounds__(128, 1)
+    gemm_w256_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmQ, const WideArgs args) {
+  constexpr int BN = TCW_BN, STAGES = TCW_STAGES;
+  constexpr uint32_t HALF_A = TC_BM * TC_BK * 2;     // 16 KiB: one 128-row half of an A tile
+  constexpr uint32_t A_BYTES = 2 * HALF_A;
+  constexpr uint32_t B_BYTES = BN * TC_BK * 2;       // 32 KiB
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t IDESC = sm100::idesc_bf16_f32(TC_BM, BN, false, B_MN);
+  constexpr uint32_t IDESC2 = sm100::idesc_bf16_f32(TC_BM, BN, false, Q_MN);
+  using namespace sm100;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  const uint32_t smem0 = smem_u32(smem);
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
+  const uint32_t q_full = smem_u32(bars + 2 * STAGES + 1);
+  const uint32_t acc2_bar = smem_u32(bars + 2 * STAGES + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * TCW_BM, n0 = blockIdx.x * BN;
+  const int zq = blockIdx.x;
+  const int nkt = (args.K + TC_BK - 1) / TC_BK;
+  const bool fuse = args.out2 != nullptr;
+  // Ring stages used after the K loop: Q chunks 0,1 and 2,3, then the D half.
+  const int sq0 = nkt % STAGES, sq1 = (nkt + 1) % STAGES, sdh = (nkt + 2) % STAGES;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(accum_bar, 1);
+    mbar_init(q_full, 1);
+    mbar_init(acc2_bar, 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if (fuse) prefetch_tmap(&tmQ);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    bool ok = true;
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 11)) { ok = false; break; }
+      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+      const int k0 = i * TC_BK;
+      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+      tma_load_2d(sa, &tmA, full_bar(s), k0, m0);  // box 64 x 256: both halves
+      if (!B_MN) {
+        tma_load_2d(sb, &tmB, full_bar(s), k0, n0);
+      } else {
+#pragma unroll
+        for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmB, full_bar(s), n0 + 64 * h, k0);
+      }
+    }
+    if (ok && fuse) {
+      // Q's K chunks t = 0..3 into stages sq0 (t = 0, 1) and sq1 (t = 2, 3), each as soon as the
+      // last MMA reading that stage has completed (virtual iterations nkt and nkt + 1).
+      mbar_arrive_expect_tx(q_full, 4 * B_BYTES);
+      for (int u = 0; u < 2; ++u) {
+        const int v = nkt + u;
+        const int s = v % STAGES;
+        if (!mbar_wait(empty_bar(s), ((uint32_t)(v / STAGES) & 1u) ^ 1u, KID_GEMM_TC, 12)) break;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int t = 2 * u + w;
+          const uint32_t dst = smem0 + s * STAGE_BYTES + w * B_BYTES;
+          if (!Q_MN) {
+            tma_load_2d(dst, &tmQ, q_full, 64 * t, zq * BN);
+          } else {
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h) tma_load_2d(dst + h * 8192, &tmQ, q_full, 64 * h, zq * BN + 64 * t);
+          }
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer: both halves per k step
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (!mbar_wait(full_bar(s), ph, KID_GEMM_TC, 13)) break;
+      tc_fence_after();
+      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk) {
+        const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          mma_bf16(tmem_d + h * BN, smem_desc_sw128(sa + h * HALF_A + kk * 32, 16, 1024), bd, IDESC,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(empty_bar(s));
+    }
+    mma_commit(accum_bar);
+  }
+  __syncwarp();
+
+  bool ok = mbar_wait(accum_bar, 0, KID_GEMM_TC, 14);
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after();
+  const int r = warp * 32 + lane;  // TMEM lane = row within a half
+  const uint32_t tl = tmem_d + ((uint32_t)(warp * 32) << 16);
+
+  // Drains 256 columns of TMEM at column offset col0 (row m of the output): bf16 to global
+  // `dst` (if set) and, if to_smem, into the D-half stage as the swizzled K-major A operand.
+  auto drain = [&](uint32_t col0, int m, void* dst, long ld, bool to_smem) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tl + col0 + (uint32_t)c, v);
+      tmem_wait_ld();
+      uint4 q[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        q[u] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1])),
+                          pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+                          pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+                          pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+      if (dst != nullptr && m < args.M) {
+        uint4* g = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + (long)m * ld + n0 + c);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) g[u] = q[u];
+      }
+      if (to_smem) {
+        // K chunk c/64 of the D half: 16 KiB tile at sdh's stage + (c/64)*16 KiB, 16-byte chunk
+        // ch of row r at chunk position ch ^ (r % 8).
+        uint8_t* tileA = smem + sdh * STAGE_BYTES + (c / 64) * HALF_A + r * 128;
+        const int ch0 = (c % 64) / 8;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(tileA + (((ch0 + u) ^ (r & 7)) * 16)) = q[u];
+      }
+    }
+  };
+
+  if (!fuse) {
+    if (ok) {
+      drain(0, m0 + r, args.d1, args.ld1, false);
+      drain(BN, m0 + TC_BM + r, args.d1, args.ld1, false);
+    }
+  } else {
+    bool ok2 = ok;
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      // D half h -> global d1 and the D stage (free: the K loop is done, and for h = 1 the
+      // previous half's products have completed); also the previous half's result -> global.
+      if (ok2) {
+        if (h == 1) drain(0, m0 + r, args.out2, args.ld2, false);
+        drain((uint32_t)(h * BN), m0 + h * TC_BM + r, args.d1, args.ld1, true);
+      }
+      fence_proxy_async_smem();  // the tensor core reads what the threads just wrote
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (warp == 1 && lane == 0 && ok2) {
+        if (mbar_wait(q_full, 0, KID_GEMM_TC, 15)) {
+          tc_fence_after();
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const uint32_t sa = smem0 + sdh * STAGE_BYTES + t * HALF_A;
+            const uint32_t sb = smem0 + (t < 2 ? sq0 : sq1) * STAGE_BYTES + (t & 1) * B_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < TC_BK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t bd = Q_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+              mma_bf16(tmem_d + h * BN, ad, bd, IDESC2, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+        }
+        mma_commit(acc2_bar);
+      }
+      __syncwarp();
+      if (ok2) ok2 = mbar_wait(acc2_bar, (uint32_t)h, KID_GEMM_TC, 16);
+      ok2 = __all_sync(0xffffffffu, ok2);
+      tc_fence_after();
+    }
+    if (ok2) drain(BN, m0 + TC_BM + r, args.out2, args.ld2, false);
   }
   tc_fence_before();
   __syncthreads();

@@ -269,7 +269,10 @@ poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld
     int per_sm = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, smem) != cudaSuccess || per_sm < 1)
       return POETX_ERR_CUDA;
-    const int grid = (int)std::min<long>(groups, (long)kNumSms * per_sm);
+    // Rows of at most 4096 columns are software-pipelined across groups: about two groups per
+    // block (at least one block per SM); wider rows: as many blocks as fit.
+    const long want = cols <= 4096 ? std::min<long>(groups, std::max<long>(kNumSms, (groups + 1) / 2)) : groups;
+    const int grid = (int)std::min<long>(want, (long)kNumSms * per_sm);
     LaunchScope ls(POETX_KC_PERMUTE, st);
     k<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(in), ld_in, static_cast<uint16_t*>(out), ld_out, rows,
                                cols, colmap, rowmap, scatter ? 1 : 0);
@@ -361,6 +364,63 @@ poetx_status run_gemm_bd_fused(const GemmDesc& g, const void* Q, long q_rows, bo
   if (!g.b_mn && q_mn) return launch_bd_fused<false, true>(g, Q, q_rows, out2, ld2, st);
   if (g.b_mn && !q_mn) return launch_bd_fused<true, false>(g, Q, q_rows, out2, ld2, st);
   return launch_bd_fused<true, true>(g, Q, q_rows, out2, ld2, st);
+}
+
+// 256 x 256 tiles (gemm_w256_tc) for the W0' GEMM when they still occupy three quarters of the
+// SMs: plain bf16 store of D, optionally followed by the block factor (b = 256).
+bool w256_ok(int dt, const GemmDesc& g) {
+  const Epilogue& e = g.epi;
+  const bool plain_epi = e.d1 != nullptr && e.d1_dtype == BF16 && e.alpha1 == 1.f && e.beta1 == 0.f && !e.c &&
+                         !e.d2 && !e.diag1 && !e.split_stride1;
+  return dt == BF16 && !g.a_mn && g.N % 256 == 0 && g.batch == 1 && g.splits == 1 && g.K > 0 && plain_epi &&
+         4L * ((g.M + TCW_BM - 1) / TCW_BM) * (g.N / TCW_BN) >= 3L * kNumSms;
+}
+
+template <bool BMN, bool QMN>
+poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st) {
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
+  constexpr size_t smem = tcw_smem_bytes();
+  auto kern = gemm_w256_tc<BMN, QMN>;
+  if (!attr_done[dev]) {
+    if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  CUtensorMap ta, tb, tq;
+  if (!make_tmap(&ta, g.A, 64, TCW_BM)) return POETX_ERR_CUDA;
+  if (!make_tmap(&tb, g.B, 64, BMN ? 64 : TCW_BN)) return POETX_ERR_CUDA;
+  if (out2 != nullptr) {
+    if (!make_tmap(&tq, view(Q, q_rows, 256, 256), 64, QMN ? 64 : 256)) return POETX_ERR_CUDA;
+  } else {
+    tq = ta;  // unused without the block factor
+  }
+  WideArgs a;
+  a.M = g.M; a.N = g.N; a.K = g.K;
+  a.d1 = g.epi.d1; a.ld1 = g.epi.ld1;
+  a.out2 = out2; a.ld2 = ld2;
+  dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
+  LaunchScope ls(POETX_KC_W_GEMM, st);
+  kern<<<grid, 128, smem, st>>>(ta, tb, tq, a);
+  return last_launch();
+}
+
+// The W0' GEMM D = A . B^T -> d1, and (out2 != null, b = 256) out2 = D . Q^T or D . Q.
+poetx_status run_w_gemm(int dt, const GemmDesc& g, const void* Q, long q_rows, bool q_mn, void* out2, long ld2,
+                        cudaStream_t st) {
+  if (out2 == nullptr) {
+    if (!w256_ok(dt, g)) return run_gemm(dt, g, st, POETX_KC_W_GEMM);
+    POETX_TRY(check_gemm(g, BF16));
+    return g.b_mn ? launch_w256<true, false>(g, nullptr, 0, nullptr, 0, st)
+                  : launch_w256<false, false>(g, nullptr, 0, nullptr, 0, st);
+  }
+  if (!w256_ok(dt, g)) return run_gemm_bd_fused(g, Q, q_rows, q_mn, out2, ld2, st);
+  POETX_TRY(check_gemm(g, BF16));
+  if (q_rows < g.N || !aligned16(Q) || !aligned16(out2) || ld2 % 8) return POETX_ERR_ALIGNMENT;
+  if (!g.b_mn && !q_mn) return launch_w256<false, false>(g, Q, q_rows, out2, ld2, st);
+  if (!g.b_mn && q_mn) return launch_w256<false, true>(g, Q, q_rows, out2, ld2, st);
+  if (g.b_mn && !q_mn) return launch_w256<true, false>(g, Q, q_rows, out2, ld2, st);
+  return launch_w256<true, true>(g, Q, q_rows, out2, ld2, st);
 }
 
 // Out[:, blk z] = In[:, blk z] . Q_z^T  (forward block-diagonal application; tokens are rows).
@@ -600,6 +660,7 @@ struct CnpSide {
   int splits = 1;
   float* grad = nullptr;            // adjoint output
   char* ws = nullptr;               // this side's scratch
+  char* powers = nullptr;           // [nb*b, k*b] bf16 stack [M_k | ... | M_1] kept by the forward (or null)
 };
 
 CnpStageDesc stage_desc(int kind) {
@@ -709,15 +770,22 @@ poetx_status cnp_fwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaS
     Plan p;
     char* Sop = sd.ws + p.take(blk * 2);
     char* Mbuf[2] = {nullptr, nullptr};
-    if (k >= 2) { Mbuf[0] = sd.ws + p.take(blk * 2); Mbuf[1] = sd.ws + p.take(blk * 2); }
+    if (k >= 2 && sd.powers == nullptr) { Mbuf[0] = sd.ws + p.take(blk * 2); Mbuf[1] = sd.ws + p.take(blk * 2); }
     S.Sb0 = Sop; S.ld0 = b;
-    const void* Mprev = Sop;
+    const long kb = (long)k * b;
+    // Kept powers: M_j goes to slot k - j of the stack (M_1 = S by the UNPACK stage).
+    auto slot = [&](int j) { return static_cast<void*>(sd.powers + (size_t)(k - j) * b * 2); };
+    if (sd.powers) { S.Sb1 = slot(1); S.ld1 = kb; }
+    const void* Mprev = sd.powers ? slot(1) : Sop;
+    long ldprev = sd.powers ? kb : b;
     int s = 1;
     for (int j = 2; j <= k + 1; ++j, ++s) {
       const bool last = (j == k + 1);
-      void* out = last ? sd.Q : Mbuf[j & 1];
-      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, Mprev, b, true, b, out, b));
+      void* out = last ? sd.Q : (sd.powers ? slot(j) : Mbuf[j & 1]);
+      const long ldout = (last || !sd.powers) ? b : kb;
+      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, Mprev, ldprev, true, b, out, ldout));
       Mprev = out;
+      ldprev = ldout;
     }
   }
   return run_cnp_program(pr, nb_total, st);
@@ -736,11 +804,15 @@ poetx_status cnp_bwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaS
   for (int q = 0; q < nsides; ++q) nb_total += sides[q].nb;
   if (nb_total == 0) return POETX_OK;
   const long kb = (long)k * b;
+  // The power stages are skipped when the forward kept M_1..M_k (all sides or none).
+  const bool kept = sides[0].powers != nullptr;
+  for (int q = 1; q < nsides; ++q)
+    if ((sides[q].powers != nullptr) != kept) return POETX_ERR_INVALID_ARG;
   // stage list (same for both segments)
   int ns = 0;
   pr.st[ns++] = stage_desc(CNP_REDUCE_UNPACK);
   if (k >= 1) {
-    for (int j = 2; j <= k; ++j) {  // M_j = S.M_{j-1} + S
+    for (int j = 2; j <= k && !kept; ++j) {  // M_j = S.M_{j-1} + S
       CnpStageDesc d = stage_desc(CNP_GEMM);
       d.c_reg = CNP_R1; d.beta1 = 1.f;
       pr.st[ns++] = d;
@@ -783,13 +855,18 @@ poetx_status cnp_bwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaS
     }
     char* Sop = sd.ws + p.take(blk * 2);
     char* Ast = sd.ws + p.take(blk * (size_t)k * 2);
-    char* Bst = sd.ws + p.take(blk * (size_t)k * 2);
+    char* Bst = kept ? sd.powers : sd.ws + p.take(blk * (size_t)k * 2);
     auto aslot = [&](int t) { return static_cast<void*>(Ast + (size_t)t * b * 2); };
     auto bslot = [&](int t) { return static_cast<void*>(Bst + (size_t)t * b * 2); };
-    S.Sb0 = Sop; S.ld0 = b; S.Sb1 = bslot(k - 1); S.ld1 = kb;
+    S.Sb0 = Sop; S.ld0 = b;
+    if (kept) {
+      S.no_sreg = 1;  // S in TMEM only feeds the power stages
+    } else {
+      S.Sb1 = bslot(k - 1); S.ld1 = kb;
+    }
     S.Gb = aslot(0); S.ldg = kb;
     int s = 1;
-    for (int j = 2; j <= k; ++j, ++s)
+    for (int j = 2; j <= k && !kept; ++j, ++s)
       POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, bslot(k - j + 1), kb, true, b, bslot(k - j), kb));
     POETX_TRY(set_seg_gemm(pr, s++, q, sd.nb, Sop, b, aslot(0), kb, true, b, k >= 2 ? aslot(1) : nullptr, kb));
     for (int j = k - 1; j >= 1; --j, ++s)
@@ -906,12 +983,12 @@ poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const voi
   g.A = view(V, n, d->d_in, d->d_in);
   g.B = view(W0p, d->d_out, d->d_in, d->d_in);
   g.epi.d1 = Z; g.epi.d1_dtype = dt; g.epi.ld1 = d->d_out;
-  if (Y == nullptr) return run_gemm(dt, g, st, POETX_KC_W_GEMM);  // recompute only (mem-mode backward)
+  if (Y == nullptr) return run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, st);  // recompute only (mem-mode backward)
   if (bd_fusable(dt, b, g)) {
     // Z = V.W0'^T and Y'_i = Z_i.Q_R,i^T in one kernel.
-    POETX_TRY(run_gemm_bd_fused(g, QR, d->d_out, false, Yp, d->d_out, st));
+    POETX_TRY(run_w_gemm(dt, g, QR, d->d_out, false, Yp, d->d_out, st));
   } else {
-    POETX_TRY(run_gemm(dt, g, st, POETX_KC_W_GEMM));
+    POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, st));
     POETX_TRY(bd_forward(dt, n, d->d_out, b, Z, QR, Yp, st));
   }
   return permute_cols(dt, Yp, d->d_out, Y, d->d_out, n, d->d_out, pL, nullptr, true, st);
@@ -990,10 +1067,29 @@ poetx_status poetx_cnp_blocks(const poetx_desc* desc, int n_blocks, const float*
   return cnp_fwd_run(desc->b, desc->k, desc->dtype, n_blocks, theta, Q, static_cast<char*>(workspace), stream);
 }
 
+size_t poetx_cnp_powers_size(const poetx_desc* desc) {
+  if (check_desc(desc) != POETX_OK || !cnp_fused_ok(desc->b, desc->dtype) || desc->k < 1) return 0;
+  return (size_t)desc->k * desc->b * ((size_t)desc->d_in + desc->d_out) * 2;
+}
+
+// The kept powers of the R side ([d_out, k*b] bf16), then those of the P side ([d_in, k*b]).
+static void split_powers(const poetx_desc* d, const void* powers, char** pr, char** pp) {
+  char* base = static_cast<char*>(const_cast<void*>(powers));
+  *pr = base;
+  *pp = base ? base + (size_t)d->k * d->b * d->d_out * 2 : nullptr;
+}
+
+static poetx_status check_powers(const poetx_desc* desc, const void* powers) {
+  if (powers == nullptr) return POETX_OK;
+  if (poetx_cnp_powers_size(desc) == 0) return POETX_ERR_INVALID_ARG;
+  return aligned16(powers) ? POETX_OK : POETX_ERR_ALIGNMENT;
+}
+
 poetx_status poetx_cnp(const poetx_desc* desc, const float* theta_R, const float* theta_P, void* Q_R, void* Q_P,
-                       void* workspace, size_t ws_bytes, poetx_stream stream) {
+                       void* powers, void* workspace, size_t ws_bytes, poetx_stream stream) {
   POETX_TRY(check_desc(desc));
   POETX_TRY(check_ptrs({theta_R, theta_P, Q_R, Q_P}));
+  POETX_TRY(check_powers(desc, powers));
   POETX_TRY(check_ws(workspace, ws_bytes, cnp_layer_ws(desc)));
   char* ws = static_cast<char*>(workspace);
   const int b = desc->b;
@@ -1002,6 +1098,7 @@ poetx_status poetx_cnp(const poetx_desc* desc, const float* theta_R, const float
     CnpSide sides[2];
     sides[0].nb = desc->d_out / b; sides[0].theta = theta_R; sides[0].Q = Q_R; sides[0].ws = ws;
     sides[1].nb = desc->d_in / b; sides[1].theta = theta_P; sides[1].Q = Q_P; sides[1].ws = ws + offP;
+    split_powers(desc, powers, &sides[0].powers, &sides[1].powers);
     return cnp_fwd_fused(b, desc->k, sides, 2, stream);
   }
   POETX_TRY(cnp_fwd_generic(b, desc->k, desc->dtype, desc->d_out / b, theta_R, Q_R, ws, stream));
@@ -1037,12 +1134,57 @@ poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, 
   return forward_chain(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, Z, U, ws + f.V, ws + f.Yp, stream);
 }
 
+// Side stream of the backward pass.  Two chains of the backward are independent: the
+// gradient of theta_R's block partials (needs dY' and Z) runs beside dZ -> dV -> dU, and the dX
+// scatter (needs dU) runs beside the gradient of theta_P and the CNP adjoint.  They go to a
+// per-device non-blocking side stream, ordered with the caller's stream by events only, which
+// is also valid under stream capture (the side stream then joins the caller's graph).  A
+// per-device mutex keeps concurrent host callers from interleaving the fork and join records.
+struct SideStream {
+  std::mutex mu;
+  cudaStream_t st = nullptr;
+  cudaEvent_t ev[4] = {};
+  bool ready = false;
+};
+SideStream g_side[kMaxDevices];
+
+poetx_status side_stream(SideStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
+  SideStream& s = g_side[dev];
+  if (!s.ready) {
+    if (cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking) != cudaSuccess) return POETX_ERR_CUDA;
+    for (cudaEvent_t& e : s.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return POETX_ERR_CUDA;
+    s.ready = true;
+  }
+  *out = &s;
+  return POETX_OK;
+}
+
+// `to` waits for what `from` has enqueued so far.
+poetx_status stream_edge(cudaStream_t from, cudaStream_t to, cudaEvent_t e) {
+  if (cudaEventRecord(e, from) != cudaSuccess) return POETX_ERR_CUDA;
+  return cudaStreamWaitEvent(to, e, 0) == cudaSuccess ? POETX_OK : POETX_ERR_CUDA;
+}
+
+// Joins the side stream back into the caller's stream on every exit path once forked.
+struct SideJoin {
+  cudaStream_t main, side;
+  cudaEvent_t e;
+  bool armed = false;
+  ~SideJoin() {
+    if (armed) stream_edge(side, main, e);
+  }
+};
+
 poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X, const void* W0p,
                             const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
-                            const float* theta_R, const float* theta_P, const void* saved, void* dX,
-                            float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
+                            const float* theta_R, const float* theta_P, const void* saved, const void* powers,
+                            void* dX, float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
                             poetx_stream stream) {
   POETX_TRY(check_desc(desc));
+  POETX_TRY(check_powers(desc, powers));
   if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
   if (desc->mode == POETX_FAST && saved == nullptr && n_tokens > 0) return POETX_ERR_INVALID_ARG;
   if (desc->mode == POETX_MEM && saved != nullptr) return POETX_ERR_INVALID_ARG;
@@ -1070,10 +1212,18 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
                             nullptr, stream));
     Z = ws + w.Z;
   }
-  // Output side: dY' = dY[:, pi_L]; G_R partials; dZ = BD_R^T-adjoint.
+  SideStream* ss = nullptr;
+  POETX_TRY(side_stream(&ss));
+  std::lock_guard<std::mutex> side_lock(ss->mu);
+  const cudaStream_t side = ss->st;
+  // Output side: dY' = dY[:, pi_L]; dZ = BD_R^T-adjoint; G_R partials on the side stream, beside
+  // the W0' GEMM below (which leaves SMs idle in its last wave).
   POETX_TRY(permute_cols(dt, dY, dout, ws + w.dYp, dout, n, dout, perm_L, nullptr, false, stream));
-  POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, stream));
   POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
+  POETX_TRY(stream_edge(stream, side, ss->ev[0]));
+  SideJoin join{stream, side, ss->ev[3], true};
+  POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, side));
+  if (cudaEventRecord(ss->ev[1], side) != cudaSuccess) return POETX_ERR_CUDA;  // G_R partials done
   // dV = dZ . W0' (and, for b = 256, dU_i = dV_i . Q_P,i in the same kernel)
   GemmDesc g;
   g.M = (int)n; g.N = din; g.K = dout;
@@ -1081,19 +1231,23 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
   g.B = view(W0p, dout, din, din); g.b_mn = true;
   g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
   const bool fused_du = bd_fusable(dt, b, g);
-  if (fused_du) POETX_TRY(run_gemm_bd_fused(g, Q_P, din, true, ws + w.dU, din, stream));
-  else POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM));
-  // Input side: G_P partials (U saved or recomputed); dU; dX[:, pi_R] = dU.
-  POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
+  if (fused_du) POETX_TRY(run_w_gemm(dt, g, Q_P, din, true, ws + w.dU, din, stream));
+  else POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream));
   if (!fused_du) POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
-  POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, stream));
-  // CNP adjoint, packed gradients only.
+  // Input side: dX[:, pi_R] = dU (side stream, after G_R); G_P partials (U saved or recomputed).
+  POETX_TRY(stream_edge(stream, side, ss->ev[2]));
+  POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, side));
+  POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
+  // CNP adjoint, packed gradients only: it needs G_R's partials from the side stream.  The
+  // scatter may still run beside it; the join at exit waits for it.
+  if (cudaStreamWaitEvent(stream, ss->ev[1], 0) != cudaSuccess) return POETX_ERR_CUDA;
   if (cnp_fused_ok(b, dt)) {
     CnpSide sides[2];
     sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + w.GpR);
     sides[0].splits = w.sR; sides[0].grad = grad_theta_R; sides[0].ws = ws + w.cnpR;
     sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + w.GpP);
     sides[1].splits = w.sP; sides[1].grad = grad_theta_P; sides[1].ws = ws + w.cnpP;
+    split_powers(desc, powers, &sides[0].powers, &sides[1].powers);
     return cnp_bwd_fused(b, desc->k, sides, 2, stream);
   }
   POETX_TRY(cnp_bwd_generic(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + w.GpR), w.sR,

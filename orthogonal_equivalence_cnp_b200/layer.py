@@ -9,7 +9,7 @@ import numpy as np
 import torch
 
 from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_backward, poetx_cnp,
-               poetx_desc, poetx_forward, poetx_merge, poetx_workspace_size)
+               poetx_cnp_powers_size, poetx_desc, poetx_forward, poetx_merge, poetx_workspace_size)
 
 TORCH_DTYPE = {POETX_F32: torch.float32, POETX_BF16: torch.bfloat16}
 
@@ -41,6 +41,9 @@ class PoetxLayer:
         self.Y = torch.empty(self.n, dout, dtype=dt, device=dev)
         # POET-Xfast keeps Z [N, d_out] and U = X[:, pi_R] [N, d_in] for the backward pass.
         self.saved = torch.empty(self.n * (dout + din), dtype=dt, device=dev) if desc.mode == POETX_FAST else None
+        # POET-Xfast also keeps the CNP powers M_1..M_k for the adjoint (where the library keeps any).
+        pw = poetx_cnp_powers_size(desc) if desc.mode == POETX_FAST else 0
+        self.powers = torch.empty(pw, dtype=torch.uint8, device=dev) if pw else None
         self.dX = torch.empty(self.n, din, dtype=dt, device=dev)
         self.g_R = torch.empty_like(self.theta_R)
         self.g_P = torch.empty_like(self.theta_P)
@@ -63,7 +66,7 @@ class PoetxLayer:
 
     # ------------------------------------------------------------------------- the step
     def cnp(self):
-        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.ws)
+        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.powers, self.ws)
 
     def forward(self, X: torch.Tensor):
         poetx_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
@@ -72,7 +75,7 @@ class PoetxLayer:
 
     def backward(self, dY: torch.Tensor, X: torch.Tensor):
         poetx_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
-                       self.theta_R, self.theta_P, self.saved, self.dX, self.g_R, self.g_P, self.ws)
+                       self.theta_R, self.theta_P, self.saved, self.powers, self.dX, self.g_R, self.g_P, self.ws)
         return self.dX, self.g_R, self.g_P
 
     def step(self, X: torch.Tensor, dY: torch.Tensor):

@@ -62,11 +62,14 @@ def test_unpack_bit_exact():
 
 
 # ------------------------------------------------------------------------ index plumbing
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_absorb_bit_exact(dtype):
-    s = I.small_shape(512, 384, 64, 3, 4, dtype)
+# (1216 rows, 4096 columns): several four-row groups per block in the pipelined permutation;
+# 6144 columns: the wide-row path.
+@pytest.mark.parametrize("dtype,d_in,d_out", [("f32", 512, 384), ("bf16", 512, 384), ("bf16", 4096, 1216),
+                                              ("bf16", 6144, 512)])
+def test_absorb_bit_exact(dtype, d_in, d_out):
+    s = I.small_shape(d_in, d_out, 64, 3, 4, dtype)
     inp = I.make_layer(s, 11, with_activations=False)
-    L = PoetxLayer(make_desc(512, 384, 64, 3, dtype, "fast"), 4)
+    L = PoetxLayer(make_desc(d_in, d_out, 64, 3, dtype, "fast"), 4)
     L.load_state(inp.W0, inp.theta_R, inp.theta_P, inp.pi_L, inp.pi_R)
     torch.cuda.synchronize()
     assert np.array_equal(to_np(L.W0p), O.absorb(inp.W0, inp.pi_L, inp.pi_R))
@@ -118,6 +121,19 @@ def test_layer_bf16_small(d_in, d_out, b, n, mode):
     _check_all(g, oracle_layer(inp), TOL["bf16"])
 
 
+# Shapes whose W0' GEMMs take the 256 x 256-tile kernel (>= 111 tiles) with a ragged last row
+# tile: forward (d_out wide) and backward (d_in wide), with (b = 256) and without the fused
+# block factor.
+@pytest.mark.parametrize("d_in,d_out,b", [(512, 7168, 256), (7168, 512, 256), (512, 7168, 128), (7168, 512, 128)])
+@pytest.mark.parametrize("mode", ["fast", "mem"])
+def test_layer_bf16_wide_tiles(d_in, d_out, b, mode):
+    s = I.small_shape(d_in, d_out, b, 3, 1000, "bf16", theta_std=0.005, w_std=0.02)
+    inp = I.make_layer(s, 5 + d_in + b)
+    g, _ = gpu_layer(inp, mode=mode)
+    device_clean()
+    _check_all(g, oracle_layer(inp), TOL["bf16"])
+
+
 @pytest.mark.parametrize("k", [0, 1, 2])
 def test_layer_bf16_orders(k):
     s = I.small_shape(512, 512, 128, k, 160, "bf16", theta_std=0.005, w_std=0.02)
@@ -134,6 +150,21 @@ def test_fast_and_mem_agree():
     gm, _ = gpu_layer(inp, mode="mem")
     for k in KEYS:
         assert np.array_equal(gf[k], gm[k]), k
+
+
+@pytest.mark.parametrize("b,k", [(256, 3), (128, 2), (64, 1)])
+def test_kept_cnp_powers_match_recomputed(b, k):
+    """The adjoint gives bit-identical results with the forward's kept powers and without them."""
+    s = I.small_shape(2 * b, 3 * b, b, k, 130, "bf16", theta_std=0.005, w_std=0.02)
+    inp = I.make_layer(s, 91 + b)
+    g1, L = gpu_layer(inp, mode="fast")
+    assert L.powers is not None
+    X, dY = L.to_dev(inp.X), L.to_dev(inp.dY)
+    L.powers = None  # the adjoint recomputes M_2..M_k
+    L.step(X, dY)
+    torch.cuda.synchronize()
+    for key, t in (("dX", L.dX), ("g_R", L.g_R), ("g_P", L.g_P), ("Y", L.Y)):
+        assert np.array_equal(g1[key], to_np(t)), key
 
 
 def test_layer_llama8b_attn_full_size():
