@@ -155,6 +155,146 @@ __global__ void __launch_bounds__(256, ROWS == 4 ? 3 : 2)
   }
 }
 
+// Bulk-copy variant (bf16, 16-byte aligned rows): one thread streams each group's ROWS source
+// rows into a two-slot shared-memory ring with 1-D TMA bulk copies (cp.async.bulk, completion
+// on an mbarrier), so the loads of a block's next two groups are in flight without holding any
+// registers; the threads then interleave the slot into the word array W (16-byte, conflict-free
+// shared reads) and gather/store exactly as above.  With two blocks per SM and about two groups
+// per block, the whole input is requested at once.  Waits are bounded (device error word, kernel
+// id KID_PERMUTE); a block that gives up still reaches every barrier and skips its stores.
+enum : int { KID_PERMUTE = 3 };
+
+template <int ROWS>
+__host__ __device__ constexpr size_t permute_bulk_smem_bytes(int cols) {
+  return 2 * (size_t)ROWS * cols * 2        // ring: two slots of ROWS rows
+         + (size_t)cols * 2 * ROWS          // W: one word of ROWS elements per column
+         + ((size_t)cols * 2 + 15) / 16 * 16  // source map
+         + 64;                               // two mbarriers (+ padding)
+}
+
+template <int ROWS>
+__global__ void __launch_bounds__(256, 2)
+    permute_cols_bulk_kernel(const uint16_t* __restrict__ in, long ld_in, uint16_t* __restrict__ out, long ld_out,
+                             long rows, int cols, const int32_t* __restrict__ colmap,
+                             const int32_t* __restrict__ rowmap, int scatter) {
+  using Word = typename std::conditional<ROWS == 4, uint64_t, uint32_t>::type;
+  extern __shared__ __align__(128) uint8_t smem_bulk[];
+  const size_t slot_bytes = (size_t)ROWS * cols * 2;
+  uint8_t* ring = smem_bulk;
+  Word* W = reinterpret_cast<Word*>(smem_bulk + 2 * slot_bytes);
+  uint16_t* src_of = reinterpret_cast<uint16_t*>(smem_bulk + 2 * slot_bytes + (size_t)cols * 2 * ROWS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_bulk + 2 * slot_bytes + (size_t)cols * 2 * ROWS +
+                                               ((size_t)cols * 2 + 15) / 16 * 16);
+  const int nvec = cols / 8;
+  const long ngroups = (rows + ROWS - 1) / ROWS;
+  const uint32_t row_bytes = (uint32_t)cols * 2;
+
+  // Thread 0: request the ROWS source rows of group g into ring slot `slot`.
+  auto request = [&](long g, int slot) {
+    const long r0 = g * ROWS;
+    const int nr = (int)min((long)ROWS, rows - r0);
+    const uint32_t bar = sm100::smem_u32(bars + slot);
+    sm100::mbar_arrive_expect_tx(bar, (uint32_t)nr * row_bytes);
+    for (int r = 0; r < nr; ++r) {
+      const long sr = (!scatter && rowmap) ? (long)__ldg(rowmap + r0 + r) : r0 + r;
+      sm100::bulk_load_1d(sm100::smem_u32(ring + (size_t)slot * slot_bytes + (size_t)r * row_bytes),
+                          in + sr * ld_in, row_bytes, bar);
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(sm100::smem_u32(bars + 0), 1);
+    sm100::mbar_init(sm100::smem_u32(bars + 1), 1);
+    sm100::fence_mbar_init();
+    if (blockIdx.x < ngroups) request(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < ngroups) request(blockIdx.x + gridDim.x, 1);
+  }
+  // Source map (overlaps the first copies).
+  {
+    const int n4 = cols / 4;
+    for (int base = 0; base < n4; base += 4 * (int)blockDim.x) {
+      int4 t[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = base + u * (int)blockDim.x + (int)threadIdx.x;
+        if (v < n4) t[u] = __ldg(reinterpret_cast<const int4*>(colmap) + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = base + u * (int)blockDim.x + (int)threadIdx.x;
+        if (v >= n4) continue;
+        const int m4[4] = {t[u].x, t[u].y, t[u].z, t[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * v + e;
+          if (scatter) src_of[m4[e]] = (uint16_t)j; else src_of[j] = (uint16_t)m4[e];
+        }
+      }
+    }
+  }
+  __syncthreads();  // barriers initialised, map complete
+
+  bool ok = true;
+  int i = 0;
+#pragma unroll 1
+  for (long g = blockIdx.x; g < ngroups; g += gridDim.x, ++i) {
+    const int slot = i & 1;
+    const long r0 = g * ROWS;
+    const int nr = (int)min((long)ROWS, rows - r0);
+    const bool got = sm100::mbar_wait(sm100::smem_u32(bars + slot), (uint32_t)(i >> 1) & 1u, KID_PERMUTE, 1);
+    ok = __syncthreads_and(got);
+    if (!ok) break;  // block-uniform
+    // Interleave the slot into W (rows past nr repeat the last row).
+    {
+      const uint8_t* sl = ring + (size_t)slot * slot_bytes;
+      for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+        uint4 v[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r)
+          v[r] = reinterpret_cast<const uint4*>(sl + (size_t)min(r, nr - 1) * row_bytes)[c];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          Word w = 0;
+#pragma unroll
+          for (int r = 0; r < ROWS; ++r) w |= (Word)reinterpret_cast<const uint16_t*>(&v[r])[q] << (16 * r);
+          W[q * nvec + c] = w;
+        }
+      }
+    }
+    __syncthreads();  // W complete; the slot has been read by every thread
+    if (threadIdx.x == 0 && g + 2 * (long)gridDim.x < ngroups) {
+      sm100::fence_proxy_async_smem();  // the copy engine overwrites what the threads just read
+      request(g + 2 * (long)gridDim.x, slot);
+    }
+    {
+      for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+        const uint4 ix4 = reinterpret_cast<const uint4*>(src_of)[c];
+        const uint16_t* ix = reinterpret_cast<const uint16_t*>(&ix4);
+        Word w[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) w[q] = W[(ix[q] & 7) * nvec + (ix[q] >> 3)];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          if (r >= nr) break;
+          uint16_t e[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) e[q] = (uint16_t)(w[q] >> (16 * r));
+          reinterpret_cast<uint4*>(out + (r0 + r) * ld_out)[c] = *reinterpret_cast<const uint4*>(e);
+        }
+      }
+    }
+    __syncthreads();  // W free again
+  }
+  // A block that gave up (at its group i) waits, bounded, for the copies it still has in flight
+  // (groups i and i + 1) before its shared memory is released.
+  if (!ok && threadIdx.x == 0) {
+    long g = blockIdx.x + (long)i * gridDim.x;
+    for (int k = i; k < i + 2 && g < ngroups; ++k, g += gridDim.x)
+      sm100::mbar_wait(sm100::smem_u32(bars + (k & 1)), (uint32_t)(k >> 1) & 1u, KID_PERMUTE, 2);
+  }
+  __syncthreads();
+}
+
 // fp32 variant for the fp32 path (small layers): one row at a time, staged in shared memory.
 __global__ void __launch_bounds__(256)
     permute_cols_f32_kernel(const float* __restrict__ in, long ld_in, float* __restrict__ out, long ld_out, long rows,

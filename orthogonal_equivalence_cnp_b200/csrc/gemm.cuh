@@ -183,6 +183,7 @@ __device__ __forceinline__ void epilogue1(const Epilogue& e, int z, int split, i
 struct TcArgs {
   int M, N, K, splits;
   int a_zrow, a_zcol, b_zrow, b_zcol;
+  int tma_store;  // plain bf16 d1 (no addend/alpha/diag/d2/splits, zrow1 = 0): TMA-store epilogue
   Epilogue epi;
 };
 
@@ -203,7 +204,7 @@ __host__ __device__ constexpr size_t tc_smem_bytes() {
 template <int BN, int STAGES, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(128)
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const TcArgs args) {
+                 const __grid_constant__ CUtensorMap tmD, const TcArgs args) {
   constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
   constexpr uint32_t B_BYTES = BN * TC_BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -295,7 +296,45 @@ __global__ void __launch_bounds__(128)
   bool ok = mbar_wait(accum_bar, 0, KID_GEMM_TC, 3);
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
-  if (ok) {
+  if (ok && args.tma_store) {
+    // Each warp stages its 32 rows x 64 columns as a 128-byte-swizzled box (two 4 KiB buffers
+    // per warp in the idle ring) and lane 0 stores it with TMA: whole lines instead of one
+    // 16-byte piece per row, and rows past M are clipped by the map.
+    const uint32_t taddr = tmem_d + ((uint32_t)(warp * 32) << 16);
+    const Epilogue& e = args.epi;
+#pragma unroll 1
+    for (int c64 = 0; c64 < BN / 64; ++c64) {
+      uint8_t* buf = smem + warp * 8192 + (c64 & 1) * 4096;
+      if (c64 >= 2) {
+        if (lane == 0) bulk_wait_read<1>();  // the store two boxes back has read this buffer
+        __syncwarp();
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + (uint32_t)(c64 * 64 + hh * 32), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 8 * u;
+          const float f0 = nkt == 0 ? 0.f : __uint_as_float(v[j]), f1 = nkt == 0 ? 0.f : __uint_as_float(v[j + 1]);
+          const float f2 = nkt == 0 ? 0.f : __uint_as_float(v[j + 2]), f3 = nkt == 0 ? 0.f : __uint_as_float(v[j + 3]);
+          const float f4 = nkt == 0 ? 0.f : __uint_as_float(v[j + 4]), f5 = nkt == 0 ? 0.f : __uint_as_float(v[j + 5]);
+          const float f6 = nkt == 0 ? 0.f : __uint_as_float(v[j + 6]), f7 = nkt == 0 ? 0.f : __uint_as_float(v[j + 7]);
+          const uint4 q = make_uint4(pack_bf16x2(f0, f1), pack_bf16x2(f2, f3), pack_bf16x2(f4, f5), pack_bf16x2(f6, f7));
+          const int ch = hh * 4 + u;
+          *reinterpret_cast<uint4*>(buf + lane * 128 + ((ch ^ (lane & 7)) * 16)) = q;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tmD, smem_u32(buf), (int)(z * e.zcol1) + n0 + c64 * 64, m0 + warp * 32);
+        bulk_commit();
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  } else if (ok) {
     const int m = m0 + warp * 32 + lane;
     drain_tile<BN>(tmem_d + ((uint32_t)(warp * 32) << 16), args.epi, z, split, m, m < args.M, n0, nkt == 0);
   }
@@ -529,7 +568,8 @@ __host__ __device__ constexpr size_t tcw_smem_bytes() {
 template <bool B_MN, bool Q_MN>
 __global__ void __launch_bounds__(128, 1)
     gemm_w256_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmQ, const WideArgs args) {
+                 const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmD,
+                 const __grid_constant__ CUtensorMap tmO, const WideArgs args) {
   constexpr int BN = TCW_BN, STAGES = TCW_STAGES;
   constexpr uint32_t HALF_A = TC_BM * TC_BK * 2;     // 16 KiB: one 128-row half of an A tile
   constexpr uint32_t A_BYTES = 2 * HALF_A;
@@ -649,8 +689,9 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tl = tmem_d + ((uint32_t)(warp * 32) << 16);
 
   // Drains 256 columns of TMEM at column offset col0 (row m of the output): bf16 to global
-  // `dst` (if set) and, if to_smem, into the D-half stage as the swizzled K-major A operand.
-  auto drain = [&](uint32_t col0, int m, void* dst, long ld, bool to_smem) {
+  // `dst` (if set) and, if stage >= 0, into that ring stage as four swizzled K-major 128 x 64
+  // tiles, which are both the A operand of the block factor and TMA-store boxes of D.
+  auto drain = [&](uint32_t col0, int m, void* dst, long ld, int stage) {
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       uint32_t v[32];
@@ -668,10 +709,10 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u) g[u] = q[u];
       }
-      if (to_smem) {
-        // K chunk c/64 of the D half: 16 KiB tile at sdh's stage + (c/64)*16 KiB, 16-byte chunk
-        // ch of row r at chunk position ch ^ (r % 8).
-        uint8_t* tileA = smem + sdh * STAGE_BYTES + (c / 64) * HALF_A + r * 128;
+      if (stage >= 0) {
+        // K chunk c/64: 16 KiB tile at the stage + (c/64)*16 KiB, 16-byte chunk ch of row r at
+        // chunk position ch ^ (r % 8).
+        uint8_t* tileA = smem + stage * STAGE_BYTES + (c / 64) * HALF_A + r * 128;
         const int ch0 = (c % 64) / 8;
 #pragma unroll
         for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(tileA + (((ch0 + u) ^ (r & 7)) * 16)) = q[u];
@@ -679,25 +720,45 @@ __global__ void __launch_bounds__(128, 1)
     }
   };
 
+  // D goes out through TMA stores of the swizzled tiles (whole 128-byte lines; rows past M are
+  // clipped by the tensor map), issued by thread 0 in its bulk group.
+  const bool store_d = args.d1 != nullptr;
+  auto store_half = [&](int stage, int h) {
+    if (threadIdx.x == 0 && store_d) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        tma_store_2d(&tmD, smem0 + stage * STAGE_BYTES + t * HALF_A, n0 + 64 * t, m0 + h * TC_BM);
+      bulk_commit();
+    }
+  };
   if (!fuse) {
     if (ok) {
-      drain(0, m0 + r, args.d1, args.ld1, false);
-      drain(BN, m0 + TC_BM + r, args.d1, args.ld1, false);
+      drain(0, m0 + r, nullptr, 0, 0);
+      drain(BN, m0 + TC_BM + r, nullptr, 0, 1);
+    }
+    fence_proxy_async_smem();  // the TMA engine reads what the threads just wrote
+    __syncthreads();
+    if (ok) {
+      store_half(0, 0);
+      store_half(1, 1);
     }
   } else {
     bool ok2 = ok;
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
-      // D half h -> global d1 and the D stage (free: the K loop is done, and for h = 1 the
-      // previous half's products have completed); also the previous half's result -> global.
-      if (ok2) {
-        if (h == 1) drain(0, m0 + r, args.out2, args.ld2, false);
-        drain((uint32_t)(h * BN), m0 + h * TC_BM + r, args.d1, args.ld1, true);
+      // D half h -> the D stage (free: the K loop is done, and for h = 1 the previous half's
+      // products and D stores have finished reading it) -> global d1 by TMA.  The block-factor
+      // result of half h lands in the same TMEM columns and stays there until both are done.
+      if (h == 1) {
+        if (threadIdx.x == 0) bulk_wait_read<0>();
+        __syncthreads();
       }
-      fence_proxy_async_smem();  // the tensor core reads what the threads just wrote
+      if (ok2) drain((uint32_t)(h * BN), m0 + h * TC_BM + r, nullptr, 0, sdh);
+      fence_proxy_async_smem();  // the tensor core and the TMA engine read what the threads wrote
       tc_fence_before();
       __syncthreads();
       tc_fence_after();
+      if (ok2) store_half(sdh, h);
       if (warp == 1 && lane == 0 && ok2) {
         if (mbar_wait(q_full, 0, KID_GEMM_TC, 15)) {
           tc_fence_after();
@@ -720,8 +781,24 @@ __global__ void __launch_bounds__(128, 1)
       ok2 = __all_sync(0xffffffffu, ok2);
       tc_fence_after();
     }
-    if (ok2) drain(BN, m0 + TC_BM + r, args.out2, args.ld2, false);
+    // Both products are complete, so Q's stages are free: stage both halves of out2 there and
+    // store them with TMA.
+    if (ok2) {
+      drain(0, m0 + r, nullptr, 0, sq0);
+      drain(BN, m0 + TC_BM + r, nullptr, 0, sq1);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (ok2 && threadIdx.x == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          tma_store_2d(&tmO, smem0 + (h ? sq1 : sq0) * STAGE_BYTES + t * HALF_A, n0 + 64 * t, m0 + h * TC_BM);
+      bulk_commit();
+    }
   }
+  if (threadIdx.x == 0) bulk_wait<0>();  // shared memory stays valid until the stores are done
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem_d, 2 * BN);

@@ -177,6 +177,12 @@ EncodeTiledFn encode_fn() {
 
 // bf16 2-D tensor map over a whole operand array with a box of (inner x outer) elements and
 // 128-byte swizzle; reads beyond the array extent return zeros.
+Operand view(const void* base, long rows, long cols, long ld, long zrow = 0, long zcol = 0) {
+  Operand o;
+  o.base = base; o.rows = rows; o.cols = cols; o.ld = ld; o.zrow = zrow; o.zcol = zcol;
+  return o;
+}
+
 bool make_tmap(CUtensorMap* m, const Operand& op, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
@@ -200,16 +206,26 @@ poetx_status launch_tc(const GemmDesc& g, cudaStream_t st, int cls) {
     if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, td;
   if (!make_tmap(&ta, g.A, 64, AMN ? 64 : TC_BM)) return POETX_ERR_CUDA;
   if (!make_tmap(&tb, g.B, 64, BMN ? 64 : BN)) return POETX_ERR_CUDA;
   TcArgs a;
   a.M = g.M; a.N = g.N; a.K = g.K; a.splits = g.splits;
   a.a_zrow = (int)g.A.zrow; a.a_zcol = (int)g.A.zcol; a.b_zrow = (int)g.B.zrow; a.b_zcol = (int)g.B.zcol;
   a.epi = g.epi;
+  // TMA-store epilogue for a plain bf16 result batched (if at all) along columns: the map spans
+  // every batch's columns, boxes of 64 columns x 32 rows.
+  const Epilogue& e = g.epi;
+  a.tma_store = e.d1 != nullptr && e.d1_dtype == BF16 && e.alpha1 == 1.f && e.beta1 == 0.f && !e.c && !e.diag1 &&
+                !e.d2 && e.split_stride1 == 0 && e.zrow1 == 0 && g.splits == 1 && e.zcol1 % 8 == 0;
+  if (a.tma_store) {
+    if (!make_tmap(&td, view(e.d1, g.M, (long)(g.batch - 1) * e.zcol1 + g.N, e.ld1), 64, 32)) return POETX_ERR_CUDA;
+  } else {
+    td = ta;  // unused
+  }
   dim3 grid(g.N / BN, (g.M + TC_BM - 1) / TC_BM, g.batch * g.splits);
   LaunchScope ls(cls, st);
-  kern<<<grid, 128, smem, st>>>(ta, tb, a);
+  kern<<<grid, 128, smem, st>>>(ta, tb, td, a);
   return last_launch();
 }
 
@@ -258,7 +274,22 @@ poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld
   if (rows <= 0) return POETX_OK;
   if (cols > 65536) return POETX_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(colmap)) return POETX_ERR_ALIGNMENT;
-  if (dt == BF16) {
+  if (dt == BF16 && aligned16(in) && ld_in % 8 == 0 && cols <= 16384) {
+    // Bulk-copy kernel: groups of four rows (two above 8192 columns), two groups per block in
+    // flight from the start, as many blocks as fit (two per SM at 4096 columns).
+    const bool four = cols <= 8192;
+    const size_t smem = four ? permute_bulk_smem_bytes<4>(cols) : permute_bulk_smem_bytes<2>(cols);
+    auto k = four ? permute_cols_bulk_kernel<4> : permute_cols_bulk_kernel<2>;
+    if (!set_smem(k, smem)) return POETX_ERR_CUDA;
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, smem) != cudaSuccess || per_sm < 1)
+      return POETX_ERR_CUDA;
+    const long groups = (rows + (four ? 4 : 2) - 1) / (four ? 4 : 2);
+    const int grid = (int)std::min<long>(groups, (long)kNumSms * per_sm);
+    LaunchScope ls(POETX_KC_PERMUTE, st);
+    k<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(in), ld_in, static_cast<uint16_t*>(out), ld_out, rows,
+                               cols, colmap, rowmap, scatter ? 1 : 0);
+  } else if (dt == BF16) {
     // Groups of four rows (two for very wide rows); as many blocks as fit.
     const bool four = permute_smem_bytes<4>(cols) <= 160 * 1024;
     const size_t smem = four ? permute_smem_bytes<4>(cols) : permute_smem_bytes<2>(cols);
@@ -317,11 +348,6 @@ poetx_status reduce_splits(const float* part, int splits, long rows, int cols, f
 }
 
 // -------------------------------------------------------------------- GEMM building blocks
-Operand view(const void* base, long rows, long cols, long ld, long zrow = 0, long zcol = 0) {
-  Operand o;
-  o.base = base; o.rows = rows; o.cols = cols; o.ld = ld; o.zrow = zrow; o.zcol = zcol;
-  return o;
-}
 
 // W0' GEMM fused with the following block-diagonal factor (b = 256 only): out2 = D . Q^T
 // (q_mn = false, forward BD_R) or D . Q (q_mn = true, adjoint of BD_P), D also stored to d1.
@@ -387,13 +413,17 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
     if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
-  CUtensorMap ta, tb, tq;
+  CUtensorMap ta, tb, tq, td, to;
   if (!make_tmap(&ta, g.A, 64, TCW_BM)) return POETX_ERR_CUDA;
   if (!make_tmap(&tb, g.B, 64, BMN ? 64 : TCW_BN)) return POETX_ERR_CUDA;
+  // Store boxes of D and out2: 64 columns x 128 rows (one half's K chunk).
+  if (!make_tmap(&td, view(g.epi.d1, g.M, g.N, g.epi.ld1), 64, TC_BM)) return POETX_ERR_CUDA;
   if (out2 != nullptr) {
     if (!make_tmap(&tq, view(Q, q_rows, 256, 256), 64, QMN ? 64 : 256)) return POETX_ERR_CUDA;
+    if (!make_tmap(&to, view(out2, g.M, g.N, ld2), 64, TC_BM)) return POETX_ERR_CUDA;
   } else {
     tq = ta;  // unused without the block factor
+    to = ta;
   }
   WideArgs a;
   a.M = g.M; a.N = g.N; a.K = g.K;
@@ -401,7 +431,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.out2 = out2; a.ld2 = ld2;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(POETX_KC_W_GEMM, st);
-  kern<<<grid, 128, smem, st>>>(ta, tb, tq, a);
+  kern<<<grid, 128, smem, st>>>(ta, tb, tq, td, to, a);
   return last_launch();
 }
 

@@ -62,10 +62,11 @@ def test_unpack_bit_exact():
 
 
 # ------------------------------------------------------------------------ index plumbing
-# (1216 rows, 4096 columns): several four-row groups per block in the pipelined permutation;
-# 6144 columns: the wide-row path.
+# Every permutation kernel path: 1216 rows x 4096 columns (several four-row groups per block,
+# ragged last group), 6144 columns (four-row groups), 10240 columns (two-row groups), 17408
+# columns (the register-staged kernel for rows too wide for the bulk-copy ring).
 @pytest.mark.parametrize("dtype,d_in,d_out", [("f32", 512, 384), ("bf16", 512, 384), ("bf16", 4096, 1216),
-                                              ("bf16", 6144, 512)])
+                                              ("bf16", 6144, 512), ("bf16", 10240, 256), ("bf16", 17408, 128)])
 def test_absorb_bit_exact(dtype, d_in, d_out):
     s = I.small_shape(d_in, d_out, 64, 3, 4, dtype)
     inp = I.make_layer(s, 11, with_activations=False)
