@@ -25,6 +25,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -54,8 +56,14 @@ def step_flops(s: I.LayerShape) -> dict:
 
 
 def w_gemm_flops(s: I.LayerShape) -> int:
-    """FLOPs of one launch of the dominant kernel, the W0' GEMM (Z = V W0'^T or dV = dZ W0')."""
-    return 2 * s.n_tokens * s.d_in * s.d_out
+    """Algorithmic FLOPs of one launch of the dominant kernel, the W0' GEMM (Z = V W0'^T or
+    dV = dZ W0'); for bf16 and b = 256 that launch also applies the block factor on its output
+    side (Y'_i = Z_i Q_R,i^T: 2 N d_out b more; dU_i = dV_i Q_P,i: 2 N d_in b more).  Returned
+    per launch, averaged over the forward and the backward launch."""
+    f = 2 * s.n_tokens * s.d_in * s.d_out
+    if s.dtype == "bf16" and s.b == 256:
+        f += s.n_tokens * s.b * (s.d_in + s.d_out)
+    return f
 
 
 def read_peaks() -> dict:
@@ -297,34 +305,78 @@ def run_poetx(args):
     if graph is not None:
         del pgraph
 
-    # End to end through the public API with host buffers: H2D of X and dY from pinned memory,
-    # the step, D2H of dX and the packed gradients, all inside the timed interval.
+    # End to end through the public API with host buffers, as a training loop runs it: every step
+    # copies its X and dY from pinned host memory and reads its result (the packed gradients of
+    # theta_R and theta_P) back to pinned host memory.  The copies run on their own streams so
+    # that step i+1's inputs cross PCIe while step i computes (device inputs double-buffered, one
+    # captured step per buffer; the gradients are staged on the device before their read-back).
+    # The L2 flush runs before every step's compute, inside the timed interval.
     hX = torch.from_numpy(acts.X).to(layer.dtype).pin_memory()
     hdY = torch.from_numpy(acts.dY).to(layer.dtype).pin_memory()
-    h_dX = torch.empty(layer.dX.shape, dtype=layer.dtype).pin_memory()
     h_gR = torch.empty(layer.g_R.shape, dtype=torch.float32).pin_memory()
     h_gP = torch.empty(layer.g_P.shape, dtype=torch.float32).pin_memory()
-    Xe, dYe = torch.empty_like(X), torch.empty_like(dY)
+    Xb = [torch.empty_like(X) for _ in range(2)]
+    dYb = [torch.empty_like(dY) for _ in range(2)]
+    gRs = [torch.empty_like(layer.g_R) for _ in range(2)]
+    gPs = [torch.empty_like(layer.g_P) for _ in range(2)]
+    egraphs = []
+    if graph is not None:
+        for j in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                layer.step(Xb[j], dYb[j])
+            egraphs.append(g)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     Ke = K
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    ev_in = [torch.cuda.Event() for _ in range(Ke)]
+    ev_done = [torch.cuda.Event() for _ in range(Ke)]
+    ev_read = [torch.cuda.Event() for _ in range(Ke)]
+    t_beg, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def h2d(i):
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[i - 2])  # step i-2 no longer reads this buffer
+            Xb[i % 2].copy_(hX, non_blocking=True)
+            dYb[i % 2].copy_(hdY, non_blocking=True)
+            ev_in[i].record(s_in)
+
     barrier()
     torch.cuda.synchronize()
+    t_beg.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    h2d(0)
     for i in range(Ke):
+        if i + 1 < Ke:
+            h2d(i + 1)
+        stream.wait_event(ev_in[i])
+        if i >= 2:
+            stream.wait_event(ev_read[i - 2])  # the staged gradients of step i-2 have been read
         flush.zero_()
-        e0[i].record(stream)
-        Xe.copy_(hX, non_blocking=True)
-        dYe.copy_(hdY, non_blocking=True)
-        layer.step(Xe, dYe)
-        h_dX.copy_(layer.dX, non_blocking=True)
-        h_gR.copy_(layer.g_R, non_blocking=True)
-        h_gP.copy_(layer.g_P, non_blocking=True)
-        e1[i].record(stream)
+        if egraphs:
+            egraphs[i % 2].replay()
+        else:
+            layer.step(Xb[i % 2], dYb[i % 2])
+        gRs[i % 2].copy_(layer.g_R)
+        gPs[i % 2].copy_(layer.g_P)
+        ev_done[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[i])
+            h_gR.copy_(gRs[i % 2], non_blocking=True)
+            h_gP.copy_(gPs[i % 2], non_blocking=True)
+            ev_read[i].record(s_out)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
+    t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
-    te_ms = max_over_ranks(sum(e0[i].elapsed_time(e1[i]) for i in range(Ke)), world, dev)
+    te_ms = max_over_ranks(t_beg.elapsed_time(t_end), world, dev)
+    del egraphs
     h2d = hX.numel() * hX.element_size() + hdY.numel() * hdY.element_size()
-    d2h = (h_dX.numel() * h_dX.element_size() + h_gR.numel() * 4 + h_gP.numel() * 4)
+    d2h = h_gR.numel() * 4 + h_gP.numel() * 4
+    if not np.array_equal(h_gR.numpy(), layer.g_R.cpu().numpy()):
+        raise RuntimeError("end-to-end read-back differs from the device gradients")
 
     fl = step_flops(s)
     value = world * s.n_tokens * K / (t_ms / 1e3)
@@ -356,7 +408,8 @@ def run_poetx(args):
                    "launch": "CUDA graph of one step, replayed" if graph is not None else "direct launches",
                    "parallelism": f"replicas x{world} (data parallel over tokens, no collective on the path)",
                    "algorithmic_gflop_per_step": round(fl["total"] / 1e9, 2)},
-        "roofline": {"bound": "tensor", "kernel": "w0_gemm (Z = V W0'^T, dV = dZ W0')",
+        "roofline": {"bound": "tensor",
+                     "kernel": "w0_gemm (Z = V W0'^T with Y' = BD_R Z; dV = dZ W0' with dU = BD_P^T dV)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_source": f"{peaks['source']} bf16_tflops (burst)",
@@ -368,7 +421,11 @@ def run_poetx(args):
         "kernel_ms_per_step": {k: round(v[1] / K, 4) for k, v in prof.items() if v[0]},
         "gpu_launches": int(launches),
         "e2e": {"value": round(world * s.n_tokens * Ke / (te_ms / 1e3), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": round(te_ms / Ke, 4),
+                "protocol": "pinned X, dY in and packed theta gradients out every step; copies on their "
+                            "own streams overlap the previous/next step; L2 flushed before every step "
+                            "inside the interval"},
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -31,9 +31,6 @@ constexpr int CNP_THREADS = 256;  // 8 warps: warp w owns TMEM lane quarter w%4,
 enum CnpStageKind : int { CNP_GEMM = 0, CNP_UNPACK = 1, CNP_REDUCE_UNPACK = 2, CNP_PACK = 3 };
 enum CnpReg : int { CNP_NONE = -1, CNP_ACC = 0, CNP_R1 = 1, CNP_R2 = 2, CNP_R3 = 3 };
 enum : int { KID_CNP_FUSED = 2 };
-// Rows (or columns) per lane batch in the elementwise stages: all loads of a batch are issued
-// before the first shared-memory store.
-template <int BN> struct EwBatch { static constexpr int value = 8; };
 
 // Stage description shared by the segments (register-form epilogue):
 //   out1 = alpha1*acc + beta1*REG[c_reg] (+ I if diag1)  -> global g1 (g1_dtype) and/or REG[r1]
@@ -165,7 +162,6 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
   // Two 128 x BN f32 staging tiles (padded row stride), overlaid on the TMA ring, which is idle
   // whenever they are in use (between the last MMA of a stage and the first TMA load of the next).
   constexpr int TS = BN + 4;  // padded row stride (16-byte aligned rows for float4 access)
-  constexpr int EW_B = EwBatch<BN>::value;
   float* T0 = reinterpret_cast<float*>(smem);
   float* T1 = T0 + TC_BM * TS;
   // Coalesced write of a staged tile to global: warps over rows, lanes along columns.
@@ -279,69 +275,64 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         }
       }
     } else if (D.kind == CNP_UNPACK || D.kind == CNP_REDUCE_UNPACK) {
-      // theta -> T0 with coalesced, batched loads: above the diagonal warps walk rows (theta's
-      // packed row i is contiguous in j), below it warps walk columns (packed row j is
-      // contiguous in i).  Each lane issues EW_B loads before its first shared-memory store.
+      // theta -> T0 by per-thread asynchronous copies (all of a thread's copies in flight at
+      // once, no registers held): above the diagonal warps walk rows (theta's packed row i is
+      // contiguous in j), below it warps walk columns (packed row j is contiguous in i); the
+      // lower triangle is negated in place once the copies have landed.
       constexpr int RW = TC_BM / (CNP_THREADS / 32);  // rows (or columns) per warp
       constexpr int CPL = BN / 32;                    // columns (or rows / 32) per lane
-#pragma unroll 1
-      for (int t0 = 0; t0 < RW; t0 += EW_B) {
-        float v[EW_B][CPL];
+      constexpr int RPL = TC_BM / 32;                 // rows per lane in the column walk
+#pragma unroll 4
+      for (int t = 0; t < RW; ++t)
 #pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) {
-            const int ii = m0 + warp + 8 * (t0 + t), jj = n0 + lane + 32 * q;
-            v[t][q] = (ii < b && jj > ii) ? __ldg(th + packed_pos(ii, jj, b)) : 0.f;
+        for (int q = 0; q < CPL; ++q) {
+          const int r = warp + 8 * t, cc = lane + 32 * q, ii = m0 + r, jj = n0 + cc;
+          float* dst = T0 + r * TS + cc;
+          if (jj > ii) {
+            if (ii < b) cp_async4(dst, th + packed_pos(ii, jj, b));
+            else *dst = 0.f;
+          } else if (jj == ii) {
+            *dst = S.add_identity ? 1.f : 0.f;
           }
+        }
+#pragma unroll 4
+      for (int t = 0; t < BN / 8; ++t)
 #pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) {
-            const int r = warp + 8 * (t0 + t), cc = lane + 32 * q, ii = m0 + r, jj = n0 + cc;
-            if (jj > ii) T0[r * TS + cc] = v[t][q];
-            else if (jj == ii) T0[r * TS + cc] = S.add_identity ? 1.f : 0.f;
+        for (int q = 0; q < RPL; ++q) {
+          const int cc = warp + 8 * t, r = lane + 32 * q, jj = n0 + cc, ii = m0 + r;
+          if (ii > jj) {
+            float* dst = T0 + r * TS + cc;
+            if (ii < b) cp_async4(dst, th + packed_pos(jj, ii, b));
+            else *dst = 0.f;
           }
+        }
+      if (D.kind == CNP_REDUCE_UNPACK && S.splits == 1) {
+        // G (one partial: the gradient GEMM did not split K) -> T1, 16-byte copies by rows.
+        if (lane * 4 < BN) {
+#pragma unroll 4
+          for (int t = 0; t < RW; ++t) {
+            const int ii = m0 + warp + 8 * t;
+            float* dst = T1 + (warp + 8 * t) * TS + lane * 4;
+            if (ii < b) cp_async16(dst, S.part + ((long)z * b + ii) * b + n0 + lane * 4);
+            else *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
       }
-      constexpr int RPL = TC_BM / 32;  // rows per lane in the column walk
-#pragma unroll 1
-      for (int t0 = 0; t0 < BN / 8; t0 += EW_B) {
-        float v[EW_B][RPL];
+      cp_async_wait_all();
+      // Negate what this thread copied below the diagonal (its own copies are now visible to it).
+#pragma unroll 4
+      for (int t = 0; t < BN / 8; ++t)
 #pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < RPL; ++q) {
-            const int jj = n0 + warp + 8 * (t0 + t), ii = m0 + lane + 32 * q;
-            v[t][q] = (ii < b && ii > jj) ? -__ldg(th + packed_pos(jj, ii, b)) : 0.f;
-          }
-#pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < RPL; ++q) {
-            const int cc = warp + 8 * (t0 + t), r = lane + 32 * q;
-            if (m0 + r > n0 + cc) T0[r * TS + cc] = v[t][q];
-          }
-      }
-      if (D.kind == CNP_REDUCE_UNPACK) {
+        for (int q = 0; q < RPL; ++q) {
+          const int cc = warp + 8 * t, r = lane + 32 * q, ii = m0 + r;
+          if (ii > n0 + cc && ii < b) T0[r * TS + cc] = -T0[r * TS + cc];
+        }
+      if (D.kind == CNP_REDUCE_UNPACK && S.splits > 1) {
         // G = sum of split-K partials -> T1, row walk with one float4 per lane per row.
         const long sstride = (long)S.nb * b * b;
         constexpr int RB = 4;
-        if (S.splits == 1) {
-          // One partial (the gradient GEMM did not split K): all of a warp's rows in flight.
-          float4 ld4[RW];
-#pragma unroll
-          for (int t = 0; t < RW; ++t) {
-            const int ii = m0 + warp + 8 * t;
-            ld4[t] = (ii < b && lane * 4 < BN)
-                         ? __ldg(reinterpret_cast<const float4*>(S.part + ((long)z * b + ii) * b + n0) + lane)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-          for (int t = 0; t < RW; ++t)
-            if (lane * 4 < BN) *reinterpret_cast<float4*>(T1 + (warp + 8 * t) * TS + lane * 4) = ld4[t];
-        }
 #pragma unroll 1
-        for (int t0 = 0; t0 < (S.splits == 1 ? 0 : RW); t0 += RB) {
+        for (int t0 = 0; t0 < RW; t0 += RB) {
           float4 acc4[RB];
 #pragma unroll
           for (int t = 0; t < RB; ++t) acc4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -404,41 +395,26 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         }
       }
     } else if (D.kind == CNP_PACK) {
-      // T0 = own tile of G_S (row walk), T1[i][j] = G_S[j][i] (column walk, contiguous in i);
-      // then g[p(i,j)] = T0 - T1 with lanes along j (contiguous in p).
+      // T0 = own tile of G_S (16-byte copies by rows), T1[i][j] = G_S[j][i] (4-byte copies,
+      // column walk, contiguous in i); then g[p(i,j)] = T0 - T1 with lanes along j (contiguous
+      // in p).  All copies of a thread are in flight at once.
       constexpr int RW = TC_BM / (CNP_THREADS / 32);
-      constexpr int CPL = BN / 32;
       constexpr int RPL = TC_BM / 32;
-#pragma unroll 1
-      for (int t0 = 0; t0 < RW; t0 += EW_B) {
-        float v[EW_B][CPL];
-#pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) {
-            const int ii = m0 + warp + 8 * (t0 + t);
-            v[t][q] = ii < b ? S.GS[((long)z * b + ii) * b + n0 + lane + 32 * q] : 0.f;
-          }
-#pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) T0[(warp + 8 * (t0 + t)) * TS + lane + 32 * q] = v[t][q];
+      if (lane * 4 < BN) {
+#pragma unroll 4
+        for (int t = 0; t < RW; ++t) {
+          const int ii = m0 + warp + 8 * t;
+          if (ii < b) cp_async16(T0 + (warp + 8 * t) * TS + lane * 4, S.GS + ((long)z * b + ii) * b + n0 + lane * 4);
+        }
       }
-#pragma unroll 1
-      for (int t0 = 0; t0 < BN / 8; t0 += EW_B) {
-        float v[EW_B][RPL];
+#pragma unroll 4
+      for (int t = 0; t < BN / 8; ++t)
 #pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < RPL; ++q) {
-            const int jj = n0 + warp + 8 * (t0 + t), ii = m0 + lane + 32 * q;
-            v[t][q] = ii < b ? S.GS[((long)z * b + jj) * b + ii] : 0.f;
-          }
-#pragma unroll
-        for (int t = 0; t < EW_B; ++t)
-#pragma unroll
-          for (int q = 0; q < RPL; ++q) T1[(lane + 32 * q) * TS + warp + 8 * (t0 + t)] = v[t][q];
-      }
+        for (int q = 0; q < RPL; ++q) {
+          const int jj = n0 + warp + 8 * t, ii = m0 + lane + 32 * q;
+          if (ii < b) cp_async4(T1 + (lane + 32 * q) * TS + warp + 8 * t, S.GS + ((long)z * b + jj) * b + ii);
+        }
+      cp_async_wait_all();
       __syncthreads();
       for (int r = warp; r < TC_BM; r += CNP_THREADS / 32) {
         const int ii = m0 + r;

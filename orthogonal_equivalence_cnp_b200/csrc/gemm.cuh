@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(128)
         bulk_commit();
       }
     }
-    if (lane == 0) bulk_wait<0>();
+    if (lane == 0) bulk_wait_read<0>();
   } else if (ok) {
     const int m = m0 + warp * 32 + lane;
     drain_tile<BN>(tmem_d + ((uint32_t)(warp * 32) << 16), args.epi, z, split, m, m < args.M, n0, nkt == 0);
@@ -777,28 +777,29 @@ __global__ void __launch_bounds__(128, 1)
         mma_commit(acc2_bar);
       }
       __syncwarp();
+      // While the second half's products run, the first half's result (complete: its products
+      // were awaited at the end of h = 0) goes straight to global memory.
+      if (h == 1 && ok2) {
+        tc_fence_after();
+        drain(0, m0 + r, args.out2, args.ld2, -1);
+      }
       if (ok2) ok2 = mbar_wait(acc2_bar, (uint32_t)h, KID_GEMM_TC, 16);
       ok2 = __all_sync(0xffffffffu, ok2);
       tc_fence_after();
     }
-    // Both products are complete, so Q's stages are free: stage both halves of out2 there and
-    // store them with TMA.
-    if (ok2) {
-      drain(0, m0 + r, nullptr, 0, sq0);
-      drain(BN, m0 + TC_BM + r, nullptr, 0, sq1);
-    }
+    // Both products are complete, so Q's stages are free: stage the second half's result there
+    // and store it with TMA.
+    if (ok2) drain(BN, m0 + TC_BM + r, nullptr, 0, sq0);
     fence_proxy_async_smem();
     __syncthreads();
     if (ok2 && threadIdx.x == 0) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          tma_store_2d(&tmO, smem0 + (h ? sq1 : sq0) * STAGE_BYTES + t * HALF_A, n0 + 64 * t, m0 + h * TC_BM);
+      for (int t = 0; t < 4; ++t) tma_store_2d(&tmO, smem0 + sq0 * STAGE_BYTES + t * HALF_A, n0 + 64 * t, m0 + TC_BM);
       bulk_commit();
     }
   }
-  if (threadIdx.x == 0) bulk_wait<0>();  // shared memory stays valid until the stores are done
+  // Shared memory stays valid until the stores have read it (the writes complete with the grid).
+  if (threadIdx.x == 0) bulk_wait_read<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem_d, 2 * BN);

@@ -62,6 +62,16 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 }
 // 2-D tiled load of one box into shared memory; completion is signalled on `bar` (tx bytes).
 // c0 is the innermost (contiguous) coordinate; callers keep c0 * elem_size a multiple of 16.
+// Per-thread asynchronous global -> shared copies (no register is held while in flight).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// Waits for all of this thread's cp.async copies (their data is then visible to this thread).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Tiled TMA store of a shared-memory box (laid out as the map's swizzle expects) to global, in
 // the issuing thread's bulk async-group.  Coordinates are never negative here.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
