@@ -51,6 +51,7 @@ struct CnpStageDesc {
 struct CnpSegStage {
   CUtensorMap tmA;  // K-major A operand map (box 64 x 128)
   CUtensorMap tmB;  // B operand map (K-major box 64 x BN, or MN-major box 64 x 64)
+  CUtensorMap tmD;  // store map of g1 (128-byte x 32-row boxes: 64 bf16 or 32 fp32 columns)
   int K;
   int a_zrow, b_zrow, b_zcol;
   void* g1;         // global out1: element (z*b+i, j) at g1[(z*b+i)*g1_ld + j]
@@ -164,14 +165,22 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
   constexpr int TS = BN + 4;  // padded row stride (16-byte aligned rows for float4 access)
   float* T0 = reinterpret_cast<float*>(smem);
   float* T1 = T0 + TC_BM * TS;
-  // Coalesced write of a staged tile to global: warps over rows, lanes along columns.
-  auto tile_store = [&](const float* T, void* dst, long ld, int dt) {
+  // Coalesced write of a staged tile to global: warps over rows, lanes along columns.  With
+  // `skew` the tile holds theta unsigned and entries below the diagonal are negated on the way.
+  auto tile_store = [&](const float* T, void* dst, long ld, int dt, bool skew) {
     for (int r = warp; r < TC_BM; r += CNP_THREADS / 32) {
       const int ii = m0 + r;
       if (ii >= b) break;
       const long base = ((long)z * b + ii) * ld + n0;
       for (int cc = lane * 4; cc < BN; cc += 128) {
-        const float4 f = *reinterpret_cast<const float4*>(T + r * TS + cc);
+        float4 f = *reinterpret_cast<const float4*>(T + r * TS + cc);
+        if (skew) {
+          const int jj = n0 + cc;
+          if (jj < ii) f.x = -f.x;
+          if (jj + 1 < ii) f.y = -f.y;
+          if (jj + 2 < ii) f.z = -f.z;
+          if (jj + 3 < ii) f.w = -f.w;
+        }
         if (dt == BF16) {
           uint2 u;
           u.x = pack_bf16x2(f.x, f.y);
@@ -236,6 +245,15 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
       acc_phase ^= 1u;
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
+      // Staging of this warp's 32 x HALF slice of out1 for the TMA store: 128-byte rows,
+      // 16-byte chunk ch of row `lane` at position ch ^ (lane % 8), one 4 KiB box per 128 bytes
+      // of row (the ring is idle: every MMA of the stage has completed).
+      const bool f32_out = D.g1_dtype == F32;
+      uint8_t* stg = smem + warp * 8192;
+      const bool rows_ok = m0 + quarter * 32 < b;  // b % 32 == 0: a 32-row box is all in or all out
+      // A bf16 box is 64 columns wide: with BN = 64 a warp's slice is narrower, so those tiles
+      // keep per-row stores.
+      const bool tma_out = G.g1 != nullptr && (f32_out ? HALF % 32 : HALF % 64) == 0;
       if (ok) {
 #pragma unroll 1
         for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
@@ -268,44 +286,85 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
             tmem_st_32x32b_x32(treg(D.r1, c), reinterpret_cast<const uint32_t (&)[32]>(o1));
             wrote_tmem = true;
           }
-          if (G.g1 != nullptr && row_ok) {
+          if (G.g1 != nullptr && !tma_out && row_ok) {
             store32(G.g1, grow * G.g1_ld + n, D.g1_dtype, o1);
             wrote_global = true;
+          } else if (tma_out) {
+            const int cl = c - half * HALF;  // column of this chunk within the warp's slice
+            if (f32_out) {
+              uint8_t* box = stg + (cl / 32) * 4096 + lane * 128;
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<float4*>(box + ((u ^ (lane & 7)) * 16)) =
+                    make_float4(o1[4 * u], o1[4 * u + 1], o1[4 * u + 2], o1[4 * u + 3]);
+            } else {
+              uint8_t* box = stg + (cl / 64) * 4096 + lane * 128;
+              const int ch0 = (cl % 64) / 8;
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<uint4*>(box + (((ch0 + u) ^ (lane & 7)) * 16)) =
+                    make_uint4(pack_bf16x2(o1[8 * u], o1[8 * u + 1]), pack_bf16x2(o1[8 * u + 2], o1[8 * u + 3]),
+                               pack_bf16x2(o1[8 * u + 4], o1[8 * u + 5]), pack_bf16x2(o1[8 * u + 6], o1[8 * u + 7]));
+            }
           }
         }
+      }
+      if (tma_out) {
+        // One lane stores the warp's boxes; the stores are complete (visible to the peers' TMA
+        // loads of the next stage after the cluster barrier) before the barrier.
+        wrote_global = true;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && ok && rows_ok) {
+          const int x0 = n0 + half * HALF, y0 = z * b + m0 + quarter * 32;
+          const int nbox = f32_out ? HALF / 32 : HALF / 64;
+          for (int t = 0; t < nbox; ++t)
+            tma_store_2d(&G.tmD, smem_u32(stg + t * 4096), x0 + t * (f32_out ? 32 : 64), y0);
+          bulk_commit();
+          bulk_wait<0>();
+        }
+        __syncwarp();
       }
     } else if (D.kind == CNP_UNPACK || D.kind == CNP_REDUCE_UNPACK) {
       // theta -> T0 by per-thread asynchronous copies (all of a thread's copies in flight at
       // once, no registers held): above the diagonal warps walk rows (theta's packed row i is
-      // contiguous in j), below it warps walk columns (packed row j is contiguous in i); the
-      // lower triangle is negated in place once the copies have landed.
+      // contiguous in j), below it warps walk columns (packed row j is contiguous in i).  T0
+      // holds theta unsigned; the consumers negate below the diagonal.  Packed row i starts at
+      // ro(i) + i + 1 with ro(i) = i*b - i(i+1)/2 - i - 1, so element (i, j) is ro(i) + j.
       constexpr int RW = TC_BM / (CNP_THREADS / 32);  // rows (or columns) per warp
       constexpr int CPL = BN / 32;                    // columns (or rows / 32) per lane
       constexpr int RPL = TC_BM / 32;                 // rows per lane in the column walk
+      const float diag = S.add_identity ? 1.f : 0.f;
 #pragma unroll 4
-      for (int t = 0; t < RW; ++t)
+      for (int t = 0; t < RW; ++t) {
+        const int r = warp + 8 * t, ii = m0 + r;
+        const int ro = ii * b - (ii * (ii + 1)) / 2 - ii - 1;
 #pragma unroll
         for (int q = 0; q < CPL; ++q) {
-          const int r = warp + 8 * t, cc = lane + 32 * q, ii = m0 + r, jj = n0 + cc;
+          const int cc = lane + 32 * q, jj = n0 + cc;
           float* dst = T0 + r * TS + cc;
           if (jj > ii) {
-            if (ii < b) cp_async4(dst, th + packed_pos(ii, jj, b));
+            if (ii < b) cp_async4(dst, th + (ro + jj));
             else *dst = 0.f;
           } else if (jj == ii) {
-            *dst = S.add_identity ? 1.f : 0.f;
+            *dst = diag;
           }
         }
+      }
 #pragma unroll 4
-      for (int t = 0; t < BN / 8; ++t)
+      for (int t = 0; t < BN / 8; ++t) {
+        const int cc = warp + 8 * t, jj = n0 + cc;
+        const int ro = jj * b - (jj * (jj + 1)) / 2 - jj - 1;
 #pragma unroll
         for (int q = 0; q < RPL; ++q) {
-          const int cc = warp + 8 * t, r = lane + 32 * q, jj = n0 + cc, ii = m0 + r;
+          const int r = lane + 32 * q, ii = m0 + r;
           if (ii > jj) {
             float* dst = T0 + r * TS + cc;
-            if (ii < b) cp_async4(dst, th + packed_pos(jj, ii, b));
+            if (ii < b) cp_async4(dst, th + (ro + ii));
             else *dst = 0.f;
           }
         }
+      }
       if (D.kind == CNP_REDUCE_UNPACK && S.splits == 1) {
         // G (one partial: the gradient GEMM did not split K) -> T1, 16-byte copies by rows.
         if (lane * 4 < BN) {
@@ -319,14 +378,6 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         }
       }
       cp_async_wait_all();
-      // Negate what this thread copied below the diagonal (its own copies are now visible to it).
-#pragma unroll 4
-      for (int t = 0; t < BN / 8; ++t)
-#pragma unroll
-        for (int q = 0; q < RPL; ++q) {
-          const int cc = warp + 8 * t, r = lane + 32 * q, ii = m0 + r;
-          if (ii > n0 + cc && ii < b) T0[r * TS + cc] = -T0[r * TS + cc];
-        }
       if (D.kind == CNP_REDUCE_UNPACK && S.splits > 1) {
         // G = sum of split-K partials -> T1, row walk with one float4 per lane per row.
         const long sstride = (long)S.nb * b * b;
@@ -361,11 +412,11 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
       }
       __syncthreads();
       // Coalesced global copies from the tiles; then each thread moves its row into TMEM.
-      if (S.Sb0) tile_store(T0, S.Sb0, S.ld0, BF16);
-      if (S.Sb1) tile_store(T0, S.Sb1, S.ld1, BF16);
+      if (S.Sb0) tile_store(T0, S.Sb0, S.ld0, BF16, true);
+      if (S.Sb1) tile_store(T0, S.Sb1, S.ld1, BF16, true);
       if (D.kind == CNP_REDUCE_UNPACK) {
-        if (S.Gb) tile_store(T1, S.Gb, S.ldg, BF16);
-        if (S.G32) tile_store(T1, S.G32, b, F32);
+        if (S.Gb) tile_store(T1, S.Gb, S.ldg, BF16, false);
+        if (S.G32) tile_store(T1, S.G32, b, F32, false);
       }
       wrote_global = true;
 #pragma unroll 1
@@ -373,11 +424,14 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         uint32_t w[32];
         if (!S.no_sreg) {
           const float4* trow = reinterpret_cast<const float4*>(T0 + (quarter * 32 + lane) * TS + c);
+          const int neg_below = i - (n0 + c);  // columns j < neg_below of this chunk lie below the diagonal
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float4 f = trow[j];
-            w[4 * j] = __float_as_uint(f.x); w[4 * j + 1] = __float_as_uint(f.y);
-            w[4 * j + 2] = __float_as_uint(f.z); w[4 * j + 3] = __float_as_uint(f.w);
+            w[4 * j] = __float_as_uint(4 * j < neg_below ? -f.x : f.x);
+            w[4 * j + 1] = __float_as_uint(4 * j + 1 < neg_below ? -f.y : f.y);
+            w[4 * j + 2] = __float_as_uint(4 * j + 2 < neg_below ? -f.z : f.z);
+            w[4 * j + 3] = __float_as_uint(4 * j + 3 < neg_below ? -f.w : f.w);
           }
           tmem_st_32x32b_x32(treg(CNP_R1, c), w);
           wrote_tmem = true;

@@ -569,7 +569,7 @@ template <bool B_MN, bool Q_MN>
 __global__ void __launch_bounds__(128, 1)
     gemm_w256_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmD,
-                 const __grid_constant__ CUtensorMap tmO, const WideArgs args) {
+                 const WideArgs args) {
   constexpr int BN = TCW_BN, STAGES = TCW_STAGES;
   constexpr uint32_t HALF_A = TC_BM * TC_BK * 2;     // 16 KiB: one 128-row half of an A tile
   constexpr uint32_t A_BYTES = 2 * HALF_A;
@@ -748,12 +748,15 @@ __global__ void __launch_bounds__(128, 1)
     for (int h = 0; h < 2; ++h) {
       // D half h -> the D stage (free: the K loop is done, and for h = 1 the previous half's
       // products and D stores have finished reading it) -> global d1 by TMA.  The block-factor
-      // result of half h lands in the same TMEM columns and stays there until both are done.
+      // result of half h lands in the half's own TMEM columns and is stored from registers.
       if (h == 1) {
         if (threadIdx.x == 0) bulk_wait_read<0>();
         __syncthreads();
       }
-      if (ok2) drain((uint32_t)(h * BN), m0 + h * TC_BM + r, nullptr, 0, sdh);
+      if (ok2) {
+        if (h == 1) drain(0, m0 + r, args.out2, args.ld2, -1);  // first half's result
+        drain((uint32_t)(h * BN), m0 + h * TC_BM + r, nullptr, 0, sdh);
+      }
       fence_proxy_async_smem();  // the tensor core and the TMA engine read what the threads wrote
       tc_fence_before();
       __syncthreads();
@@ -777,26 +780,11 @@ __global__ void __launch_bounds__(128, 1)
         mma_commit(acc2_bar);
       }
       __syncwarp();
-      // While the second half's products run, the first half's result (complete: its products
-      // were awaited at the end of h = 0) goes straight to global memory.
-      if (h == 1 && ok2) {
-        tc_fence_after();
-        drain(0, m0 + r, args.out2, args.ld2, -1);
-      }
       if (ok2) ok2 = mbar_wait(acc2_bar, (uint32_t)h, KID_GEMM_TC, 16);
       ok2 = __all_sync(0xffffffffu, ok2);
       tc_fence_after();
     }
-    // Both products are complete, so Q's stages are free: stage the second half's result there
-    // and store it with TMA.
-    if (ok2) drain(BN, m0 + TC_BM + r, nullptr, 0, sq0);
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (ok2 && threadIdx.x == 0) {
-#pragma unroll
-      for (int t = 0; t < 4; ++t) tma_store_2d(&tmO, smem0 + sq0 * STAGE_BYTES + t * HALF_A, n0 + 64 * t, m0 + TC_BM);
-      bulk_commit();
-    }
+    if (ok2) drain(BN, m0 + TC_BM + r, args.out2, args.ld2, -1);
   }
   // Shared memory stays valid until the stores have read it (the writes complete with the grid).
   if (threadIdx.x == 0) bulk_wait_read<0>();

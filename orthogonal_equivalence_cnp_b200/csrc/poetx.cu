@@ -183,15 +183,19 @@ Operand view(const void* base, long rows, long cols, long ld, long zrow = 0, lon
   return o;
 }
 
-bool make_tmap(CUtensorMap* m, const Operand& op, uint32_t box_inner, uint32_t box_outer) {
+// 2-D tensor map of a row-major bf16 (or fp32) array, 128-byte swizzle; box_inner elements must
+// span 128 bytes (64 bf16 / 32 fp32).
+bool make_tmap(CUtensorMap* m, const Operand& op, uint32_t box_inner, uint32_t box_outer, int dt = BF16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
+  const uint64_t es = dt == F32 ? 4 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)op.cols, (cuuint64_t)op.rows};
-  cuuint64_t strides[1] = {(cuuint64_t)op.ld * 2};
+  cuuint64_t strides[1] = {(cuuint64_t)op.ld * es};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(op.base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(m, dt == F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(op.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -413,17 +417,15 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
     if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
-  CUtensorMap ta, tb, tq, td, to;
+  CUtensorMap ta, tb, tq, td;
   if (!make_tmap(&ta, g.A, 64, TCW_BM)) return POETX_ERR_CUDA;
   if (!make_tmap(&tb, g.B, 64, BMN ? 64 : TCW_BN)) return POETX_ERR_CUDA;
-  // Store boxes of D and out2: 64 columns x 128 rows (one half's K chunk).
+  // Store boxes of D: 64 columns x 128 rows (one half's K chunk).
   if (!make_tmap(&td, view(g.epi.d1, g.M, g.N, g.epi.ld1), 64, TC_BM)) return POETX_ERR_CUDA;
   if (out2 != nullptr) {
     if (!make_tmap(&tq, view(Q, q_rows, 256, 256), 64, QMN ? 64 : 256)) return POETX_ERR_CUDA;
-    if (!make_tmap(&to, view(out2, g.M, g.N, ld2), 64, TC_BM)) return POETX_ERR_CUDA;
   } else {
     tq = ta;  // unused without the block factor
-    to = ta;
   }
   WideArgs a;
   a.M = g.M; a.N = g.N; a.K = g.K;
@@ -431,7 +433,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.out2 = out2; a.ld2 = ld2;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(POETX_KC_W_GEMM, st);
-  kern<<<grid, 128, smem, st>>>(ta, tb, tq, td, to, a);
+  kern<<<grid, 128, smem, st>>>(ta, tb, tq, td, a);
   return last_launch();
 }
 
@@ -716,9 +718,16 @@ poetx_status set_seg_gemm(CnpProgram& pr, int s, int q, long nb, const void* A, 
   G.K = K; G.a_zrow = b; G.b_zrow = b; G.b_zcol = 0;
   G.g1 = g1; G.g1_ld = g1_ld;
   if (g1 && (!aligned16(g1) || g1_ld % 8)) return POETX_ERR_ALIGNMENT;
+  if (g1) {
+    // The stage's output leaves through TMA stores of 32-row boxes (128-byte rows).
+    const bool f32 = pr.st[s].g1_dtype == F32;
+    if (!make_tmap(&G.tmD, view(g1, nb * b, b, g1_ld), f32 ? 32 : 64, 32, f32 ? F32 : BF16)) return POETX_ERR_CUDA;
+  }
   pr.st[s].b_mn = b_mn ? 1 : 0;
   return POETX_OK;
 }
+
+static_assert(sizeof(CnpProgram) <= 32764, "the CNP program is passed as one kernel parameter");
 
 template <int BN>
 poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_t st) {
