@@ -35,7 +35,7 @@ __all__ = [
     "packed_pairs", "packed_index", "unpack_skew", "pack_skew_grad", "cayley_exact",
     "cayley_neumann", "cnp", "block_diag", "perm_matrix", "absorb", "unabsorb",
     "dense_transforms", "dense_weight", "forward_dense", "backward_dense", "cnp_grad",
-    "forward_chain", "backward_chain", "merge",
+    "forward_chain", "backward_chain", "merge", "adamw_step", "train_schedule",
 ]
 
 
@@ -298,3 +298,42 @@ def merge(W0p, theta_R, theta_P, pi_L, pi_R, pi_L_new, pi_R_new, b, k):
     return (absorb(W_full, pi_L_new, pi_R_new),
             np.zeros_like(np.asarray(theta_R, np.float64)),
             np.zeros_like(np.asarray(theta_P, np.float64)))
+
+
+# ------------------------------------------------------------------ optimiser on packed theta
+# The trainable state is the packed theta, so the optimiser state lives at the packed size too
+# ([AD], the section on compact storage: gradients and optimiser state shrink with it).  The
+# pages name AdamW as the baseline optimiser and give the POET learning-rate scale gamma = 0.5
+# and the reset gap of 400 steps ([RR] "Weaknesses"), but not AdamW's own constants; those are
+# arguments here.  AdamW is the decoupled-weight-decay Adam (Loshchilov and Hutter): with
+# step t >= 1 and eta = gamma * lr,
+#   m <- beta1 m + (1 - beta1) g,   v <- beta2 v + (1 - beta2) g^2,
+#   theta <- theta - eta * (lam * theta + (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps)),
+# the decay acting on the theta before this step.
+def adamw_step(theta, grad, m, v, t, lr, gamma=0.5, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0):
+    """One AdamW step on packed parameters; returns (theta, m, v) in float64."""
+    theta = np.asarray(theta, np.float64)
+    g = np.asarray(grad, np.float64)
+    m = beta1 * np.asarray(m, np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, np.float64) + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** t)
+    v_hat = v / (1.0 - beta2 ** t)
+    eta = gamma * lr
+    theta = theta - eta * (weight_decay * theta + m_hat / (np.sqrt(v_hat) + eps))
+    return theta, m, v
+
+
+def train_schedule(n_steps, reset_gap=400):
+    """What happens after each training step s = 1..n_steps of the merge schedule: a list of
+    (s, t, merge) with t the AdamW step count used at s and merge True when step s is followed
+    by merge-then-reinitialise.  Reading of the pages' reset gap: after every reset_gap steps
+    the transforms are merged and theta is zeroed; the moments of theta restart with it (they
+    belonged to the parameters that were folded away), so t counts from 1 again."""
+    out, t = [], 0
+    for s in range(1, n_steps + 1):
+        t += 1
+        merge_now = s % reset_gap == 0
+        out.append((s, t, merge_now))
+        if merge_now:
+            t = 0
+    return out

@@ -149,6 +149,37 @@ def make_layer(shape: LayerShape, seed: int, n_tokens: Optional[int] = None,
     return LayerInputs(shape, seed, pi_L, pi_R, theta_R, theta_P, W0, X, dY)
 
 
+def make_theta(shape: LayerShape, seed: int):
+    """theta_R, theta_P of make_layer(shape, seed) (the same draws), without W0 or activations."""
+    rng = np.random.default_rng(seed)
+    rng.permutation(shape.d_out)
+    rng.permutation(shape.d_in)
+    theta_R = rng.normal(0.0, shape.theta_std, (shape.nb_out, shape.n_packed)).astype(np.float32)
+    theta_P = rng.normal(0.0, shape.theta_std, (shape.nb_in, shape.n_packed)).astype(np.float32)
+    return theta_R, theta_P
+
+
+# Stacked workloads: layer l of stack config c (4: the 32-block Llama-8B stack, 5: the 40-block
+# Llama-13B stack) is drawn with seed 1000 + 100 c + l; the layers of a block are q,k,v,o,gate,
+# up,down in that order.
+STACKS = {
+    "llama8b_stack_32x7_b256_bf16": (4, 32, llama8b_stack_shapes),
+    "llama13b_stack_40x7_b512_bf16_mem": (5, 40, llama13b_stack_shapes),
+}
+
+
+def stack_layers(name: str):
+    """[(layer index, LayerShape, seed)] of every linear of a stacked workload."""
+    config, nblocks, shapes = STACKS[name]
+    per_block = shapes()
+    out = []
+    for blk in range(nblocks):
+        for j, sh in enumerate(per_block):
+            l = blk * len(per_block) + j
+            out.append((l, sh, 1000 + 100 * config + l))
+    return out
+
+
 def make_workload(name: str, n_tokens: Optional[int] = None, with_activations: bool = True) -> LayerInputs:
     return make_layer(WORKLOADS[name], WORKLOAD_SEEDS[name], n_tokens, with_activations)
 

@@ -31,3 +31,17 @@ def test_workload_table():
     w = I.WORKLOADS["llama8b_attn_4096_b256_bf16"]
     assert (w.d_in, w.d_out, w.b, w.k, w.n_tokens, w.nb_in) == (4096, 4096, 256, 3, 2048, 16)
     assert I.WORKLOADS["layer256_b32_f32"].nb_out == 8
+
+
+def test_stack_layers_and_theta_only_draws():
+    L8 = I.stack_layers("llama8b_stack_32x7_b256_bf16")
+    L13 = I.stack_layers("llama13b_stack_40x7_b512_bf16_mem")
+    assert len(L8) == 224 and len(L13) == 280
+    assert [seed for _, _, seed in L8[:2]] == [1400, 1401] and L8[-1][2] == 1623
+    assert [seed for _, _, seed in L13[:2]] == [1500, 1501] and L13[-1][2] == 1779
+    assert sum(s.nb_in + s.nb_out for _, s, _ in L8) == 32 * (32 + 20 + 20 + 32 + 72 + 72 + 72)
+    # make_theta reproduces make_layer's theta draws exactly
+    _, sh, seed = L13[6]
+    tR, tP = I.make_theta(sh, seed)
+    full = I.make_layer(sh, seed, n_tokens=2, with_activations=False)
+    assert np.array_equal(tR, full.theta_R) and np.array_equal(tP, full.theta_P)

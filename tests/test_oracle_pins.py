@@ -10,6 +10,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 import oracle as O
 
@@ -384,3 +385,74 @@ def test_absorb_equals_permutation_matrix_product():
     pl, pr = rng.permutation(6), rng.permutation(10)
     assert np.array_equal(O.absorb(W, pl, pr), O.perm_matrix(pl) @ W @ O.perm_matrix(pr).T)
     assert np.array_equal(O.unabsorb(O.absorb(W, pl, pr), pl, pr), W)
+
+
+# ------------------------------------------------------------- optimiser on packed theta
+def test_adamw_first_step_is_the_closed_form():
+    # From zero moments the bias-corrected moments are g and g^2, so the step is
+    # -gamma*lr*(lam*theta + g/(|g| + eps)).
+    rng = np.random.default_rng(3)
+    th, g = rng.normal(size=1000), rng.normal(size=1000)
+    lr, gamma, lam, eps = 1e-3, 0.5, 0.1, 1e-8
+    th1, m1, v1 = O.adamw_step(th, g, np.zeros(1000), np.zeros(1000), 1, lr, gamma, 0.9, 0.999, eps, lam)
+    np.testing.assert_allclose(th1, th - gamma * lr * (lam * th + g / (np.abs(g) + eps)), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(m1, 0.1 * g, rtol=1e-15)
+    np.testing.assert_allclose(v1, 0.001 * g * g, rtol=1e-12)
+
+
+def test_adamw_constant_gradient_moves_linearly_and_decay_alone_is_geometric():
+    # A constant gradient keeps the corrected moments at g and g^2 exactly at every step.
+    g = np.array([0.5, -2.0, 3e-3])
+    th, m, v = np.zeros(3), np.zeros(3), np.zeros(3)
+    for t in range(1, 8):
+        th, m, v = O.adamw_step(th, g, m, v, t, 0.01, 0.5)
+    np.testing.assert_allclose(th, -7 * 0.5 * 0.01 * g / (np.abs(g) + 1e-8), rtol=1e-10)
+    # Zero gradient, weight decay only: theta shrinks by (1 - gamma*lr*lam) per step.
+    th = np.array([1.0, -3.0])
+    m = v = np.zeros(2)
+    for t in range(1, 6):
+        th, m, v = O.adamw_step(th, np.zeros(2), m, v, t, 0.1, 0.5, weight_decay=0.2)
+    np.testing.assert_allclose(th, np.array([1.0, -3.0]) * (1 - 0.5 * 0.1 * 0.2) ** 5, rtol=1e-14)
+
+
+def test_adamw_matches_the_library_optimiser():
+    # torch.optim.AdamW (CPU, float64) with lr = gamma * lr is the same algorithm.
+    rng = np.random.default_rng(11)
+    th0 = rng.normal(size=257)
+    p = torch.nn.Parameter(torch.tensor(th0, dtype=torch.float64))
+    opt = torch.optim.AdamW([p], lr=0.5 * 2e-3, betas=(0.85, 0.99), eps=1e-6, weight_decay=0.05)
+    th, m, v = th0.copy(), np.zeros(257), np.zeros(257)
+    for t in range(1, 13):
+        g = rng.normal(size=257) * (1 + t)
+        p.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        th, m, v = O.adamw_step(th, g, m, v, t, 2e-3, 0.5, 0.85, 0.99, 1e-6, 0.05)
+    np.testing.assert_allclose(th, p.detach().numpy(), rtol=0, atol=1e-14)
+
+
+def test_adamw_planted_mistakes_are_caught():
+    # Each slip below changes the constant-gradient trajectory or the library comparison.
+    g = np.array([0.5, -2.0])
+    def run(step):
+        th, m, v = np.zeros(2), np.zeros(2), np.zeros(2)
+        for t in range(1, 6):
+            th, m, v = step(th, g, m, v, t)
+        return th
+    ref = -5 * 0.5 * 0.01 * g / (np.abs(g) + 1e-8)
+    def no_bias_correction(th, g, m, v, t):
+        m = 0.9 * m + 0.1 * g; v = 0.999 * v + 0.001 * g * g
+        return th - 0.005 * m / (np.sqrt(v) + 1e-8), m, v
+    def eps_inside_sqrt(th, g, m, v, t):
+        m = 0.9 * m + 0.1 * g; v = 0.999 * v + 0.001 * g * g
+        return th - 0.005 * (m / (1 - 0.9 ** t)) / np.sqrt(v / (1 - 0.999 ** t) + 1e-2), m, v
+    def no_gamma(th, g, m, v, t):
+        return O.adamw_step(th, g, m, v, t, 0.01, 1.0)
+    for slip in (no_bias_correction, eps_inside_sqrt, no_gamma):
+        assert not np.allclose(run(slip), ref, rtol=1e-6), slip.__name__
+    assert np.allclose(run(lambda th, g, m, v, t: O.adamw_step(th, g, m, v, t, 0.01, 0.5)), ref, rtol=1e-10)
+
+
+def test_merge_schedule_resets_every_gap():
+    sch = O.train_schedule(1000, reset_gap=400)
+    assert [s for s, _, mg in sch if mg] == [400, 800]
+    assert [t for s, t, _ in sch if s in (1, 400, 401, 800, 801, 1000)] == [1, 400, 1, 400, 1, 200]
