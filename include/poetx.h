@@ -189,6 +189,35 @@ poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, con
                          const int32_t* perm_L_new, const int32_t* perm_R_new, float* theta_R,
                          float* theta_P, void* workspace, size_t ws_bytes, poetx_stream stream);
 
+/* ------------------------------------------------------------------ optimiser (packed theta)
+ * AdamW on the packed skew parameters, so that the optimiser state stays at the packed size
+ * (agidaily.cc article, compact storage: gradients and optimiser state shrink with the
+ * parameters; replication review, "Weaknesses": the POET learning-rate scale gamma = 0.5 and
+ * the reset gap of 400 steps).  The pages do not give AdamW's own constants; they are
+ * arguments.  With step t >= 1 and eta = gamma * lr, elementwise:
+ *   m <- beta1 m + (1 - beta1) g;   v <- beta2 v + (1 - beta2) g^2;
+ *   theta <- theta - eta * (weight_decay * theta + (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps)).
+ * The paper has no separate routine for it: this is the decoupled-weight-decay Adam of
+ * Loshchilov and Hutter applied to theta. */
+typedef struct {
+  float lr;            /* base learning rate (>= 0)                         */
+  float gamma;         /* POET learning-rate scale (the pages use 0.5)       */
+  float beta1, beta2;  /* moment decay rates, each in [0, 1)                 */
+  float eps;           /* > 0                                                */
+  float weight_decay;  /* decoupled decay coefficient (>= 0)                 */
+} poetx_adamw_cfg;
+
+/* One AdamW step over n packed parameters (e.g. theta_R and theta_P stored back to back).
+ *   theta, m, v float32 [n] (in/out); grad float32 [n] (in); t = step count of the moments (>= 1).
+ * All pointers 16-byte aligned, caller-owned device memory.  n == 0 launches nothing.
+ * Errors: INVALID_ARG (bad cfg, t < 1, n < 0, NULL pointer), ALIGNMENT, CUDA. */
+poetx_status poetx_adamw_step(const poetx_adamw_cfg* cfg, long long n, int t, float* theta,
+                              const float* grad, float* m, float* v, poetx_stream stream);
+
+/* Zeroes the moments (m, v float32 [n]) after a merge re-initialises theta: the merge schedule
+ * restarts the moments with the parameters (their step count t starts again at 1). */
+poetx_status poetx_adamw_reset(long long n, float* m, float* v, poetx_stream stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* poetx_status_string(poetx_status s);
 
@@ -210,7 +239,8 @@ typedef enum {
   POETX_KC_PERMUTE = 5,      /* feature-dimension gather / scatter                          */
   POETX_KC_ELEMENTWISE = 6,  /* unpack, pack, split-K reduction, permutation inverse        */
   POETX_KC_TEST_GEMM = 7,    /* poetx_test_gemm                                              */
-  POETX_KC_COUNT = 8
+  POETX_KC_OPTIMIZER = 8,    /* poetx_adamw_step                                             */
+  POETX_KC_COUNT = 9
 } poetx_kernel_class;
 
 /* Number of kernels this library has launched in the process so far. */

@@ -17,7 +17,8 @@ __all__ = [
     "poetx_cnp_blocks_workspace_size", "poetx_absorb", "poetx_forward", "poetx_backward",
     "poetx_merge", "poetx_status_string", "poetx_device_status", "poetx_test_gemm",
     "poetx_launch_count", "poetx_profile_enable", "poetx_profile_summary", "KERNEL_CLASSES",
-    "poetx_cnp_blocks_noalloc", "poetx_cnp_powers_size",
+    "poetx_cnp_blocks_noalloc", "poetx_cnp_powers_size", "poetx_adamw_cfg", "poetx_adamw_step",
+    "poetx_adamw_reset",
 ]
 
 POETX_F32, POETX_BF16 = 0, 1
@@ -27,7 +28,8 @@ STATUS = {
     4: "POETX_ERR_WORKSPACE", 5: "POETX_ERR_CUDA", 6: "POETX_ERR_DEVICE_TIMEOUT",
 }
 
-KERNEL_CLASSES = ["w_gemm", "bd_gemm", "grad_gemm", "cnp_gemm", "merge_gemm", "permute", "elementwise", "test_gemm"]
+KERNEL_CLASSES = ["w_gemm", "bd_gemm", "grad_gemm", "cnp_gemm", "merge_gemm", "permute", "elementwise", "test_gemm",
+                  "optimizer"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -43,6 +45,11 @@ class poetx_desc(ctypes.Structure):
     def __repr__(self):
         return (f"poetx_desc(d_in={self.d_in}, d_out={self.d_out}, b={self.b}, k={self.k}, "
                 f"dtype={self.dtype}, mode={self.mode})")
+
+
+class poetx_adamw_cfg(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("gamma", ctypes.c_float), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float)]
 
 
 class PoetxError(RuntimeError):
@@ -68,6 +75,8 @@ _SIGNATURES = {
     "poetx_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_adamw_step": (_I, [ctypes.POINTER(poetx_adamw_cfg), _LL, _I, _P, _P, _P, _P, _P]),
+    "poetx_adamw_reset": (_I, [_LL, _P, _P, _P]),
     "poetx_status_string": (ctypes.c_char_p, [_I]),
     "poetx_device_status": (_I, [ctypes.POINTER(ctypes.c_int)]),
     "poetx_launch_count": (ctypes.c_ulonglong, []),
@@ -179,6 +188,15 @@ def poetx_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, Q_P, theta_R
                                 _ptr(perm_R), _ptr(Q_R), _ptr(Q_P), _ptr(theta_R), _ptr(theta_P), _ptr(saved),
                                 _ptr(powers), _ptr(dX), _ptr(grad_theta_R), _ptr(grad_theta_P), _ptr(workspace),
                                 ws_bytes, _stream(stream)), "poetx_backward")
+
+
+def poetx_adamw_step(cfg, n, t, theta, grad, m, v, stream=None):
+    _check(lib().poetx_adamw_step(ctypes.byref(cfg), n, t, _ptr(theta), _ptr(grad), _ptr(m), _ptr(v),
+                                  _stream(stream)), "poetx_adamw_step")
+
+
+def poetx_adamw_reset(n, m, v, stream=None):
+    _check(lib().poetx_adamw_reset(n, _ptr(m), _ptr(v), _stream(stream)), "poetx_adamw_reset")
 
 
 def poetx_merge(desc, W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P, workspace,

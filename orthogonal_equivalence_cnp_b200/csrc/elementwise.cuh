@@ -295,6 +295,46 @@ __global__ void __launch_bounds__(256, 2)
   __syncthreads();
 }
 
+// AdamW on packed parameters (decoupled weight decay), fp32: per parameter 16 bytes read
+// (theta, g, m, v) and 12 written (theta, m, v), so HBM bound.  float4 grid-stride over the
+// first n - n % 4 parameters, the tail by the first threads.
+struct AdamwArgs {
+  float eta;          // gamma * lr
+  float beta1, beta2;
+  float inv_bc1;      // 1 / (1 - beta1^t)
+  float inv_sqrt_bc2; // 1 / sqrt(1 - beta2^t)
+  float eps, decay;
+};
+
+__device__ __forceinline__ void adamw_one(float& th, float g, float& m, float& v, const AdamwArgs& a) {
+  m = a.beta1 * m + (1.f - a.beta1) * g;
+  v = a.beta2 * v + (1.f - a.beta2) * g * g;
+  const float denom = sqrtf(v) * a.inv_sqrt_bc2 + a.eps;
+  th = th - a.eta * (a.decay * th + (m * a.inv_bc1) / denom);
+}
+
+__global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ theta, const float* __restrict__ grad,
+                                                    float* __restrict__ m, float* __restrict__ v, long n,
+                                                    const AdamwArgs a) {
+  const long n4 = n / 4;
+  const long stride = (long)gridDim.x * blockDim.x;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 t4 = reinterpret_cast<const float4*>(theta)[i];
+    const float4 g4 = __ldg(reinterpret_cast<const float4*>(grad) + i);
+    float4 m4 = reinterpret_cast<const float4*>(m)[i];
+    float4 v4 = reinterpret_cast<const float4*>(v)[i];
+    adamw_one(t4.x, g4.x, m4.x, v4.x, a);
+    adamw_one(t4.y, g4.y, m4.y, v4.y, a);
+    adamw_one(t4.z, g4.z, m4.z, v4.z, a);
+    adamw_one(t4.w, g4.w, m4.w, v4.w, a);
+    reinterpret_cast<float4*>(theta)[i] = t4;
+    reinterpret_cast<float4*>(m)[i] = m4;
+    reinterpret_cast<float4*>(v)[i] = v4;
+  }
+  const long tail = 4 * n4 + (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tail < n) adamw_one(theta[tail], grad[tail], m[tail], v[tail], a);
+}
+
 // fp32 variant for the fp32 path (small layers): one row at a time, staged in shared memory.
 __global__ void __launch_bounds__(256)
     permute_cols_f32_kernel(const float* __restrict__ in, long ld_in, float* __restrict__ out, long ld_out, long rows,

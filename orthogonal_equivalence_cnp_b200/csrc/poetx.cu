@@ -8,6 +8,7 @@
 #include <utility>
 #include <vector>
 #include <initializer_list>
+#include <cmath>
 #include <mutex>
 
 #include "../../include/poetx_testing.h"
@@ -1068,6 +1069,37 @@ poetx_status noalloc_scratch(char** out) {
 
 // =============================================================================== C ABI
 extern "C" {
+
+poetx_status poetx_adamw_step(const poetx_adamw_cfg* cfg, long long n, int t, float* theta, const float* grad,
+                              float* m, float* v, poetx_stream stream) {
+  if (cfg == nullptr || n < 0 || t < 1) return POETX_ERR_INVALID_ARG;
+  if (!(cfg->lr >= 0.f) || !(cfg->gamma >= 0.f) || !(cfg->beta1 >= 0.f && cfg->beta1 < 1.f) ||
+      !(cfg->beta2 >= 0.f && cfg->beta2 < 1.f) || !(cfg->eps > 0.f) || !(cfg->weight_decay >= 0.f))
+    return POETX_ERR_INVALID_ARG;
+  if (n == 0) return POETX_OK;
+  POETX_TRY(check_ptrs({theta, grad, m, v}));
+  const double bc1 = 1.0 - std::pow((double)cfg->beta1, (double)t);
+  const double bc2 = 1.0 - std::pow((double)cfg->beta2, (double)t);
+  AdamwArgs a;
+  a.eta = cfg->gamma * cfg->lr;
+  a.beta1 = cfg->beta1; a.beta2 = cfg->beta2;
+  a.inv_bc1 = (float)(1.0 / bc1);
+  a.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(bc2));
+  a.eps = cfg->eps; a.decay = cfg->weight_decay;
+  const long n4 = (long)(n / 4);
+  const int grid = (int)std::max<long>(1, std::min<long>((n4 + 255) / 256, (long)kNumSms * 8));
+  LaunchScope ls(POETX_KC_OPTIMIZER, stream);
+  adamw_kernel<<<grid, 256, 0, stream>>>(theta, grad, m, v, (long)n, a);
+  return last_launch();
+}
+
+poetx_status poetx_adamw_reset(long long n, float* m, float* v, poetx_stream stream) {
+  if (n < 0) return POETX_ERR_INVALID_ARG;
+  if (n == 0) return POETX_OK;
+  POETX_TRY(check_ptrs({m, v}));
+  if (cudaMemsetAsync(m, 0, (size_t)n * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
+  return cudaMemsetAsync(v, 0, (size_t)n * 4, stream) == cudaSuccess ? POETX_OK : POETX_ERR_CUDA;
+}
 
 const char* poetx_status_string(poetx_status s) {
   switch (s) {

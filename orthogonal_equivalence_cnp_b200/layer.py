@@ -8,8 +8,9 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_backward, poetx_cnp,
-               poetx_cnp_powers_size, poetx_desc, poetx_forward, poetx_merge, poetx_workspace_size)
+from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_adamw_cfg, poetx_adamw_reset,
+               poetx_adamw_step, poetx_backward, poetx_cnp, poetx_cnp_powers_size, poetx_desc, poetx_forward,
+               poetx_merge, poetx_workspace_size)
 
 TORCH_DTYPE = {POETX_F32: torch.float32, POETX_BF16: torch.bfloat16}
 
@@ -32,8 +33,11 @@ class PoetxLayer:
         P = b * (b - 1) // 2
         dev = self.device
         self.W0p = torch.empty(dout, din, dtype=dt, device=dev)
-        self.theta_R = torch.zeros(dout // b, P, dtype=torch.float32, device=dev)
-        self.theta_P = torch.zeros(din // b, P, dtype=torch.float32, device=dev)
+        # theta_R and theta_P (and their gradients and AdamW moments) are stored back to back so
+        # that one optimiser launch covers both sides.
+        nbo, nbi = dout // b, din // b
+        self.theta = torch.zeros(nbo + nbi, P, dtype=torch.float32, device=dev)
+        self.theta_R, self.theta_P = self.theta[:nbo], self.theta[nbo:]
         self.perm_L = torch.arange(dout, dtype=torch.int32, device=dev)
         self.perm_R = torch.arange(din, dtype=torch.int32, device=dev)
         self.Q_R = torch.empty(dout // b, b, b, dtype=dt, device=dev)
@@ -45,8 +49,12 @@ class PoetxLayer:
         pw = poetx_cnp_powers_size(desc) if desc.mode == POETX_FAST else 0
         self.powers = torch.empty(pw, dtype=torch.uint8, device=dev) if pw else None
         self.dX = torch.empty(self.n, din, dtype=dt, device=dev)
-        self.g_R = torch.empty_like(self.theta_R)
-        self.g_P = torch.empty_like(self.theta_P)
+        self.grad = torch.zeros_like(self.theta)
+        self.g_R, self.g_P = self.grad[:nbo], self.grad[nbo:]
+        self.m = torch.zeros_like(self.theta)
+        self.v = torch.zeros_like(self.theta)
+        self.t = 0       # AdamW step count of the current moments
+        self.steps = 0   # training steps taken (drives the merge schedule)
         ws = poetx_workspace_size(desc, self.n)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
 
@@ -83,6 +91,29 @@ class PoetxLayer:
         self.cnp()
         self.forward(X)
         self.backward(dY, X)
+
+    def optimizer_step(self, cfg: poetx_adamw_cfg):
+        """AdamW on the packed theta (both sides in one launch)."""
+        self.t += 1
+        poetx_adamw_step(cfg, self.theta.numel(), self.t, self.theta, self.grad, self.m, self.v)
+
+    def train_step(self, X: torch.Tensor, dY: torch.Tensor, cfg: poetx_adamw_cfg, reset_gap: int = 400,
+                   new_perms=None):
+        """One training step with the merge schedule: CNP, forward, backward, AdamW; after every
+        reset_gap steps merge-then-reinitialise with the permutations new_perms() returns
+        (host int32 arrays pi_L, pi_R) and restart the moments."""
+        self.step(X, dY)
+        self.optimizer_step(cfg)
+        self.steps += 1
+        if reset_gap and self.steps % reset_gap == 0:
+            if new_perms is None:
+                raise ValueError("the merge schedule needs new permutations")
+            pL, pR = new_perms()
+            self.cnp()  # Q of the theta being folded in
+            self.merge(torch.from_numpy(np.asarray(pL, np.int32)).to(self.device),
+                       torch.from_numpy(np.asarray(pR, np.int32)).to(self.device))
+            poetx_adamw_reset(self.m.numel(), self.m, self.v)
+            self.t = 0
 
     def merge(self, pi_L_new: torch.Tensor, pi_R_new: torch.Tensor):
         """Folds R and P into W0', absorbs the new permutations and resets theta (Q must be current)."""

@@ -113,3 +113,18 @@ def test_gemm_hook_rejects_out_of_range_views():
                                  1 << 20, 64, 64, 64, 0, 0, 0, 1 << 20, 0, 64, 0, 0, 0,
                                  1.0, 0.0, None, 0, 0, 0, 0, None)
     assert st == 1
+
+
+def test_adamw_host_validation():
+    L = P.lib()
+    A = 1 << 20
+    ok = P.poetx_adamw_cfg(1e-3, 0.5, 0.9, 0.999, 1e-8, 0.0)
+    assert L.poetx_adamw_step(ctypes.byref(ok), 0, 1, A, A, A, A, None) == 0  # nothing to do
+    assert L.poetx_adamw_step(ctypes.byref(ok), 16, 0, A, A, A, A, None) == 1  # t < 1
+    assert L.poetx_adamw_step(ctypes.byref(ok), -1, 1, A, A, A, A, None) == 1
+    assert L.poetx_adamw_step(ctypes.byref(ok), 16, 1, A, None, A, A, None) == 1
+    assert L.poetx_adamw_step(ctypes.byref(ok), 16, 1, A, A, A + 4, A, None) == 3
+    for bad in (P.poetx_adamw_cfg(1e-3, 0.5, 1.0, 0.999, 1e-8, 0.0), P.poetx_adamw_cfg(1e-3, 0.5, 0.9, 0.999, 0.0, 0.0),
+                P.poetx_adamw_cfg(-1.0, 0.5, 0.9, 0.999, 1e-8, 0.0), P.poetx_adamw_cfg(1e-3, 0.5, 0.9, 0.999, 1e-8, -1.0)):
+        assert L.poetx_adamw_step(ctypes.byref(bad), 16, 1, A, A, A, A, None) == 1
+    assert L.poetx_adamw_reset(-1, A, A, None) == 1 and L.poetx_adamw_reset(0, None, None, None) == 0
