@@ -55,6 +55,12 @@ def step_flops(s: I.LayerShape) -> dict:
     return {"fwd": fwd, "bwd": bwd, "cnp": cnp, "total": fwd + bwd + cnp}
 
 
+# DRAM bytes (read + write) of one W0' launch, from the ncu capture summarised in
+# profiles/gemm_w256_fwd_2048x4096x4096_b256_ncu.md (bench workload, forward launch).  Only valid
+# for that workload and that kernel build; None otherwise.
+W_GEMM_TRAFFIC = {"llama8b_attn_4096_b256_bf16": 52.461056e6 + 3.457792e6}
+
+
 def w_gemm_flops(s: I.LayerShape) -> int:
     """Algorithmic FLOPs of one launch of the dominant kernel, the W0' GEMM (Z = V W0'^T or
     dV = dZ W0'); for bf16 and b = 256 that launch also applies the block factor on its output
@@ -159,6 +165,15 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def dp_allreduce(grad, world: int) -> None:
+    """The exchange step of data-parallel training: sum the packed theta gradients of all ranks
+    in place (theta_R and theta_P are stored back to back, so one collective moves both)."""
+    if world <= 1:
+        return
+    import torch.distributed as dist
+    dist.all_reduce(grad, op=dist.ReduceOp.SUM)
+
+
 def shard_seed(base_seed: int, rank: int) -> int:
     """Each rank draws its own tokens (the layer state is shared by construction)."""
     return base_seed + 7919 * rank
@@ -234,6 +249,7 @@ def run_poetx(args):
 
     for _ in range(args.warmup):
         layer.step(X, dY)
+        dp_allreduce(layer.grad, world)
     torch.cuda.synchronize()
     st, det = P.poetx_device_status()
     if st != 0:
@@ -255,6 +271,7 @@ def run_poetx(args):
             graph.replay()
         else:
             layer.step(X, dY)
+        dp_allreduce(layer.grad, world)  # N > 1: the packed gradients are summed over ranks
 
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -358,6 +375,7 @@ def run_poetx(args):
             egraphs[i % 2].replay()
         else:
             layer.step(Xb[i % 2], dYb[i % 2])
+        dp_allreduce(layer.grad, world)
         gRs[i % 2].copy_(layer.g_R)
         gPs[i % 2].copy_(layer.g_P)
         ev_done[i].record(stream)
@@ -431,12 +449,16 @@ def run_poetx(args):
                    "step": "CNP fwd (R,P) + forward + backward incl. CNP adjoint",
                    "l2": "flushed between steps (256 MiB write outside the timed intervals)",
                    "launch": "CUDA graph of one step, replayed" if graph is not None else "direct launches",
-                   "parallelism": f"replicas x{world} (data parallel over tokens, no collective on the path)",
+                   "parallelism": (f"dp{world}: data parallel over tokens, replicas plus an NCCL all-reduce of the "
+                                   f"packed theta gradients ({4 * layer.grad.numel()} bytes) every step"
+                                   if world > 1 else "dp1 (one replica; the gradient all-reduce needs N > 1)"),
                    "algorithmic_gflop_per_step": round(fl["total"] / 1e9, 2)},
         "roofline": {"bound": "tensor",
                      "kernel": "w0_gemm (Z = V W0'^T with Y' = BD_R Z; dV = dZ W0' with dU = BD_P^T dV)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": W_GEMM_TRAFFIC.get(args.workload),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one forward launch "
+                                       "(profiles/gemm_w256_fwd_2048x4096x4096_b256_ncu.md)",
                      "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                      "frac_of_sustained": round(achieved / float(peaks["bf16_tflops_sustained"]), 4),
                      "launch_ms": round(w_avg_ms, 4), "launches": wcnt},

@@ -95,13 +95,27 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Shared memory of the program kernel: the TMA ring, or two padded 128 x BN f32 staging tiles
-// (whichever is larger), then the barriers.
+// Shared memory of the program kernel: the TMA ring of the GEMM stages, overlaid by the staging
+// of the elementwise stages (UNPACK: theta row segments above the diagonal, 128 x (BN + 8) f32,
+// and column segments below it, BN x 136 f32, plus the G tile, 128 x (BN + 4) f32; PACK: the
+// own G_S tile and the rows of the mirrored one, 128 x (BN + 4) and BN x 132 f32), then the
+// barriers.
+// UNPACK staging: the theta segments of a tile (at most 128 x BN elements in all, plus 11
+// floats of alignment slack per segment), then the assembled S tile (pitch BN + 1) and the G
+// tile (pitch BN + 4).
+template <int BN>
+__host__ __device__ constexpr size_t cnp_stage_bytes() {
+  return (((size_t)TC_BM * BN + 11 * (size_t)(TC_BM + BN)) * 4 + 1023) / 1024 * 1024;
+}
+template <int BN>
+__host__ __device__ constexpr size_t cnp_ew_bytes() {
+  return cnp_stage_bytes<BN>() + (size_t)TC_BM * (BN + 1) * 4 + (size_t)TC_BM * (BN + 4) * 4 + 2048;
+}
 template <int BN, int STAGES>
 __host__ __device__ constexpr size_t cnp_data_bytes() {
-  return (size_t)STAGES * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) > (size_t)2 * TC_BM * (BN + 4) * 4
-             ? (size_t)STAGES * (TC_BM * TC_BK * 2 + BN * TC_BK * 2)
-             : ((size_t)2 * TC_BM * (BN + 4) * 4 + 1023) / 1024 * 1024;
+  return ((size_t)STAGES * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) > cnp_ew_bytes<BN>()
+              ? (size_t)STAGES * (TC_BM * TC_BK * 2 + BN * TC_BK * 2)
+              : cnp_ew_bytes<BN>() + 1023) / 1024 * 1024;
 }
 template <int BN, int STAGES>
 __host__ __device__ constexpr size_t cnp_smem_bytes() {
@@ -121,11 +135,12 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + cnp_data_bytes<BN, STAGES>());
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
   const uint32_t smem0 = smem_u32(smem);
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
   const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
+  const uint32_t ew_bar = smem_u32(bars + 2 * STAGES + 1);  // bulk copies of an elementwise stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3, half = warp >> 2;
@@ -147,6 +162,7 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(accum_bar, 1);
+    mbar_init(ew_bar, CNP_THREADS);
     fence_mbar_init();
     fence_proxy_async_smem();
   }
@@ -159,28 +175,21 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
   tc_fence_after();
   const uint32_t tmem0 = *tmem_holder;
   const uint32_t tlane = tmem0 + ((uint32_t)(quarter * 32) << 16);
+  griddep_wait();  // theta and the gradient partials come from earlier kernels
   auto treg = [&](int reg, int col) { return tlane + (uint32_t)(reg * BN + col); };
-  // Two 128 x BN f32 staging tiles (padded row stride), overlaid on the TMA ring, which is idle
-  // whenever they are in use (between the last MMA of a stage and the first TMA load of the next).
-  constexpr int TS = BN + 4;  // padded row stride (16-byte aligned rows for float4 access)
-  float* T0 = reinterpret_cast<float*>(smem);
-  float* T1 = T0 + TC_BM * TS;
-  // Coalesced write of a staged tile to global: warps over rows, lanes along columns.  With
-  // `skew` the tile holds theta unsigned and entries below the diagonal are negated on the way.
-  auto tile_store = [&](const float* T, void* dst, long ld, int dt, bool skew) {
+  // The elementwise stages stage their tiles in the TMA ring, which is idle whenever they run
+  // (between the last MMA of a stage and the first TMA load of the next).
+  constexpr int TS = BN + 4;  // padded row stride of a staged f32 tile (16-byte aligned rows)
+  // Coalesced write of a staged f32 tile (row pitch `pitch` floats) to global: warps over rows,
+  // lanes along columns, four columns per lane.
+  auto tile_store = [&](const float* T, int pitch, void* dst, long ld, int dt) {
     for (int r = warp; r < TC_BM; r += CNP_THREADS / 32) {
       const int ii = m0 + r;
       if (ii >= b) break;
       const long base = ((long)z * b + ii) * ld + n0;
       for (int cc = lane * 4; cc < BN; cc += 128) {
-        float4 f = *reinterpret_cast<const float4*>(T + r * TS + cc);
-        if (skew) {
-          const int jj = n0 + cc;
-          if (jj < ii) f.x = -f.x;
-          if (jj + 1 < ii) f.y = -f.y;
-          if (jj + 2 < ii) f.z = -f.z;
-          if (jj + 3 < ii) f.w = -f.w;
-        }
+        const float* src = T + r * pitch + cc;
+        const float4 f = make_float4(src[0], src[1], src[2], src[3]);
         if (dt == BF16) {
           uint2 u;
           u.x = pack_bf16x2(f.x, f.y);
@@ -194,9 +203,22 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
   };
   uint32_t it = 0;
   uint32_t acc_phase = 0;
+  uint32_t ew_phase = 0;
+  // One 1-D bulk copy per thread (or none) of `bytes` from global `src` to shared `dst`, counted
+  // on ew_bar; every thread arrives exactly once.
+  auto bulk_one = [&](void* dst, const void* src, uint32_t bytes) {
+    if (bytes > 0) {
+      fence_proxy_async_smem();  // the copy overwrites what earlier stages wrote and read
+      mbar_arrive_expect_tx(ew_bar, bytes);
+      bulk_load_1d(smem_u32(dst), src, bytes, ew_bar);
+    } else {
+      mbar_arrive(ew_bar);
+    }
+  };
 
   for (int s = 0; s < prog.nstages; ++s) {
     const CnpStageDesc& D = prog.st[s];
+    if (s == prog.nstages - 1) griddep_launch();
     bool wrote_global = false, wrote_tmem = false;
     if (D.kind == CNP_GEMM) {
       const CnpSegStage& G = prog.g[s][seg];
@@ -326,60 +348,67 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         __syncwarp();
       }
     } else if (D.kind == CNP_UNPACK || D.kind == CNP_REDUCE_UNPACK) {
-      // theta -> T0 by per-thread asynchronous copies (all of a thread's copies in flight at
-      // once, no registers held): above the diagonal warps walk rows (theta's packed row i is
-      // contiguous in j), below it warps walk columns (packed row j is contiguous in i).  T0
-      // holds theta unsigned; the consumers negate below the diagonal.  Packed row i starts at
-      // ro(i) + i + 1 with ro(i) = i*b - i(i+1)/2 - i - 1, so element (i, j) is ro(i) + j.
-      constexpr int RW = TC_BM / (CNP_THREADS / 32);  // rows (or columns) per warp
-      constexpr int CPL = BN / 32;                    // columns (or rows / 32) per lane
-      constexpr int RPL = TC_BM / 32;                 // rows per lane in the column walk
-      const float diag = S.add_identity ? 1.f : 0.f;
-#pragma unroll 4
-      for (int t = 0; t < RW; ++t) {
-        const int r = warp + 8 * t, ii = m0 + r;
-        const int ro = ii * b - (ii * (ii + 1)) / 2 - ii - 1;
-#pragma unroll
-        for (int q = 0; q < CPL; ++q) {
-          const int cc = lane + 32 * q, jj = n0 + cc;
-          float* dst = T0 + r * TS + cc;
-          if (jj > ii) {
-            if (ii < b) cp_async4(dst, th + (ro + jj));
-            else *dst = 0.f;
-          } else if (jj == ii) {
-            *dst = diag;
-          }
+      // theta -> S.  Above the diagonal the tile row r (i = m0 + r) needs the segment
+      // j = max(n0, i+1) .. n0+BN-1 of packed row i; below it tile column cc (j = n0 + cc) needs
+      // the segment i = max(m0, j+1) .. min(m0+128, b)-1 of packed row j (S[i][j] = -theta[p(j,i)]).
+      // Each segment is one 1-D bulk copy of its 16-byte-aligned cover into a compact staging
+      // area (thread t < 128: row t; 128 <= t < 128 + BN: column t - 128; element e of a
+      // segment starting at packed offset e0 sits at e0 % 4 + e of its slot), then the tile is
+      // assembled in T0 (pitch BN + 1): rows with lanes along j, columns with lanes along i,
+      // both conflict-free.  Packed row i starts at ro(i) + i + 1, ro(i) = i*b - i(i+1)/2 - i - 1.
+      constexpr int RW = TC_BM / (CNP_THREADS / 32), T0P = BN + 1, CPL = BN / 32, RPL = TC_BM / 32;
+      float* Sg = reinterpret_cast<float*>(smem);
+      float* T0 = reinterpret_cast<float*>(smem + cnp_stage_bytes<BN>());
+      float* Gt = T0 + TC_BM * T0P;  // G tile (REDUCE), row pitch TS
+      int* seg_off = reinterpret_cast<int*>(Gt + TC_BM * TS);  // [256]: slot start + e0 % 4
+      auto ro = [&](int r) { return r * b - (r * (r + 1)) / 2 - r - 1; };
+      auto seg_of = [&](int t, int& e0, int& cnt) {  // segment of thread t's row / column
+        e0 = 0; cnt = 0;
+        if (t < TC_BM) {
+          const int ii = m0 + t, jlo = max(n0, ii + 1);
+          if (ii < b && jlo < n0 + BN) { e0 = ro(ii) + jlo; cnt = n0 + BN - jlo; }
+        } else if (t < TC_BM + BN) {
+          const int jj = n0 + t - TC_BM, ilo = max(m0, jj + 1), ihi = min(m0 + TC_BM, b);
+          if (ilo < ihi) { e0 = ro(jj) + ilo; cnt = ihi - ilo; }
         }
-      }
-#pragma unroll 4
-      for (int t = 0; t < BN / 8; ++t) {
-        const int cc = warp + 8 * t, jj = n0 + cc;
-        const int ro = jj * b - (jj * (jj + 1)) / 2 - jj - 1;
+      };
+      {
+        const int t = threadIdx.x;
+        int e0, cnt;
+        seg_of(t, e0, cnt);
+        // slot start: exclusive prefix sum over threads of len + 11 floats rounded up to 4
+        const int cap = cnt > 0 ? (cnt + 11) & ~3 : 0;
+        int x = cap;
 #pragma unroll
-        for (int q = 0; q < RPL; ++q) {
-          const int r = lane + 32 * q, ii = m0 + r;
-          if (ii > jj) {
-            float* dst = T0 + r * TS + cc;
-            if (ii < b) cp_async4(dst, th + (ro + ii));
-            else *dst = 0.f;
-          }
+        for (int d = 1; d < 32; d <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, d);
+          if (lane >= d) x += y;
         }
+        int* warp_sum = seg_off + CNP_THREADS;
+        if (lane == 31) warp_sum[warp] = x;
+        __syncthreads();
+        int off = x - cap;
+        for (int w = 0; w < warp; ++w) off += warp_sum[w];
+        seg_off[t] = off + (e0 & 3);
+        // block z's theta starts 16-byte aligned (P * 4 is a multiple of 16 for b % 8 == 0), so
+        // the rounded cover never leaves it
+        const int b0 = (e0 * 4) & ~15, b1 = ((e0 + cnt) * 4 + 15) & ~15;
+        bulk_one(Sg + off, reinterpret_cast<const char*>(th) + b0, cnt > 0 ? (uint32_t)(b1 - b0) : 0u);
       }
       if (D.kind == CNP_REDUCE_UNPACK && S.splits == 1) {
-        // G (one partial: the gradient GEMM did not split K) -> T1, 16-byte copies by rows.
+        // G (one partial: the gradient GEMM did not split K) -> Gt, 16-byte copies by rows.
         if (lane * 4 < BN) {
 #pragma unroll 4
           for (int t = 0; t < RW; ++t) {
             const int ii = m0 + warp + 8 * t;
-            float* dst = T1 + (warp + 8 * t) * TS + lane * 4;
+            float* dst = Gt + (warp + 8 * t) * TS + lane * 4;
             if (ii < b) cp_async16(dst, S.part + ((long)z * b + ii) * b + n0 + lane * 4);
             else *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
       }
-      cp_async_wait_all();
       if (D.kind == CNP_REDUCE_UNPACK && S.splits > 1) {
-        // G = sum of split-K partials -> T1, row walk with one float4 per lane per row.
+        // G = sum of split-K partials -> Gt, row walk with one float4 per lane per row.
         const long sstride = (long)S.nb * b * b;
         constexpr int RB = 4;
 #pragma unroll 1
@@ -407,37 +436,59 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
           }
 #pragma unroll
           for (int t = 0; t < RB; ++t)
-            if (lane * 4 < BN) *reinterpret_cast<float4*>(T1 + (warp + 8 * (t0 + t)) * TS + lane * 4) = acc4[t];
+            if (lane * 4 < BN) *reinterpret_cast<float4*>(Gt + (warp + 8 * (t0 + t)) * TS + lane * 4) = acc4[t];
+        }
+      }
+      cp_async_wait_all();
+      bool got = mbar_wait(ew_bar, ew_phase, KID_CNP_FUSED, 4);
+      ew_phase ^= 1u;
+      got = __syncthreads_and(got);
+      // Assemble T0 = S tile.  Rows (warps over rows, lanes along columns): the part above the
+      // diagonal, the diagonal, and zero rows past b.
+      const float diag = S.add_identity ? 1.f : 0.f;
+#pragma unroll 2
+      for (int t = 0; t < RW; ++t) {
+        const int r = warp + 8 * t, ii = m0 + r, c0 = max(n0, ii + 1) - n0, so = seg_off[r];
+#pragma unroll
+        for (int q = 0; q < CPL; ++q) {
+          const int cc = lane + 32 * q, jj = n0 + cc;
+          float x = 0.f;
+          if (ii < b && got) x = jj > ii ? Sg[so + cc - c0] : (jj == ii ? diag : 0.f);
+          if (jj >= ii || ii >= b) T0[r * T0P + cc] = x;
+        }
+      }
+      // Columns (threads over columns, lanes along rows): the part below the diagonal.
+#pragma unroll 2
+      for (int t = 0; t < BN / 8; ++t) {
+        const int cc = warp + 8 * t, jj = n0 + cc, r0 = max(m0, jj + 1) - m0, so = seg_off[TC_BM + cc];
+#pragma unroll
+        for (int q = 0; q < RPL; ++q) {
+          const int r = lane + 32 * q, ii = m0 + r;
+          if (ii > jj && ii < b) T0[r * T0P + cc] = got ? -Sg[so + r - r0] : 0.f;
         }
       }
       __syncthreads();
-      // Coalesced global copies from the tiles; then each thread moves its row into TMEM.
-      if (S.Sb0) tile_store(T0, S.Sb0, S.ld0, BF16, true);
-      if (S.Sb1) tile_store(T0, S.Sb1, S.ld1, BF16, true);
+      // Coalesced bf16 copies of S and G (warps over rows, lanes along columns); then each
+      // thread moves its row into TMEM.
+      if (S.Sb0) tile_store(T0, T0P, S.Sb0, S.ld0, BF16);
+      if (S.Sb1) tile_store(T0, T0P, S.Sb1, S.ld1, BF16);
       if (D.kind == CNP_REDUCE_UNPACK) {
-        if (S.Gb) tile_store(T1, S.Gb, S.ldg, BF16, false);
-        if (S.G32) tile_store(T1, S.G32, b, F32, false);
+        if (S.Gb) tile_store(Gt, TS, S.Gb, S.ldg, BF16);
+        if (S.G32) tile_store(Gt, TS, S.G32, b, F32);
       }
       wrote_global = true;
 #pragma unroll 1
       for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
         uint32_t w[32];
         if (!S.no_sreg) {
-          const float4* trow = reinterpret_cast<const float4*>(T0 + (quarter * 32 + lane) * TS + c);
-          const int neg_below = i - (n0 + c);  // columns j < neg_below of this chunk lie below the diagonal
+          const float* trow = T0 + (quarter * 32 + lane) * T0P + c;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 f = trow[j];
-            w[4 * j] = __float_as_uint(4 * j < neg_below ? -f.x : f.x);
-            w[4 * j + 1] = __float_as_uint(4 * j + 1 < neg_below ? -f.y : f.y);
-            w[4 * j + 2] = __float_as_uint(4 * j + 2 < neg_below ? -f.z : f.z);
-            w[4 * j + 3] = __float_as_uint(4 * j + 3 < neg_below ? -f.w : f.w);
-          }
+          for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(trow[j]);
           tmem_st_32x32b_x32(treg(CNP_R1, c), w);
           wrote_tmem = true;
         }
         if (D.kind == CNP_REDUCE_UNPACK) {
-          const float4* grow4 = reinterpret_cast<const float4*>(T1 + (quarter * 32 + lane) * TS + c);
+          const float4* grow4 = reinterpret_cast<const float4*>(Gt + (quarter * 32 + lane) * TS + c);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float4 f = grow4[j];
@@ -449,33 +500,36 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         }
       }
     } else if (D.kind == CNP_PACK) {
-      // T0 = own tile of G_S (16-byte copies by rows), T1[i][j] = G_S[j][i] (4-byte copies,
-      // column walk, contiguous in i); then g[p(i,j)] = T0 - T1 with lanes along j (contiguous
-      // in p).  All copies of a thread are in flight at once.
-      constexpr int RW = TC_BM / (CNP_THREADS / 32);
-      constexpr int RPL = TC_BM / 32;
-      if (lane * 4 < BN) {
-#pragma unroll 4
-        for (int t = 0; t < RW; ++t) {
-          const int ii = m0 + warp + 8 * t;
-          if (ii < b) cp_async16(T0 + (warp + 8 * t) * TS + lane * 4, S.GS + ((long)z * b + ii) * b + n0 + lane * 4);
+      // Own tile of G_S -> Tp (rows, pitch TS) and rows n0.. of G_S restricted to columns m0..
+      // -> Tt (row cc holds G_S[n0+cc][m0 + r], pitch 132): one 1-D bulk copy per row (thread
+      // t < 128: own row t; 128 <= t < 128 + BN: mirrored row t - 128).  Then
+      // g[p(i,j)] = G_S[i][j] - G_S[j][i] with lanes along j (contiguous in p).
+      constexpr int TP = TC_BM + 4;
+      float* Tp = reinterpret_cast<float*>(smem);
+      float* Tt = Tp + TC_BM * TS;
+      {
+        const int t = threadIdx.x;
+        if (t < TC_BM) {
+          const int ii = m0 + t;
+          bulk_one(Tp + t * TS, S.GS + ((long)z * b + ii) * b + n0, ii < b ? (uint32_t)(BN * 4) : 0u);
+        } else if (t < TC_BM + BN) {
+          const int cc = t - TC_BM;
+          bulk_one(Tt + cc * TP, S.GS + ((long)z * b + n0 + cc) * b + m0, (uint32_t)(min(TC_BM, b - m0) * 4));
+        } else {
+          bulk_one(nullptr, nullptr, 0u);
         }
       }
-#pragma unroll 4
-      for (int t = 0; t < BN / 8; ++t)
-#pragma unroll
-        for (int q = 0; q < RPL; ++q) {
-          const int jj = n0 + warp + 8 * t, ii = m0 + lane + 32 * q;
-          if (ii < b) cp_async4(T1 + (lane + 32 * q) * TS + warp + 8 * t, S.GS + ((long)z * b + jj) * b + ii);
-        }
-      cp_async_wait_all();
-      __syncthreads();
-      for (int r = warp; r < TC_BM; r += CNP_THREADS / 32) {
-        const int ii = m0 + r;
-        if (ii >= b) break;
-        for (int cc = lane; cc < BN; cc += 32) {
-          const int jj = n0 + cc;
-          if (ii < jj) S.grad[(long)z * P + packed_pos(ii, jj, b)] = T0[r * TS + cc] - T1[r * TS + cc];
+      bool got = mbar_wait(ew_bar, ew_phase, KID_CNP_FUSED, 5);
+      ew_phase ^= 1u;
+      got = __syncthreads_and(got);
+      if (got) {
+        for (int r = warp; r < TC_BM; r += CNP_THREADS / 32) {
+          const int ii = m0 + r;
+          if (ii >= b) break;
+          for (int cc = lane; cc < BN; cc += 32) {
+            const int jj = n0 + cc;
+            if (ii < jj) S.grad[(long)z * P + packed_pos(ii, jj, b)] = Tp[r * TS + cc] - Tt[cc * TP + r];
+          }
         }
       }
     }

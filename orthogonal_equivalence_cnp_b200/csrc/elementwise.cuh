@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(256, ROWS == 4 ? 3 : 2)
     permute_cols_bf16_kernel(const uint16_t* __restrict__ in, long ld_in, uint16_t* __restrict__ out, long ld_out,
                              long rows, int cols, const int32_t* __restrict__ colmap,
                              const int32_t* __restrict__ rowmap, int scatter) {
+  sm100::griddep_wait();
   using Word = typename std::conditional<ROWS == 4, uint64_t, uint32_t>::type;
   extern __shared__ __align__(16) uint8_t smem_perm[];
   uint16_t* src_of = reinterpret_cast<uint16_t*>(smem_perm);  // output column j reads source column src_of[j]
@@ -177,6 +178,7 @@ __global__ void __launch_bounds__(256, 2)
     permute_cols_bulk_kernel(const uint16_t* __restrict__ in, long ld_in, uint16_t* __restrict__ out, long ld_out,
                              long rows, int cols, const int32_t* __restrict__ colmap,
                              const int32_t* __restrict__ rowmap, int scatter) {
+  sm100::griddep_wait();
   using Word = typename std::conditional<ROWS == 4, uint64_t, uint32_t>::type;
   extern __shared__ __align__(128) uint8_t smem_bulk[];
   const size_t slot_bytes = (size_t)ROWS * cols * 2;
@@ -233,6 +235,7 @@ __global__ void __launch_bounds__(256, 2)
     }
   }
   __syncthreads();  // barriers initialised, map complete
+  sm100::griddep_launch();
 
   bool ok = true;
   int i = 0;
@@ -316,6 +319,7 @@ __device__ __forceinline__ void adamw_one(float& th, float g, float& m, float& v
 __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ theta, const float* __restrict__ grad,
                                                     float* __restrict__ m, float* __restrict__ v, long n,
                                                     const AdamwArgs a) {
+  sm100::griddep_wait();
   const long n4 = n / 4;
   const long stride = (long)gridDim.x * blockDim.x;
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
@@ -340,6 +344,7 @@ __global__ void __launch_bounds__(256)
     permute_cols_f32_kernel(const float* __restrict__ in, long ld_in, float* __restrict__ out, long ld_out, long rows,
                             int cols, const int32_t* __restrict__ colmap, const int32_t* __restrict__ rowmap,
                             int scatter) {
+  sm100::griddep_wait();
   extern __shared__ __align__(16) uint8_t smem_perm[];
   float* row = reinterpret_cast<float*>(smem_perm);
   for (long r = blockIdx.x; r < rows; r += gridDim.x) {
@@ -361,6 +366,7 @@ __global__ void __launch_bounds__(256)
 // Up to two typed outputs (element (z*b+i, j) at o[(z*b+i)*ld + j]) and one contiguous f32 one.
 __global__ void unpack_skew_kernel(const float* __restrict__ theta, long nblocks, int b, void* o1, int dt1,
                                    long ld1, void* o2, int dt2, long ld2, float* of32, int add_identity) {
+  sm100::griddep_wait();
   const long bb = (long)b * b;
   const long total = nblocks * bb;
   const long P = (long)b * (b - 1) / 2;
@@ -382,6 +388,7 @@ __global__ void unpack_skew_kernel(const float* __restrict__ theta, long nblocks
 // Gradient w.r.t. the packed parameters: g[p(i,j)] = GS[i][j] - GS[j][i] (theta enters S with
 // +1 above and -1 below the diagonal).  GS is [nblocks, b, b] f32 contiguous.
 __global__ void pack_antisym_kernel(const float* __restrict__ GS, long nblocks, int b, float* __restrict__ g) {
+  sm100::griddep_wait();
   const long bb = (long)b * b;
   const long total = nblocks * bb;
   const long P = (long)b * (b - 1) / 2;
@@ -397,6 +404,7 @@ __global__ void pack_antisym_kernel(const float* __restrict__ GS, long nblocks, 
 // row stride ld2.
 __global__ void reduce_splits_kernel(const float* __restrict__ part, int splits, long split_stride, long rows,
                                      int cols, float* __restrict__ out, void* out2, int dt2, long ld2) {
+  sm100::griddep_wait();
   const long total = rows * cols;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (long)gridDim.x * blockDim.x) {
     float s = 0.f;
@@ -410,12 +418,14 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, int splits,
 }
 
 __global__ void perm_inverse_kernel(const int32_t* __restrict__ perm, int n, int32_t* __restrict__ inv) {
+  sm100::griddep_wait();
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < n; j += gridDim.x * blockDim.x) inv[perm[j]] = j;
 }
 
 // sigma[i] = inv_old[new[i]]
 __global__ void perm_compose_kernel(const int32_t* __restrict__ inv_old, const int32_t* __restrict__ pnew, int n,
                                     int32_t* __restrict__ sigma) {
+  sm100::griddep_wait();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) sigma[i] = inv_old[pnew[i]];
 }
 

@@ -247,6 +247,7 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_holder;
+  griddep_wait();  // operands and epilogue addends may come from the previous kernel
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -296,6 +297,7 @@ __global__ void __launch_bounds__(128)
   bool ok = mbar_wait(accum_bar, 0, KID_GEMM_TC, 3);
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
+  griddep_launch();
   if (ok && args.tma_store) {
     // Each warp stages its 32 rows x 64 columns as a 128-byte-swizzled box (two 4 KiB buffers
     // per warp in the idle ring) and lane 0 stores it with TMA: whole lines instead of one
@@ -409,6 +411,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_holder;
+  griddep_wait();
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer: the K loop, then this block's Q into the ring's B halves.
@@ -470,6 +473,7 @@ __global__ void __launch_bounds__(128, 1)
   bool ok = mbar_wait(accum_bar, 0, KID_GEMM_TC, 8);
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
+  griddep_launch();
   const int r = warp * 32 + lane;  // tile row
   const int m = m0 + r;
   if (ok) {
@@ -620,6 +624,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_holder;
+  griddep_wait();
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -685,6 +690,7 @@ __global__ void __launch_bounds__(128, 1)
   bool ok = mbar_wait(accum_bar, 0, KID_GEMM_TC, 14);
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
+  griddep_launch();
   const int r = warp * 32 + lane;  // TMEM lane = row within a half
   const uint32_t tl = tmem_d + ((uint32_t)(warp * 32) << 16);
 
@@ -807,6 +813,7 @@ struct SimtArgs {
 
 // 64x64 output tile per 256-thread block, 4x4 per thread, k-steps of 16 staged in smem.
 __global__ void __launch_bounds__(256) gemm_f32_simt(const SimtArgs p) {
+  sm100::griddep_wait();
   __shared__ float As[16][65];
   __shared__ float Bs[16][65];
   const int z = blockIdx.z / p.splits, split = blockIdx.z % p.splits;

@@ -111,6 +111,24 @@ struct LaunchScope {
   }
 };
 
+// Launch with a programmatic dependency on the previous kernel of the stream: the kernel may
+// be scheduled while that one finishes and waits for it in griddep_wait() before touching its
+// results (every kernel of this library does).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 poetx_status check_desc(const poetx_desc* d) {
   if (d == nullptr) return POETX_ERR_INVALID_ARG;
   if (d->dtype != POETX_F32 && d->dtype != POETX_BF16) return POETX_ERR_INVALID_ARG;
@@ -230,7 +248,7 @@ poetx_status launch_tc(const GemmDesc& g, cudaStream_t st, int cls) {
   }
   dim3 grid(g.N / BN, (g.M + TC_BM - 1) / TC_BM, g.batch * g.splits);
   LaunchScope ls(cls, st);
-  kern<<<grid, 128, smem, st>>>(ta, tb, td, a);
+  if (launch_pdl(kern, grid, dim3(128), smem, st, ta, tb, td, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
 }
 
@@ -267,7 +285,7 @@ poetx_status run_gemm(int dt, const GemmDesc& g, cudaStream_t st, int cls) {
   p.epi = g.epi;
   dim3 grid((g.N + 63) / 64, (g.M + 63) / 64, g.batch * g.splits);
   LaunchScope ls(cls, st);
-  gemm_f32_simt<<<grid, 256, 0, st>>>(p);
+  if (launch_pdl(gemm_f32_simt, grid, dim3(256), 0, st, p) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
 }
 
@@ -292,8 +310,9 @@ poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld
     const long groups = (rows + (four ? 4 : 2) - 1) / (four ? 4 : 2);
     const int grid = (int)std::min<long>(groups, (long)kNumSms * per_sm);
     LaunchScope ls(POETX_KC_PERMUTE, st);
-    k<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(in), ld_in, static_cast<uint16_t*>(out), ld_out, rows,
-                               cols, colmap, rowmap, scatter ? 1 : 0);
+    if (launch_pdl(k, dim3(grid), dim3(256), smem, st, static_cast<const uint16_t*>(in), ld_in,
+                   static_cast<uint16_t*>(out), ld_out, rows, cols, colmap, rowmap, scatter ? 1 : 0) != cudaSuccess)
+      return POETX_ERR_CUDA;
   } else if (dt == BF16) {
     // Groups of four rows (two for very wide rows); as many blocks as fit.
     const bool four = permute_smem_bytes<4>(cols) <= 160 * 1024;
@@ -310,8 +329,9 @@ poetx_status permute_cols(int dt, const void* in, long ld_in, void* out, long ld
     const long want = cols <= 4096 ? std::min<long>(groups, std::max<long>(kNumSms, (groups + 1) / 2)) : groups;
     const int grid = (int)std::min<long>(want, (long)kNumSms * per_sm);
     LaunchScope ls(POETX_KC_PERMUTE, st);
-    k<<<grid, 256, smem, st>>>(static_cast<const uint16_t*>(in), ld_in, static_cast<uint16_t*>(out), ld_out, rows,
-                               cols, colmap, rowmap, scatter ? 1 : 0);
+    if (launch_pdl(k, dim3(grid), dim3(256), smem, st, static_cast<const uint16_t*>(in), ld_in,
+                   static_cast<uint16_t*>(out), ld_out, rows, cols, colmap, rowmap, scatter ? 1 : 0) != cudaSuccess)
+      return POETX_ERR_CUDA;
   } else {
     const size_t smem = (size_t)cols * 4;
     if (smem > 200 * 1024) return POETX_ERR_UNSUPPORTED_SHAPE;
@@ -381,7 +401,7 @@ poetx_status launch_bd_fused(const GemmDesc& g, const void* Q, long q_rows, void
   a.out2 = out2; a.ld2 = ld2;
   dim3 grid(g.N / 256, (g.M + TC_BM - 1) / TC_BM, 1);
   LaunchScope ls(POETX_KC_W_GEMM, st);
-  kern<<<grid, 128, smem, st>>>(ta, tb, tq, a);
+  if (launch_pdl(kern, grid, dim3(128), smem, st, ta, tb, tq, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
 }
 
@@ -434,7 +454,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.out2 = out2; a.ld2 = ld2;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(POETX_KC_W_GEMM, st);
-  kern<<<grid, 128, smem, st>>>(ta, tb, tq, td, a);
+  if (launch_pdl(kern, grid, dim3(128), smem, st, ta, tb, tq, td, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
 }
 
@@ -749,13 +769,15 @@ poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_
   cfg.blockDim = dim3(CNP_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = nt;
   attr[0].val.clusterDim.y = mt;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   LaunchScope ls(POETX_KC_CNP_GEMM, st);
   if (cudaLaunchKernelEx(&cfg, kern, pr) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
@@ -811,19 +833,21 @@ poetx_status cnp_fwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaS
     char* Sop = sd.ws + p.take(blk * 2);
     char* Mbuf[2] = {nullptr, nullptr};
     if (k >= 2 && sd.powers == nullptr) { Mbuf[0] = sd.ws + p.take(blk * 2); Mbuf[1] = sd.ws + p.take(blk * 2); }
-    S.Sb0 = Sop; S.ld0 = b;
     const long kb = (long)k * b;
-    // Kept powers: M_j goes to slot k - j of the stack (M_1 = S by the UNPACK stage).
+    // Kept powers: M_j goes to slot k - j of the stack, and M_1 = S is written there once by
+    // the UNPACK stage and read back from there as the A operand of every product.
     auto slot = [&](int j) { return static_cast<void*>(sd.powers + (size_t)(k - j) * b * 2); };
-    if (sd.powers) { S.Sb1 = slot(1); S.ld1 = kb; }
-    const void* Mprev = sd.powers ? slot(1) : Sop;
-    long ldprev = sd.powers ? kb : b;
+    const void* Sa = sd.powers ? slot(1) : Sop;
+    const long lds = sd.powers ? kb : b;
+    S.Sb0 = const_cast<void*>(Sa); S.ld0 = lds;
+    const void* Mprev = Sa;
+    long ldprev = lds;
     int s = 1;
     for (int j = 2; j <= k + 1; ++j, ++s) {
       const bool last = (j == k + 1);
       void* out = last ? sd.Q : (sd.powers ? slot(j) : Mbuf[j & 1]);
       const long ldout = (last || !sd.powers) ? b : kb;
-      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, Mprev, ldprev, true, b, out, ldout));
+      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sa, lds, Mprev, ldprev, true, b, out, ldout));
       Mprev = out;
       ldprev = ldout;
     }
@@ -1089,7 +1113,8 @@ poetx_status poetx_adamw_step(const poetx_adamw_cfg* cfg, long long n, int t, fl
   const long n4 = (long)(n / 4);
   const int grid = (int)std::max<long>(1, std::min<long>((n4 + 255) / 256, (long)kNumSms * 8));
   LaunchScope ls(POETX_KC_OPTIMIZER, stream);
-  adamw_kernel<<<grid, 256, 0, stream>>>(theta, grad, m, v, (long)n, a);
+  if (launch_pdl(adamw_kernel, dim3(grid), dim3(256), 0, stream, theta, grad, m, v, (long)n, a) != cudaSuccess)
+    return POETX_ERR_CUDA;
   return last_launch();
 }
 

@@ -62,6 +62,14 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 }
 // 2-D tiled load of one box into shared memory; completion is signalled on `bar` (tx bytes).
 // c0 is the innermost (contiguous) coordinate; callers keep c0 * elem_size a multiple of 16.
+// Programmatic dependent launch.  griddep_wait: block until the previous kernel of the stream
+// has completed and its memory operations are visible (a no-op without a programmatic
+// dependency); every kernel calls it before touching memory another kernel may have written.
+// griddep_launch: allow the next kernel of the stream to be scheduled (it still waits in its
+// own griddep_wait), so its prologue overlaps this kernel's tail.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Per-thread asynchronous global -> shared copies (no register is held while in flight).
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");

@@ -9,6 +9,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch.multiprocessing as mp
 
@@ -34,9 +35,13 @@ def _worker(rank, world, port, out):
     local_ms = 10.0 + 5.0 * rank                     # rank 1 is the slow one
     t_max = bench.max_over_ranks(local_ms, w)        # what rank 0 reports
     seed = bench.shard_seed(1002, r)
+    # the exchange step: packed gradients (theta_R then theta_P, back to back) summed over ranks
+    g = torch.arange(12, dtype=torch.float32).reshape(3, 4) * (rank + 1)
+    bench.dp_allreduce(g, w)
+    summed = g.clone()
     # the same collective steps on every rank, including after the reduction
     dist.barrier()
-    out[rank] = (r, w, t_max, seed)
+    out[rank] = (r, w, t_max, seed, summed.numpy().tolist())
     dist.destroy_process_group()
 
 
@@ -48,6 +53,8 @@ def test_two_ranks_max_over_ranks_and_token_shards():
         res = dict(out)
     assert res[0][:3] == (0, 2, 15.0) and res[1][:3] == (1, 2, 15.0)
     assert res[0][3] != res[1][3]  # each rank draws its own tokens
+    expect = (np.arange(12, dtype=np.float32).reshape(3, 4) * 3).tolist()  # rank 0 (x1) + rank 1 (x2)
+    assert res[0][4] == expect and res[1][4] == expect
     sys.path.insert(0, ROOT)
     import bench
     import poetx_inputs as I
