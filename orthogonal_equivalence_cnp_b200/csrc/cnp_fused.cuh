@@ -68,6 +68,7 @@ struct CnpSegment {
   void* Sb1;
   long ld1;
   int add_identity;
+  CUtensorMap tmS0, tmS1;  // store maps of Sb0 / Sb1 (bf16, 64-column x 32-row boxes)
   // REDUCE: G = sum of split-K partials -> R2, optional bf16 copy Gb, optional f32 copy G32.
   const float* part;  // [splits][nb*b][b]
   int splits;
@@ -101,15 +102,15 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // own G_S tile and the rows of the mirrored one, 128 x (BN + 4) and BN x 132 f32), then the
 // barriers.
 // UNPACK staging: the theta segments of a tile (at most 128 x BN elements in all, plus 11
-// floats of alignment slack per segment), then the assembled S tile (pitch BN + 1) and the G
-// tile (pitch BN + 4).
+// floats of alignment slack per segment), 8 warps x 4 KiB of bf16 boxes for the TMA store of S,
+// the G tile (pitch BN + 4) and the segment offsets.
 template <int BN>
 __host__ __device__ constexpr size_t cnp_stage_bytes() {
   return (((size_t)TC_BM * BN + 11 * (size_t)(TC_BM + BN)) * 4 + 1023) / 1024 * 1024;
 }
 template <int BN>
 __host__ __device__ constexpr size_t cnp_ew_bytes() {
-  return cnp_stage_bytes<BN>() + (size_t)TC_BM * (BN + 1) * 4 + (size_t)TC_BM * (BN + 4) * 4 + 2048;
+  return cnp_stage_bytes<BN>() + 8 * 4096 + (size_t)TC_BM * (BN + 4) * 4 + 4096;
 }
 template <int BN, int STAGES>
 __host__ __device__ constexpr size_t cnp_data_bytes() {
@@ -356,11 +357,12 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
       // segment starting at packed offset e0 sits at e0 % 4 + e of its slot), then the tile is
       // assembled in T0 (pitch BN + 1): rows with lanes along j, columns with lanes along i,
       // both conflict-free.  Packed row i starts at ro(i) + i + 1, ro(i) = i*b - i(i+1)/2 - i - 1.
-      constexpr int RW = TC_BM / (CNP_THREADS / 32), T0P = BN + 1, CPL = BN / 32, RPL = TC_BM / 32;
+      constexpr int RW = TC_BM / (CNP_THREADS / 32);
       float* Sg = reinterpret_cast<float*>(smem);
-      float* T0 = reinterpret_cast<float*>(smem + cnp_stage_bytes<BN>());
-      float* Gt = T0 + TC_BM * T0P;  // G tile (REDUCE), row pitch TS
+      uint8_t* stg = smem + cnp_stage_bytes<BN>() + warp * 4096;  // this warp's bf16 box
+      float* Gt = reinterpret_cast<float*>(smem + cnp_stage_bytes<BN>() + 8 * 4096);  // G tile, pitch TS
       int* seg_off = reinterpret_cast<int*>(Gt + TC_BM * TS);  // [256]: slot start + e0 % 4
+      int* colbase = seg_off + CNP_THREADS + 8;               // [BN]: Sg index of row 0 of column cc
       auto ro = [&](int r) { return r * b - (r * (r + 1)) / 2 - r - 1; };
       auto seg_of = [&](int t, int& e0, int& cnt) {  // segment of thread t's row / column
         e0 = 0; cnt = 0;
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
         int off = x - cap;
         for (int w = 0; w < warp; ++w) off += warp_sum[w];
         seg_off[t] = off + (e0 & 3);
+        if (t >= TC_BM && t < TC_BM + BN) colbase[t - TC_BM] = off + (e0 & 3) - (max(m0, n0 + t - TC_BM + 1) - m0);
         // block z's theta starts 16-byte aligned (P * 4 is a multiple of 16 for b % 8 == 0), so
         // the rounded cover never leaves it
         const int b0 = (e0 * 4) & ~15, b1 = ((e0 + cnt) * 4 + 15) & ~15;
@@ -443,35 +446,17 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
       bool got = mbar_wait(ew_bar, ew_phase, KID_CNP_FUSED, 4);
       ew_phase ^= 1u;
       got = __syncthreads_and(got);
-      // Assemble T0 = S tile.  Rows (warps over rows, lanes along columns): the part above the
-      // diagonal, the diagonal, and zero rows past b.
+      // Each thread builds its tile row (r = 32 quarter + lane) over its half of the columns
+      // straight from the staging: above the diagonal from the row's own segment, below it from
+      // the column segments (lanes read consecutive rows of one segment); S goes to TMEM (R1)
+      // and, as bf16, through a swizzled 32 x 64 box and a TMA store to Sb0 / Sb1.
       const float diag = S.add_identity ? 1.f : 0.f;
-#pragma unroll 2
-      for (int t = 0; t < RW; ++t) {
-        const int r = warp + 8 * t, ii = m0 + r, c0 = max(n0, ii + 1) - n0, so = seg_off[r];
-#pragma unroll
-        for (int q = 0; q < CPL; ++q) {
-          const int cc = lane + 32 * q, jj = n0 + cc;
-          float x = 0.f;
-          if (ii < b && got) x = jj > ii ? Sg[so + cc - c0] : (jj == ii ? diag : 0.f);
-          if (jj >= ii || ii >= b) T0[r * T0P + cc] = x;
-        }
-      }
-      // Columns (threads over columns, lanes along rows): the part below the diagonal.
-#pragma unroll 2
-      for (int t = 0; t < BN / 8; ++t) {
-        const int cc = warp + 8 * t, jj = n0 + cc, r0 = max(m0, jj + 1) - m0, so = seg_off[TC_BM + cc];
-#pragma unroll
-        for (int q = 0; q < RPL; ++q) {
-          const int r = lane + 32 * q, ii = m0 + r;
-          if (ii > jj && ii < b) T0[r * T0P + cc] = got ? -Sg[so + r - r0] : 0.f;
-        }
-      }
-      __syncthreads();
-      // Coalesced bf16 copies of S and G (warps over rows, lanes along columns); then each
-      // thread moves its row into TMEM.
-      if (S.Sb0) tile_store(T0, T0P, S.Sb0, S.ld0, BF16);
-      if (S.Sb1) tile_store(T0, T0P, S.Sb1, S.ld1, BF16);
+      const int r_own = quarter * 32 + lane, i_own = m0 + r_own;
+      const int ld_c = i_own - n0;  // this row's diagonal column
+      const int rowbase = seg_off[r_own] - (max(n0, i_own + 1) - n0);
+      const bool s_out = S.Sb0 != nullptr || S.Sb1 != nullptr;
+      const bool s_tma = HALF % 64 == 0;  // a bf16 box is 64 columns wide
+      const bool rows_ok = m0 + quarter * 32 < b;
       if (D.kind == CNP_REDUCE_UNPACK) {
         if (S.Gb) tile_store(Gt, TS, S.Gb, S.ldg, BF16);
         if (S.G32) tile_store(Gt, TS, S.G32, b, F32);
@@ -480,12 +465,37 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
 #pragma unroll 1
       for (int c = half * HALF; c < (half + 1) * HALF; c += 32) {
         uint32_t w[32];
-        if (!S.no_sreg) {
-          const float* trow = T0 + (quarter * 32 + lane) * T0P + c;
+        float v[32];
+        // One unconditional shared load per element (its address selected; element 0 of the
+        // staging where nothing is read: dead rows and the diagonal), so the 32 loads of a chunk
+        // are independent and pipeline.
+        const bool live = i_own < b && got;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(trow[j]);
+        for (int j = 0; j < 32; ++j) {
+          const int cc = c + j;
+          const bool up = cc > ld_c;
+          const int idx = (!live || cc == ld_c) ? 0 : (up ? rowbase + cc : colbase[cc] + r_own);
+          const float x = Sg[idx];
+          v[j] = !live ? 0.f : (up ? x : (cc == ld_c ? diag : -x));
+          w[j] = __float_as_uint(v[j]);
+        }
+        if (!S.no_sreg) {
           tmem_st_32x32b_x32(treg(CNP_R1, c), w);
           wrote_tmem = true;
+        }
+        if (s_out) {
+          if (s_tma) {
+            uint8_t* box = stg + lane * 128;
+            const int ch0 = ((c - half * HALF) % 64) / 8;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              *reinterpret_cast<uint4*>(box + (((ch0 + u) ^ (lane & 7)) * 16)) =
+                  make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                             pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+          } else if (i_own < b) {
+            if (S.Sb0) store32(S.Sb0, ((long)z * b + i_own) * S.ld0 + n0 + c, BF16, v);
+            if (S.Sb1) store32(S.Sb1, ((long)z * b + i_own) * S.ld1 + n0 + c, BF16, v);
+          }
         }
         if (D.kind == CNP_REDUCE_UNPACK) {
           const float4* grow4 = reinterpret_cast<const float4*>(Gt + (quarter * 32 + lane) * TS + c);
@@ -498,6 +508,19 @@ __global__ void __launch_bounds__(CNP_THREADS, 1) cnp_program_kernel(const __gri
           tmem_st_32x32b_x32(treg(CNP_R2, c), w);
           wrote_tmem = true;
         }
+      }
+      if (s_out && s_tma) {
+        // one lane stores the warp's box (complete before the stage barrier: peers read S next)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && got && rows_ok) {
+          const int x0 = n0 + half * HALF, y0 = z * b + m0 + quarter * 32;
+          if (S.Sb0) tma_store_2d(&S.tmS0, smem_u32(stg), x0, y0);
+          if (S.Sb1) tma_store_2d(&S.tmS1, smem_u32(stg), x0, y0);
+          bulk_commit();
+          bulk_wait<0>();
+        }
+        __syncwarp();
       }
     } else if (D.kind == CNP_PACK) {
       // Own tile of G_S -> Tp (rows, pitch TS) and rows n0.. of G_S restricted to columns m0..

@@ -752,7 +752,7 @@ static_assert(sizeof(CnpProgram) <= 32764, "the CNP program is passed as one ker
 
 template <int BN>
 poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_t st) {
-  constexpr int ST = 4;
+  constexpr int ST = 6;  // ring depth: the long-K product of the adjoint (K = k b) streams in two rounds
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
@@ -783,7 +783,14 @@ poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_
   return last_launch();
 }
 
-poetx_status run_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_t st) {
+poetx_status run_cnp_program(CnpProgram& pr, long nb_total, cudaStream_t st) {
+  // Store maps of the S copies written by the UNPACK stage (64-column x 32-row bf16 boxes).
+  for (int q = 0; q < pr.nseg; ++q) {
+    CnpSegment& S = pr.seg[q];
+    const long rows = (long)S.nb * pr.b;
+    if (S.Sb0 && !make_tmap(&S.tmS0, view(S.Sb0, rows, pr.b, S.ld0), 64, 32)) return POETX_ERR_CUDA;
+    if (S.Sb1 && !make_tmap(&S.tmS1, view(S.Sb1, rows, pr.b, S.ld1), 64, 32)) return POETX_ERR_CUDA;
+  }
   return cnp_bn(pr.b) == 128 ? launch_cnp_program<128>(pr, nb_total, st) : launch_cnp_program<64>(pr, nb_total, st);
 }
 
