@@ -562,9 +562,6 @@ struct WideArgs {
   long ld1;
   void* out2;  // bf16 [M, N] block-factor result, or null (plain GEMM)
   long ld2;
-  // batch z = blockIdx.z (plain GEMM only): A columns, B rows / columns and D columns shift by
-  // z times these (the block-diagonal products: one 256-column block of A, Q and D per z)
-  int a_zcol, b_zrow, b_zcol, d_zcol;
 };
 
 constexpr int TCW_BM = 256, TCW_BN = 256, TCW_STAGES = 3;
@@ -600,7 +597,6 @@ __global__ void __launch_bounds__(128, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * TCW_BM, n0 = blockIdx.x * BN;
   const int zq = blockIdx.x;
-  const int zb = blockIdx.z;  // batch (0 for the W0' GEMM)
   const int nkt = (args.K + TC_BK - 1) / TC_BK;
   const bool fuse = args.out2 != nullptr;
   // Ring stages used after the K loop: Q chunks 0,1 and 2,3, then the D half.
@@ -640,13 +636,12 @@ __global__ void __launch_bounds__(128, 1)
       mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
       const int k0 = i * TC_BK;
       const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
-      tma_load_2d(sa, &tmA, full_bar(s), zb * args.a_zcol + k0, m0);  // box 64 x 256: both halves
+      tma_load_2d(sa, &tmA, full_bar(s), k0, m0);  // box 64 x 256: both halves
       if (!B_MN) {
-        tma_load_2d(sb, &tmB, full_bar(s), zb * args.b_zcol + k0, zb * args.b_zrow + n0);
+        tma_load_2d(sb, &tmB, full_bar(s), k0, n0);
       } else {
 #pragma unroll
-        for (int h = 0; h < BN / 64; ++h)
-          tma_load_2d(sb + h * 8192, &tmB, full_bar(s), zb * args.b_zcol + n0 + 64 * h, zb * args.b_zrow + k0);
+        for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmB, full_bar(s), n0 + 64 * h, k0);
       }
     }
     if (ok && fuse) {
@@ -738,7 +733,7 @@ __global__ void __launch_bounds__(128, 1)
     if (threadIdx.x == 0 && store_d) {
 #pragma unroll
       for (int t = 0; t < 4; ++t)
-        tma_store_2d(&tmD, smem0 + stage * STAGE_BYTES + t * HALF_A, zb * args.d_zcol + n0 + 64 * t, m0 + h * TC_BM);
+        tma_store_2d(&tmD, smem0 + stage * STAGE_BYTES + t * HALF_A, n0 + 64 * t, m0 + h * TC_BM);
       bulk_commit();
     }
   };

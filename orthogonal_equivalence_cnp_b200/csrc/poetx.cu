@@ -419,21 +419,16 @@ poetx_status run_gemm_bd_fused(const GemmDesc& g, const void* Q, long q_rows, bo
 
 // 256 x 256 tiles (gemm_w256_tc) for the W0' GEMM when they still occupy three quarters of the
 // SMs: plain bf16 store of D, optionally followed by the block factor (b = 256).
-// Batched use (the block-diagonal products): batches shift A and B by whole rows / columns and
-// D by columns only, with 64-aligned column offsets.
 bool w256_ok(int dt, const GemmDesc& g) {
   const Epilogue& e = g.epi;
   const bool plain_epi = e.d1 != nullptr && e.d1_dtype == BF16 && e.alpha1 == 1.f && e.beta1 == 0.f && !e.c &&
                          !e.d2 && !e.diag1 && !e.split_stride1;
-  const bool batch_ok = g.batch == 1 || (e.zrow1 == 0 && g.A.zrow == 0 && e.zcol1 % 64 == 0 && g.A.zcol % 64 == 0 &&
-                                         g.B.zcol % 64 == 0 && g.B.zrow % 64 == 0);
-  return dt == BF16 && !g.a_mn && g.N % 256 == 0 && batch_ok && g.splits == 1 && g.K > 0 && plain_epi &&
-         4L * ((g.M + TCW_BM - 1) / TCW_BM) * (g.N / TCW_BN) * g.batch >= 3L * kNumSms;
+  return dt == BF16 && !g.a_mn && g.N % 256 == 0 && g.batch == 1 && g.splits == 1 && g.K > 0 && plain_epi &&
+         4L * ((g.M + TCW_BM - 1) / TCW_BM) * (g.N / TCW_BN) >= 3L * kNumSms;
 }
 
 template <bool BMN, bool QMN>
-poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st,
-                         int cls = POETX_KC_W_GEMM) {
+poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st) {
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
@@ -446,9 +441,8 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   CUtensorMap ta, tb, tq, td;
   if (!make_tmap(&ta, g.A, 64, TCW_BM)) return POETX_ERR_CUDA;
   if (!make_tmap(&tb, g.B, 64, BMN ? 64 : TCW_BN)) return POETX_ERR_CUDA;
-  // Store boxes of D: 64 columns x 128 rows (one half's K chunk); the map spans every batch.
-  if (!make_tmap(&td, view(g.epi.d1, g.M, (long)(g.batch - 1) * g.epi.zcol1 + g.N, g.epi.ld1), 64, TC_BM))
-    return POETX_ERR_CUDA;
+  // Store boxes of D: 64 columns x 128 rows (one half's K chunk).
+  if (!make_tmap(&td, view(g.epi.d1, g.M, g.N, g.epi.ld1), 64, TC_BM)) return POETX_ERR_CUDA;
   if (out2 != nullptr) {
     if (!make_tmap(&tq, view(Q, q_rows, 256, 256), 64, QMN ? 64 : 256)) return POETX_ERR_CUDA;
   } else {
@@ -458,9 +452,8 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.M = g.M; a.N = g.N; a.K = g.K;
   a.d1 = g.epi.d1; a.ld1 = g.epi.ld1;
   a.out2 = out2; a.ld2 = ld2;
-  a.a_zcol = (int)g.A.zcol; a.b_zrow = (int)g.B.zrow; a.b_zcol = (int)g.B.zcol; a.d_zcol = (int)g.epi.zcol1;
-  dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, g.batch);
-  LaunchScope ls(cls, st);
+  dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
+  LaunchScope ls(POETX_KC_W_GEMM, st);
   if (launch_pdl(kern, grid, dim3(128), smem, st, ta, tb, tq, td, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
 }
@@ -483,15 +476,6 @@ poetx_status run_w_gemm(int dt, const GemmDesc& g, const void* Q, long q_rows, b
   return launch_w256<true, true>(g, Q, q_rows, out2, ld2, st);
 }
 
-// A block-diagonal product (batched over blocks): 256 x 256 tiles when b = 256 and they fill
-// the SMs (Q is then read once per 256 tokens instead of once per 128), else the general kernel.
-poetx_status run_bd_gemm(int dt, const GemmDesc& g, cudaStream_t st) {
-  if (!w256_ok(dt, g)) return run_gemm(dt, g, st, POETX_KC_BD_GEMM);
-  POETX_TRY(check_gemm(g, BF16));
-  return g.b_mn ? launch_w256<true, false>(g, nullptr, 0, nullptr, 0, st, POETX_KC_BD_GEMM)
-                : launch_w256<false, false>(g, nullptr, 0, nullptr, 0, st, POETX_KC_BD_GEMM);
-}
-
 // Out[:, blk z] = In[:, blk z] . Q_z^T  (forward block-diagonal application; tokens are rows).
 poetx_status bd_forward(int dt, long n, int d, int b, const void* in, const void* Q, void* out, cudaStream_t st) {
   GemmDesc g;
@@ -499,7 +483,7 @@ poetx_status bd_forward(int dt, long n, int d, int b, const void* in, const void
   g.A = view(in, n, d, d, 0, b);
   g.B = view(Q, d, b, b, b, 0);
   g.epi.d1 = out; g.epi.d1_dtype = dt; g.epi.ld1 = d; g.epi.zcol1 = b;
-  return run_bd_gemm(dt, g, st);
+  return run_gemm(dt, g, st, POETX_KC_BD_GEMM);
 }
 
 // Out[:, blk z] = In[:, blk z] . Q_z  (adjoint of bd_forward w.r.t. its input).
@@ -510,7 +494,7 @@ poetx_status bd_backward(int dt, long n, int d, int b, const void* in, const voi
   g.B = view(Q, d, b, b, b, 0);
   g.b_mn = true;
   g.epi.d1 = out; g.epi.d1_dtype = dt; g.epi.ld1 = d; g.epi.zcol1 = b;
-  return run_bd_gemm(dt, g, st);
+  return run_gemm(dt, g, st, POETX_KC_BD_GEMM);
 }
 
 // Gpart[s][z] = Lhs[:, blk z]^T . Rhs[:, blk z] over split s of the tokens (f32 partials).
