@@ -421,6 +421,32 @@ def run_poetx(args):
     P.poetx_adamw_reset(n_par, layer.m, layer.v)
     torch.cuda.synchronize()
 
+    # Comparator: the same step in the weight-centric order (form W = R W0 P first, then dense
+    # products), captured and timed the same way (L2 flushed between steps, outside the interval).
+    wc_ms = None
+    if args.comparator:
+        layer.wc_step(X, dY)
+        torch.cuda.synchronize()
+        wgraph = None
+        if graph is not None:
+            wgraph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(wgraph):
+                layer.wc_step(X, dY)
+        Kc = min(K, 200)
+        we0 = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
+        we1 = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
+        for i in range(Kc):
+            flush.zero_()
+            we0[i].record(stream)
+            if wgraph is not None:
+                wgraph.replay()
+            else:
+                layer.wc_step(X, dY)
+            we1[i].record(stream)
+        torch.cuda.synchronize()
+        wc_ms = max_over_ranks(sum(we0[i].elapsed_time(we1[i]) for i in range(Kc)), world, dev) / Kc
+        del wgraph
+
     fl = step_flops(s)
     value = world * s.n_tokens * K / (t_ms / 1e3)
     tflops = world * fl["total"] * K / (t_ms / 1e3) / 1e12
@@ -467,6 +493,12 @@ def run_poetx(args):
         "kernel_share": {k: round(v[1] / total_prof_ms, 4) for k, v in prof.items() if v[0]},
         "kernel_ms_per_step": {k: round(v[1] / K, 4) for k, v in prof.items() if v[0]},
         "gpu_launches": int(launches),
+        "comparator": (None if wc_ms is None else
+                       {"weight_centric_ms_per_step": round(wc_ms, 4), "input_centric_ms_per_step": round(t_ms / K, 4),
+                        "input_centric_speedup": round(wc_ms / (t_ms / K), 3),
+                        "what": "same layer step with W = R W0 P formed first (original POET order): "
+                                "T = W0' BD_P, M = BD_R T, W permuted to the original basis, Y = X W^T; "
+                                "dX = dY W, dW = dY^T X, dM, gradients of Q from dM, CNP adjoint"}),
         "optimizer": {"kernel": "adamw_kernel (packed theta_R + theta_P, one launch)", "params": int(n_par),
                       "us_per_launch": round(opt_ms * 1e3, 2),
                       "achieved": round(28 * n_par / (opt_ms / 1e3) / 1e9, 1), "unit": "GB/s",
@@ -551,6 +583,8 @@ def main():
     ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
     ap.add_argument("--workload", choices=sorted(I.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparator", dest="comparator", action="store_false",
+                    help="skip timing the weight-centric comparator")
     ap.add_argument("--no-graph", action="store_true", help="launch every step directly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:

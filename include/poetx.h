@@ -189,6 +189,31 @@ poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, con
                          const int32_t* perm_L_new, const int32_t* perm_R_new, float* theta_R,
                          float* theta_P, void* workspace, size_t ws_bytes, poetx_stream stream);
 
+/* ------------------------------------------------------ weight-centric comparator (not the path)
+ * The original POET order of evaluation, for comparison with the input-centric path above
+ * (replication review, "Summary": POET-X's speed-ups are measured against forming the
+ * transformed weight; agidaily.cc article: the transformed weight W_RP = R.W0.P).  The same
+ * layer arithmetic is done weight-first: T = W0'.BD_P, M = BD_R.T, W = Pi_L^T M Pi_R (the layer
+ * weight in the original basis), Y = X.W^T; backward dX = dY.W, dW = dY^T.X, dM = Pi_L dW Pi_R^T,
+ * dL/dQ_R,i = dM[blk i,:].T[blk i,:]^T, dL/dQ_P,j = (BD_R.W0')[:,blk j]^T.dM[:,blk j], then the
+ * same CNP adjoint as poetx_backward.  Q_R, Q_P come from poetx_cnp.
+ *   wc_saved  dtype, poetx_wc_saved_size(desc) bytes: W [d_out, d_in] then T (256-byte aligned)
+ *             (out of poetx_wc_forward, in to poetx_wc_backward)
+ *   workspace poetx_wc_workspace_size(desc) bytes.
+ * poetx_wc_forward with n_tokens == 0 only forms W and T.  Errors as for poetx_forward. */
+size_t poetx_wc_saved_size(const poetx_desc* desc);
+size_t poetx_wc_workspace_size(const poetx_desc* desc);
+poetx_status poetx_wc_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                              const int32_t* perm_L, const int32_t* perm_R, const void* Q_R,
+                              const void* Q_P, void* Y, void* wc_saved, void* workspace,
+                              size_t ws_bytes, poetx_stream stream);
+poetx_status poetx_wc_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
+                               const void* W0p, const int32_t* perm_L, const int32_t* perm_R,
+                               const void* Q_R, const float* theta_R, const float* theta_P,
+                               const void* wc_saved, void* dX, float* grad_theta_R,
+                               float* grad_theta_P, void* workspace, size_t ws_bytes,
+                               poetx_stream stream);
+
 /* ------------------------------------------------------------------ optimiser (packed theta)
  * AdamW on the packed skew parameters, so that the optimiser state stays at the packed size
  * (agidaily.cc article, compact storage: gradients and optimiser state shrink with the

@@ -18,7 +18,7 @@ __all__ = [
     "poetx_merge", "poetx_status_string", "poetx_device_status", "poetx_test_gemm",
     "poetx_launch_count", "poetx_profile_enable", "poetx_profile_summary", "KERNEL_CLASSES",
     "poetx_cnp_blocks_noalloc", "poetx_cnp_powers_size", "poetx_adamw_cfg", "poetx_adamw_step",
-    "poetx_adamw_reset",
+    "poetx_adamw_reset", "poetx_wc_saved_size", "poetx_wc_workspace_size", "poetx_wc_forward", "poetx_wc_backward",
 ]
 
 POETX_F32, POETX_BF16 = 0, 1
@@ -77,6 +77,10 @@ _SIGNATURES = {
     "poetx_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_adamw_step": (_I, [ctypes.POINTER(poetx_adamw_cfg), _LL, _I, _P, _P, _P, _P, _P]),
     "poetx_adamw_reset": (_I, [_LL, _P, _P, _P]),
+    "poetx_wc_saved_size": (_SZ, [_D]),
+    "poetx_wc_workspace_size": (_SZ, [_D]),
+    "poetx_wc_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_wc_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_status_string": (ctypes.c_char_p, [_I]),
     "poetx_device_status": (_I, [ctypes.POINTER(ctypes.c_int)]),
     "poetx_launch_count": (ctypes.c_ulonglong, []),
@@ -197,6 +201,31 @@ def poetx_adamw_step(cfg, n, t, theta, grad, m, v, stream=None):
 
 def poetx_adamw_reset(n, m, v, stream=None):
     _check(lib().poetx_adamw_reset(n, _ptr(m), _ptr(v), _stream(stream)), "poetx_adamw_reset")
+
+
+def poetx_wc_saved_size(desc) -> int:
+    return lib().poetx_wc_saved_size(ctypes.byref(desc))
+
+
+def poetx_wc_workspace_size(desc) -> int:
+    return lib().poetx_wc_workspace_size(ctypes.byref(desc))
+
+
+def poetx_wc_forward(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, wc_saved, workspace, ws_bytes=None,
+                     stream=None):
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_wc_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0p), _ptr(perm_L), _ptr(perm_R),
+                                  _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(wc_saved), _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "poetx_wc_forward")
+
+
+def poetx_wc_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, theta_R, theta_P, wc_saved, dX, grad_theta_R,
+                      grad_theta_P, workspace, ws_bytes=None, stream=None):
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_wc_backward(ctypes.byref(desc), n_tokens, _ptr(dY), _ptr(X), _ptr(W0p), _ptr(perm_L),
+                                   _ptr(perm_R), _ptr(Q_R), _ptr(theta_R), _ptr(theta_P), _ptr(wc_saved), _ptr(dX),
+                                   _ptr(grad_theta_R), _ptr(grad_theta_P), _ptr(workspace), ws_bytes,
+                                   _stream(stream)), "poetx_wc_backward")
 
 
 def poetx_merge(desc, W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P, workspace,

@@ -1027,6 +1027,33 @@ MergePlan merge_plan(const poetx_desc* d) {
   return m;
 }
 
+// Weight-centric comparator (the original POET order): the transformed weight is formed first.
+//   forward:  T = W0'.BD_P, M = BD_R.T, W = Pi_L^T M Pi_R (original basis), Y = X.W^T
+//   backward: dX = dY.W, dW = dY^T.X, dM = Pi_L dW Pi_R^T, G_R,i = dM[blk i,:].T[blk i,:]^T,
+//             B1 = BD_R.W0', G_P,j = B1[:,blk j]^T.dM[:,blk j], then the CNP adjoint.
+// The caller keeps `wc_saved` = [W | T] (2 d_out d_in elements) from the forward for the backward.
+struct WcPlan {
+  size_t M2, invL, invR, dW, dM, B1, GpR, GpP, cnpR, cnpP, total;
+};
+WcPlan wc_plan(const poetx_desc* d) {
+  const size_t e = esize(d->dtype), w = (size_t)d->d_out * d->d_in * e;
+  const int b = d->b;
+  WcPlan m;
+  Plan p;
+  m.M2 = p.take(w);
+  m.invL = p.take((size_t)d->d_out * 4);
+  m.invR = p.take((size_t)d->d_in * 4);
+  m.dW = p.take(w);
+  m.dM = p.take(w);
+  m.B1 = p.take(w);
+  m.GpR = p.take((size_t)d->d_out * b * 4);
+  m.GpP = p.take((size_t)d->d_in * b * 4);
+  m.cnpR = p.take(cnp_bwd_ws(b, d->k, d->dtype, d->d_out / b));
+  m.cnpP = p.take(cnp_bwd_ws(b, d->k, d->dtype, d->d_in / b));
+  m.total = p.total;
+  return m;
+}
+
 poetx_status check_ptrs(std::initializer_list<const void*> ps) {
   for (const void* p : ps) {
     if (p == nullptr) return POETX_ERR_INVALID_ARG;
@@ -1357,6 +1384,132 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
                             grad_theta_R, ws + w.cnpR, stream));
   return cnp_bwd_generic(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + w.GpP), w.sP,
                          grad_theta_P, ws + w.cnpP, stream);
+}
+
+size_t poetx_wc_saved_size(const poetx_desc* desc) {
+  if (check_desc(desc) != POETX_OK) return 0;
+  return 2 * align256((size_t)desc->d_out * desc->d_in * esize(desc->dtype));
+}
+
+size_t poetx_wc_workspace_size(const poetx_desc* desc) {
+  if (check_desc(desc) != POETX_OK) return 0;
+  return std::max(wc_plan(desc).total, cnp_layer_ws(desc));
+}
+
+poetx_status poetx_wc_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                              const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P, void* Y,
+                              void* wc_saved, void* workspace, size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
+  POETX_TRY(check_ptrs({W0p, perm_L, perm_R, Q_R, Q_P, wc_saved}));
+  const WcPlan m = wc_plan(desc);
+  POETX_TRY(check_ws(workspace, ws_bytes, m.total));
+  char* ws = static_cast<char*>(workspace);
+  const int dt = desc->dtype, b = desc->b, din = desc->d_in, dout = desc->d_out;
+  char* Wf = static_cast<char*>(wc_saved);
+  char* T = Wf + align256((size_t)dout * din * esize(dt));
+  {  // T = W0' . BD_P (column blocks)
+    GemmDesc g;
+    g.M = dout; g.N = b; g.K = b; g.batch = din / b;
+    g.A = view(W0p, dout, din, din, 0, b);
+    g.B = view(Q_P, din, b, b, b, 0); g.b_mn = true;
+    g.epi.d1 = T; g.epi.d1_dtype = dt; g.epi.ld1 = din; g.epi.zcol1 = b;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_MERGE_GEMM));
+  }
+  {  // M = BD_R . T (row blocks)
+    GemmDesc g;
+    g.M = b; g.N = din; g.K = b; g.batch = dout / b;
+    g.A = view(Q_R, dout, b, b, b, 0);
+    g.B = view(T, dout, din, din, b, 0); g.b_mn = true;
+    g.epi.d1 = ws + m.M2; g.epi.d1_dtype = dt; g.epi.ld1 = din; g.epi.zrow1 = b;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_MERGE_GEMM));
+  }
+  // W[r][c] = M[pi_L^-1(r)][pi_R^-1(c)]
+  int32_t* invL = reinterpret_cast<int32_t*>(ws + m.invL);
+  int32_t* invR = reinterpret_cast<int32_t*>(ws + m.invR);
+  {
+    LaunchScope ls(POETX_KC_ELEMENTWISE, stream);
+    perm_inverse_kernel<<<ew_grid(dout), 256, 0, stream>>>(perm_L, dout, invL);
+  }
+  {
+    LaunchScope ls(POETX_KC_ELEMENTWISE, stream);
+    perm_inverse_kernel<<<ew_grid(din), 256, 0, stream>>>(perm_R, din, invR);
+  }
+  POETX_TRY(last_launch());
+  POETX_TRY(permute_cols(dt, ws + m.M2, din, Wf, din, dout, din, invR, invL, false, stream));
+  if (n_tokens == 0) return POETX_OK;
+  POETX_TRY(check_ptrs({X, Y}));
+  GemmDesc g;  // Y = X . W^T
+  g.M = n_tokens; g.N = dout; g.K = din;
+  g.A = view(X, n_tokens, din, din);
+  g.B = view(Wf, dout, din, din);
+  g.epi.d1 = Y; g.epi.d1_dtype = dt; g.epi.ld1 = dout;
+  return run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream);
+}
+
+poetx_status poetx_wc_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X, const void* W0p,
+                               const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const float* theta_R,
+                               const float* theta_P, const void* wc_saved, void* dX, float* grad_theta_R,
+                               float* grad_theta_P, void* workspace, size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_tokens < 1) return POETX_ERR_INVALID_ARG;
+  POETX_TRY(check_ptrs({dY, X, W0p, perm_L, perm_R, Q_R, theta_R, theta_P, wc_saved, dX, grad_theta_R, grad_theta_P}));
+  const WcPlan m = wc_plan(desc);
+  POETX_TRY(check_ws(workspace, ws_bytes, m.total));
+  char* ws = static_cast<char*>(workspace);
+  const int dt = desc->dtype, b = desc->b, din = desc->d_in, dout = desc->d_out;
+  const long n = n_tokens;
+  const char* Wf = static_cast<const char*>(wc_saved);
+  const char* T = Wf + align256((size_t)dout * din * esize(dt));
+  {  // dX = dY . W
+    GemmDesc g;
+    g.M = (int)n; g.N = din; g.K = dout;
+    g.A = view(dY, n, dout, dout);
+    g.B = view(Wf, dout, din, din); g.b_mn = true;
+    g.epi.d1 = dX; g.epi.d1_dtype = dt; g.epi.ld1 = din;
+    POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream));
+  }
+  {  // dW = dY^T . X  (K = tokens)
+    GemmDesc g;
+    g.M = dout; g.N = din; g.K = (int)n;
+    g.A = view(dY, n, dout, dout); g.a_mn = true;
+    g.B = view(X, n, din, din); g.b_mn = true;
+    g.epi.d1 = ws + m.dW; g.epi.d1_dtype = dt; g.epi.ld1 = din;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM));
+  }
+  // dM[i][j] = dW[pi_L(i)][pi_R(j)]
+  POETX_TRY(permute_cols(dt, ws + m.dW, din, ws + m.dM, din, dout, din, perm_R, perm_L, false, stream));
+  {  // G_R,i = dM[blk i, :] . T[blk i, :]^T
+    GemmDesc g;
+    g.M = b; g.N = b; g.K = din; g.batch = dout / b;
+    g.A = view(ws + m.dM, dout, din, din, b, 0);
+    g.B = view(T, dout, din, din, b, 0);
+    g.epi.d1 = ws + m.GpR; g.epi.d1_dtype = F32; g.epi.ld1 = b; g.epi.zrow1 = b;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_GRAD_GEMM));
+  }
+  {  // B1 = BD_R . W0' (row blocks)
+    GemmDesc g;
+    g.M = b; g.N = din; g.K = b; g.batch = dout / b;
+    g.A = view(Q_R, dout, b, b, b, 0);
+    g.B = view(W0p, dout, din, din, b, 0); g.b_mn = true;
+    g.epi.d1 = ws + m.B1; g.epi.d1_dtype = dt; g.epi.ld1 = din; g.epi.zrow1 = b;
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_MERGE_GEMM));
+  }
+  // G_P,j = B1[:, blk j]^T . dM[:, blk j]  (K = d_out rows)
+  POETX_TRY(block_grads(dt, dout, din, b, ws + m.B1, ws + m.dM, reinterpret_cast<float*>(ws + m.GpP), 1, stream));
+  const int nbo = dout / b, nbi = din / b;
+  if (cnp_fused_ok(b, dt)) {
+    CnpSide sides[2];
+    sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + m.GpR);
+    sides[0].splits = 1; sides[0].grad = grad_theta_R; sides[0].ws = ws + m.cnpR;
+    sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + m.GpP);
+    sides[1].splits = 1; sides[1].grad = grad_theta_P; sides[1].ws = ws + m.cnpP;
+    return cnp_bwd_fused(b, desc->k, sides, 2, stream);
+  }
+  POETX_TRY(cnp_bwd_generic(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + m.GpR), 1, grad_theta_R,
+                            ws + m.cnpR, stream));
+  return cnp_bwd_generic(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + m.GpP), 1, grad_theta_P,
+                         ws + m.cnpP, stream);
 }
 
 poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, const void* Q_P,

@@ -10,7 +10,8 @@ import torch
 
 from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_adamw_cfg, poetx_adamw_reset,
                poetx_adamw_step, poetx_backward, poetx_cnp, poetx_cnp_powers_size, poetx_desc, poetx_forward,
-               poetx_merge, poetx_workspace_size)
+               poetx_merge, poetx_wc_backward, poetx_wc_forward, poetx_wc_saved_size, poetx_wc_workspace_size,
+               poetx_workspace_size)
 
 TORCH_DTYPE = {POETX_F32: torch.float32, POETX_BF16: torch.bfloat16}
 
@@ -114,6 +115,19 @@ class PoetxLayer:
                        torch.from_numpy(np.asarray(pR, np.int32)).to(self.device))
             poetx_adamw_reset(self.m.numel(), self.m, self.v)
             self.t = 0
+
+    def wc_step(self, X: torch.Tensor, dY: torch.Tensor):
+        """The same step in the weight-centric order (comparator): CNP, form W = R W0 P, Y = X W^T,
+        dX = dY W, dW = dY^T X and the gradients of theta from dW.  Same outputs as step()."""
+        if getattr(self, "wc_saved", None) is None:
+            self.wc_saved = torch.empty(poetx_wc_saved_size(self.desc), dtype=torch.uint8, device=self.device)
+            self.wc_ws = torch.empty(max(poetx_wc_workspace_size(self.desc), 256), dtype=torch.uint8,
+                                     device=self.device)
+        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, None, self.wc_ws)
+        poetx_wc_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
+                         self.wc_saved, self.wc_ws)
+        poetx_wc_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.theta_R,
+                          self.theta_P, self.wc_saved, self.dX, self.g_R, self.g_P, self.wc_ws)
 
     def merge(self, pi_L_new: torch.Tensor, pi_R_new: torch.Tensor):
         """Folds R and P into W0', absorbs the new permutations and resets theta (Q must be current)."""
