@@ -451,7 +451,12 @@ def run_poetx(args):
     value = world * s.n_tokens * K / (t_ms / 1e3)
     tflops = world * fl["total"] * K / (t_ms / 1e3) / 1e12
     peaks = read_peaks()
-    wcnt, wms = prof["w_gemm"]
+    # Both W0' launches of the step: the forward one (alone on the GPU) and the adjoint one (which
+    # shares the GPU with theta_R's gradient GEMM on the side stream); the roofline uses their
+    # average duration.
+    fcnt, fms = prof["w_gemm"]
+    acnt, ams = prof.get("w_gemm_adj", (0, 0.0))
+    wcnt, wms = fcnt + acnt, fms + ams
     w_avg_ms = wms / max(wcnt, 1)
     achieved = w_gemm_flops(s) / (w_avg_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
@@ -487,7 +492,10 @@ def run_poetx(args):
                                        "(profiles/gemm_w256_fwd_2048x4096x4096_b256_ncu.md)",
                      "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                      "frac_of_sustained": round(achieved / float(peaks["bf16_tflops_sustained"]), 4),
-                     "launch_ms": round(w_avg_ms, 4), "launches": wcnt},
+                     "launch_ms": round(w_avg_ms, 4), "launches": wcnt,
+                     "forward_launch_ms": round(fms / max(fcnt, 1), 4),
+                     "adjoint_launch_ms": round(ams / max(acnt, 1), 4),
+                     "forward_frac": round(w_gemm_flops(s) / (fms / max(fcnt, 1) / 1e3) / 1e12 / peak, 4)},
         "step_roofline": {"t_flop_us": round(fl["total"] / (peak * 1e12) * 1e6, 1),
                           "frac": round((fl["total"] / (peak * 1e12)) / (t_ms / K / 1e3), 4)},
         "kernel_share": {k: round(v[1] / total_prof_ms, 4) for k, v in prof.items() if v[0]},

@@ -256,7 +256,7 @@ poetx_status poetx_device_status(int* detail);
 
 /* Kernel classes of the library's launches. */
 typedef enum {
-  POETX_KC_W_GEMM = 0,       /* Z = V W0'^T and dV = dZ W0' (tensor cores)                 */
+  POETX_KC_W_GEMM = 0,       /* Z = V W0'^T (tensor cores; with BD_R fused for b = 256)     */
   POETX_KC_BD_GEMM = 1,      /* block-diagonal products BD_P, BD_R and their adjoints       */
   POETX_KC_GRAD_GEMM = 2,    /* per-block gradient products G = dY'^T Z, dV^T U (split-K)   */
   POETX_KC_CNP_GEMM = 3,     /* Cayley-Neumann power products (forward and adjoint)         */
@@ -265,7 +265,8 @@ typedef enum {
   POETX_KC_ELEMENTWISE = 6,  /* unpack, pack, split-K reduction, permutation inverse        */
   POETX_KC_TEST_GEMM = 7,    /* poetx_test_gemm                                              */
   POETX_KC_OPTIMIZER = 8,    /* poetx_adamw_step                                             */
-  POETX_KC_COUNT = 9
+  POETX_KC_W_GEMM_ADJ = 9,   /* dV = dZ W0' (with the BD_P adjoint fused for b = 256)        */
+  POETX_KC_COUNT = 10
 } poetx_kernel_class;
 
 /* Number of kernels this library has launched in the process so far. */

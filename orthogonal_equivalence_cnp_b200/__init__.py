@@ -29,7 +29,7 @@ STATUS = {
 }
 
 KERNEL_CLASSES = ["w_gemm", "bd_gemm", "grad_gemm", "cnp_gemm", "merge_gemm", "permute", "elementwise", "test_gemm",
-                  "optimizer"]
+                  "optimizer", "w_gemm_adj"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 

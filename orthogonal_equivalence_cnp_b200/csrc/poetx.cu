@@ -381,7 +381,8 @@ bool bd_fusable(int dt, int b, const GemmDesc& g) {
 }
 
 template <bool BMN, bool QMN>
-poetx_status launch_bd_fused(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st) {
+poetx_status launch_bd_fused(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st,
+                             int cls) {
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
@@ -400,21 +401,21 @@ poetx_status launch_bd_fused(const GemmDesc& g, const void* Q, long q_rows, void
   a.d1 = g.epi.d1; a.ld1 = g.epi.ld1;
   a.out2 = out2; a.ld2 = ld2;
   dim3 grid(g.N / 256, (g.M + TC_BM - 1) / TC_BM, 1);
-  LaunchScope ls(POETX_KC_W_GEMM, st);
+  LaunchScope ls(cls, st);
   if (launch_pdl(kern, grid, dim3(128), smem, st, ta, tb, tq, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
 }
 
 poetx_status run_gemm_bd_fused(const GemmDesc& g, const void* Q, long q_rows, bool q_mn, void* out2, long ld2,
-                               cudaStream_t st) {
+                               cudaStream_t st, int cls) {
   POETX_TRY(check_gemm(g, BF16));
   if (q_rows < g.N || !aligned16(Q) || !aligned16(out2) || ld2 % 8) return POETX_ERR_ALIGNMENT;
   const Epilogue& e = g.epi;
   if (e.d1 && (e.d1_dtype != BF16 || e.alpha1 != 1.f || e.c || e.d2 || e.diag1 || e.split_stride1)) return POETX_ERR_INVALID_ARG;
-  if (!g.b_mn && !q_mn) return launch_bd_fused<false, false>(g, Q, q_rows, out2, ld2, st);
-  if (!g.b_mn && q_mn) return launch_bd_fused<false, true>(g, Q, q_rows, out2, ld2, st);
-  if (g.b_mn && !q_mn) return launch_bd_fused<true, false>(g, Q, q_rows, out2, ld2, st);
-  return launch_bd_fused<true, true>(g, Q, q_rows, out2, ld2, st);
+  if (!g.b_mn && !q_mn) return launch_bd_fused<false, false>(g, Q, q_rows, out2, ld2, st, cls);
+  if (!g.b_mn && q_mn) return launch_bd_fused<false, true>(g, Q, q_rows, out2, ld2, st, cls);
+  if (g.b_mn && !q_mn) return launch_bd_fused<true, false>(g, Q, q_rows, out2, ld2, st, cls);
+  return launch_bd_fused<true, true>(g, Q, q_rows, out2, ld2, st, cls);
 }
 
 // 256 x 256 tiles (gemm_w256_tc) for the W0' GEMM when they still occupy three quarters of the
@@ -428,7 +429,8 @@ bool w256_ok(int dt, const GemmDesc& g) {
 }
 
 template <bool BMN, bool QMN>
-poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st) {
+poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st,
+                         int cls) {
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
@@ -453,27 +455,27 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.d1 = g.epi.d1; a.ld1 = g.epi.ld1;
   a.out2 = out2; a.ld2 = ld2;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
-  LaunchScope ls(POETX_KC_W_GEMM, st);
+  LaunchScope ls(cls, st);
   if (launch_pdl(kern, grid, dim3(128), smem, st, ta, tb, tq, td, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
 }
 
 // The W0' GEMM D = A . B^T -> d1, and (out2 != null, b = 256) out2 = D . Q^T or D . Q.
 poetx_status run_w_gemm(int dt, const GemmDesc& g, const void* Q, long q_rows, bool q_mn, void* out2, long ld2,
-                        cudaStream_t st) {
+                        cudaStream_t st, int cls = POETX_KC_W_GEMM) {
   if (out2 == nullptr) {
-    if (!w256_ok(dt, g)) return run_gemm(dt, g, st, POETX_KC_W_GEMM);
+    if (!w256_ok(dt, g)) return run_gemm(dt, g, st, cls);
     POETX_TRY(check_gemm(g, BF16));
-    return g.b_mn ? launch_w256<true, false>(g, nullptr, 0, nullptr, 0, st)
-                  : launch_w256<false, false>(g, nullptr, 0, nullptr, 0, st);
+    return g.b_mn ? launch_w256<true, false>(g, nullptr, 0, nullptr, 0, st, cls)
+                  : launch_w256<false, false>(g, nullptr, 0, nullptr, 0, st, cls);
   }
-  if (!w256_ok(dt, g)) return run_gemm_bd_fused(g, Q, q_rows, q_mn, out2, ld2, st);
+  if (!w256_ok(dt, g)) return run_gemm_bd_fused(g, Q, q_rows, q_mn, out2, ld2, st, cls);
   POETX_TRY(check_gemm(g, BF16));
   if (q_rows < g.N || !aligned16(Q) || !aligned16(out2) || ld2 % 8) return POETX_ERR_ALIGNMENT;
-  if (!g.b_mn && !q_mn) return launch_w256<false, false>(g, Q, q_rows, out2, ld2, st);
-  if (!g.b_mn && q_mn) return launch_w256<false, true>(g, Q, q_rows, out2, ld2, st);
-  if (g.b_mn && !q_mn) return launch_w256<true, false>(g, Q, q_rows, out2, ld2, st);
-  return launch_w256<true, true>(g, Q, q_rows, out2, ld2, st);
+  if (!g.b_mn && !q_mn) return launch_w256<false, false>(g, Q, q_rows, out2, ld2, st, cls);
+  if (!g.b_mn && q_mn) return launch_w256<false, true>(g, Q, q_rows, out2, ld2, st, cls);
+  if (g.b_mn && !q_mn) return launch_w256<true, false>(g, Q, q_rows, out2, ld2, st, cls);
+  return launch_w256<true, true>(g, Q, q_rows, out2, ld2, st, cls);
 }
 
 // Out[:, blk z] = In[:, blk z] . Q_z^T  (forward block-diagonal application; tokens are rows).
@@ -1361,8 +1363,8 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
   g.B = view(W0p, dout, din, din); g.b_mn = true;
   g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
   const bool fused_du = bd_fusable(dt, b, g);
-  if (fused_du) POETX_TRY(run_w_gemm(dt, g, Q_P, din, true, ws + w.dU, din, stream));
-  else POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream));
+  if (fused_du) POETX_TRY(run_w_gemm(dt, g, Q_P, din, true, ws + w.dU, din, stream, POETX_KC_W_GEMM_ADJ));
+  else POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream, POETX_KC_W_GEMM_ADJ));
   if (!fused_du) POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
   // Input side: dX[:, pi_R] = dU (side stream, after G_R); G_P partials (U saved or recomputed).
   POETX_TRY(stream_edge(stream, side, ss->ev[2]));
@@ -1467,7 +1469,7 @@ poetx_status poetx_wc_backward(const poetx_desc* desc, int n_tokens, const void*
     g.A = view(dY, n, dout, dout);
     g.B = view(Wf, dout, din, din); g.b_mn = true;
     g.epi.d1 = dX; g.epi.d1_dtype = dt; g.epi.ld1 = din;
-    POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream));
+    POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream, POETX_KC_W_GEMM_ADJ));
   }
   {  // dW = dY^T . X  (K = tokens)
     GemmDesc g;
@@ -1475,7 +1477,7 @@ poetx_status poetx_wc_backward(const poetx_desc* desc, int n_tokens, const void*
     g.A = view(dY, n, dout, dout); g.a_mn = true;
     g.B = view(X, n, din, din); g.b_mn = true;
     g.epi.d1 = ws + m.dW; g.epi.d1_dtype = dt; g.epi.ld1 = din;
-    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM));
+    POETX_TRY(run_gemm(dt, g, stream, POETX_KC_W_GEMM_ADJ));
   }
   // dM[i][j] = dW[pi_L(i)][pi_R(j)]
   POETX_TRY(permute_cols(dt, ws + m.dW, din, ws + m.dM, din, dout, din, perm_R, perm_L, false, stream));
