@@ -35,7 +35,7 @@ __all__ = [
     "packed_pairs", "packed_index", "unpack_skew", "pack_skew_grad", "cayley_exact",
     "cayley_neumann", "cnp", "block_diag", "perm_matrix", "absorb", "unabsorb",
     "dense_transforms", "dense_weight", "forward_dense", "backward_dense", "cnp_grad",
-    "forward_chain", "backward_chain", "merge", "adamw_step", "train_schedule",
+    "forward_chain", "backward_chain", "backward_chain_G", "merge", "adamw_step", "train_schedule",
 ]
 
 
@@ -262,6 +262,13 @@ def backward_chain(X, dY, W0p, theta_R, theta_P, pi_L, pi_R, b, k):
     G_P,i = dV_i^T U_i; dU_i = dV_i Q_P,i; dX[:, pi_R] = dU; then the CNP adjoint.
     """
     Q_R, Q_P = cnp(theta_R, b, k), cnp(theta_P, b, k)
+    dX, G_R, G_P = backward_chain_G(X, dY, W0p, Q_R, Q_P, pi_L, pi_R, b)
+    return dX, cnp_grad(theta_R, G_R, b, k), cnp_grad(theta_P, G_P, b, k)
+
+
+def backward_chain_G(X, dY, W0p, Q_R, Q_P, pi_L, pi_R, b):
+    """The activation part of backward_chain: (dX, G_R, G_P) with G = dL/dQ per block, before
+    the CNP adjoint."""
     _, U, _, Z, _ = forward_chain(X, W0p, Q_R, Q_P, pi_L, pi_R)
     dY = np.asarray(dY, np.float64)
     W0p = np.asarray(W0p, np.float64)
@@ -281,7 +288,7 @@ def backward_chain(X, dY, W0p, theta_R, theta_P, pi_L, pi_R, b, k):
         dU[:, blk] = dV[:, blk] @ Q_P[i]
     dX = np.empty_like(dU)
     dX[:, np.asarray(pi_R)] = dU
-    return dX, cnp_grad(theta_R, G_R, b, k), cnp_grad(theta_P, G_P, b, k)
+    return dX, G_R, G_P
 
 
 # ----------------------------------------------------------------------------------------------
