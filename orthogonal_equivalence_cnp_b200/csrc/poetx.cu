@@ -500,10 +500,11 @@ poetx_status bd_backward(int dt, long n, int d, int b, const void* in, const voi
 }
 
 // Gpart[s][z] = Lhs[:, blk z]^T . Rhs[:, blk z] over split s of the tokens (f32 partials).
-// Split-K factor of the block-gradient GEMMs: enough CTAs of 128 x 64 tiles (bf16) to fill the
-// SMs, and no split at all when the tiles alone do (the CNP adjoint then reads one partial).
+// Split-K factor of the block-gradient GEMMs: enough CTAs of 128 x 128 tiles (bf16) to fill the
+// SMs (each operand panel is then fetched by two CTAs instead of four with 128 x 64 tiles), no
+// split when the tiles alone do.
 int grad_splits(int dt, long n, int nb, int b) {
-  const long tiles = dt == BF16 ? (long)nb * ((b + 127) / 128) * ((b + 63) / 64)
+  const long tiles = dt == BF16 ? (long)nb * ((b + 127) / 128) * ((b + 127) / 128)
                                 : (long)nb * ((b + 63) / 64) * ((b + 63) / 64);
   const long kt = dt == BF16 ? (n + 63) / 64 : (n + 15) / 16;
   long s = std::max<long>(1, kNumSms / std::max<long>(1, tiles));
