@@ -36,6 +36,7 @@ __all__ = [
     "cayley_neumann", "cnp", "block_diag", "perm_matrix", "absorb", "unabsorb",
     "dense_transforms", "dense_weight", "forward_dense", "backward_dense", "cnp_grad",
     "forward_chain", "backward_chain", "backward_chain_G", "merge", "adamw_step", "train_schedule",
+    "quantize_rows", "dequantize_rows", "xq_merge",
 ]
 
 
@@ -344,3 +345,39 @@ def train_schedule(n_steps, reset_gap=400):
         if merge_now:
             t = 0
     return out
+
+
+# ----------------------------------------------------------------- POET-XQ: 8-bit resident W0'
+# [RR] "Summary": a quantised variant, POET-XQ, is possible because POET-Xmem never keeps a
+# high-precision weight resident; [RR] "Strengths": it is implemented through POET-Xmem (the
+# recompute means the dequantised W is never stored) and compared with 8-bit Q-GaLore and
+# Q-APOLLO; [AD], the section on how POET-X differs from existing methods: POET-X has a
+# quantised version, POET-XQ.  The pages give no format.  Reading: W0' is held as int8 codes
+# with one scale per row (symmetric, absmax): s_o = max_i |W0'[o, i]| / 127 and
+# q[o, i] = round(W0'[o, i] / s_o) to nearest, ties to even, clipped to [-127, 127]; a row of
+# zeros gets s_o = 0 and q = 0.  The layer is the POET-Xmem layer with W0' = s * q.  Since the
+# codes are integers decided by floating point, the scale and the division are taken in float32
+# (the precision in which the library decides them too).
+def quantize_rows(W0p):
+    """W0' [d_out, d_in] -> (q int8 [d_out, d_in], s float32 [d_out]), per-row symmetric absmax."""
+    W = np.asarray(W0p, np.float32)
+    amax = np.max(np.abs(W), axis=1)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    q = np.zeros(W.shape, np.int8)
+    live = s > 0
+    codes = np.rint(W[live] / s[live, None])  # float32 division, round half to even
+    q[live] = np.clip(codes, -127, 127).astype(np.int8)
+    return q, s
+
+
+def dequantize_rows(q, s):
+    """The POET-XQ weight: W0'[o, i] = s_o * q[o, i] (float64)."""
+    return np.asarray(s, np.float64)[:, None] * np.asarray(q, np.float64)
+
+
+def xq_merge(q, s, theta_R, theta_P, pi_L, pi_R, pi_L_new, pi_R_new, b, k):
+    """Merge of the POET-XQ layer: the POET-X merge of W0' = s * q, then the new W0' quantised
+    again.  Returns (W0'_new before quantisation, q_new, s_new, theta_R_new, theta_P_new)."""
+    Wn, tR, tP = merge(dequantize_rows(q, s), theta_R, theta_P, pi_L, pi_R, pi_L_new, pi_R_new, b, k)
+    qn, sn = quantize_rows(Wn)
+    return Wn, qn, sn, tR, tP

@@ -456,3 +456,105 @@ def test_merge_schedule_resets_every_gap():
     sch = O.train_schedule(1000, reset_gap=400)
     assert [s for s, _, mg in sch if mg] == [400, 800]
     assert [t for s, t, _ in sch if s in (1, 400, 401, 800, 801, 1000)] == [1, 400, 1, 400, 1, 200]
+
+
+# ------------------------------------------------------- POET-XQ weight format (8-bit reading)
+def _xq_pins_pass(mod):
+    """The quantiser pins below, run against a module (the oracle or a planted variant); a variant
+    that raises counts as caught."""
+    try:
+        return _xq_pins(mod)
+    except (IndexError, ValueError, TypeError):
+        return False
+
+
+def _xq_pins(mod):
+    ok = True
+    # Hand example.  Row 0: absmax 127/128, so s = 1/128 exactly (127/128 / 127 is exact in
+    # float32) and each code is w * 128 rounded half to even: 0.5 -> 64, 64.5/128 -> 64,
+    # 65.5/128 -> 66, -127/128 -> -127, 1/256 -> 0, 3/256 -> 2.  Row 1: zeros -> s = 0, q = 0.
+    # Row 2: +-2 are the absmax -> +-127 whatever the rounding of 2/127; 0.25 -> 16 (15.875).
+    W = np.array([[0.5, 64.5 / 128, 65.5 / 128, -127 / 128, 1 / 256, 3 / 256],
+                  [0, 0, 0, 0, 0, 0],
+                  [2.0, -2.0, 0.25, 0, -0.25, 1e-6]], np.float32)
+    q, s = mod.quantize_rows(W)
+    ok &= q.dtype == np.int8 and s.dtype == np.float32
+    ok &= np.array_equal(q, np.array([[64, 64, 66, -127, 0, 2], [0] * 6, [127, -127, 16, 0, -16, 0]]))
+    ok &= s[0] == np.float32(1 / 128) and s[1] == 0 and s[2] == np.float32(np.float32(2.0) / np.float32(127))
+    # On-grid rows come back exactly: W = s0 * K with integer K (|K| <= 127, a +-127 in every
+    # row) and a power-of-two s0 per row.
+    rng = np.random.default_rng(21)
+    K = rng.integers(-127, 128, size=(5, 40))
+    K[np.arange(5), rng.integers(0, 40, 5)] = 127 * rng.choice([-1, 1], 5)
+    s0 = 2.0 ** rng.integers(-12, 3, size=5)
+    q, s = mod.quantize_rows((s0[:, None] * K).astype(np.float32))
+    ok &= np.array_equal(q, K) and np.array_equal(s, s0.astype(np.float32))
+    # Random rows of very different size: error at most half a step (plus float32 rounding of
+    # w / s), every row reaches +-127 at its absmax, odd symmetry, power-of-two scale invariance.
+    W = (rng.standard_normal((7, 300)) * (10.0 ** rng.integers(-4, 2, size=7))[:, None]).astype(np.float32)
+    q, s = mod.quantize_rows(W)
+    err = np.abs(W.astype(np.float64) - s.astype(np.float64)[:, None] * q)
+    ok &= bool(np.all(err <= s.astype(np.float64)[:, None] * (0.5 + 1e-5)))
+    ok &= bool(np.all(np.abs(q).max(axis=1) == 127))
+    ok &= bool(np.all(q[np.arange(7), np.abs(W).argmax(axis=1)] == 127 * np.sign(W[np.arange(7), np.abs(W).argmax(axis=1)])))
+    qn, sn = mod.quantize_rows(-W)
+    ok &= np.array_equal(qn, -q) and np.array_equal(sn, s)
+    q8, s8 = mod.quantize_rows(W * np.float32(8.0))
+    ok &= np.array_equal(q8, q) and np.array_equal(s8, s * np.float32(8.0))
+    return bool(ok)
+
+
+def test_quantize_rows_pins():
+    assert _xq_pins_pass(O)
+
+
+def test_dequantize_rows_is_scale_times_code():
+    q = np.array([[1, -127, 0], [5, 6, 7]], np.int8)
+    s = np.array([0.5, 0.25], np.float32)
+    assert np.array_equal(O.dequantize_rows(q, s), np.array([[0.5, -63.5, 0.0], [1.25, 1.5, 1.75]]))
+
+
+def test_xq_merge_is_merge_then_requantise_and_fixed_at_zero_theta():
+    rng = np.random.default_rng(82)
+    b = 4
+    L = _rand_layer(rng, 16, 12, b, 3)
+    q, s = O.quantize_rows(O.absorb(L["W0"], L["pi_L"], L["pi_R"]))
+    # Zero theta and the same permutations: the merged weight is the dequantised one and
+    # quantising it again gives back the same codes and scales.
+    z, zP = np.zeros_like(L["theta_R"]), np.zeros_like(L["theta_P"])
+    Wn, qn, sn, _, _ = O.xq_merge(q, s, z, zP, L["pi_L"], L["pi_R"], L["pi_L"], L["pi_R"], b, 3)
+    assert np.abs(Wn - O.dequantize_rows(q, s)).max() <= 1e-15
+    assert np.array_equal(qn, q) and np.array_equal(sn, s)
+    # General theta: the layer function of the merged (unquantised) weight is that of the
+    # dequantised layer before the merge; the new codes are within half a step of it.
+    pL2, pR2 = rng.permutation(12), rng.permutation(16)
+    Wn, qn, sn, tR, tP = O.xq_merge(q, s, L["theta_R"], L["theta_P"], L["pi_L"], L["pi_R"], pL2, pR2, b, 3)
+    assert np.all(tR == 0) and np.all(tP == 0)
+    Wdq = O.dequantize_rows(q, s)
+    Y_before = O.forward_chain(L["X"], Wdq, O.cnp(L["theta_R"], b, 3), O.cnp(L["theta_P"], b, 3), L["pi_L"], L["pi_R"])[0]
+    Y_after = O.forward_chain(L["X"], Wn, O.cnp(tR, b, 3), O.cnp(tP, b, 3), pL2, pR2)[0]
+    assert _rel(Y_after, Y_before) <= 1e-12
+    assert np.all(np.abs(np.float32(Wn) - O.dequantize_rows(qn, sn)) <= sn[:, None] * (0.5 + 1e-5) + 1e-7 * np.abs(Wn))
+
+
+def test_quantize_planted_mistakes_are_caught():
+    import types
+    src_path = os.path.join(os.path.dirname(O.__file__), "poetx_ref.py")
+    with open(src_path) as f:
+        src = f.read()
+
+    def variant(old, new):
+        assert old in src, old
+        m = types.ModuleType("oracle_variant")
+        exec(compile(src.replace(old, new, 1), "oracle_variant", "exec"), m.__dict__)
+        return m
+
+    mistakes = [
+        ("codes = np.rint(W[live] / s[live, None])", "codes = np.floor(W[live] / s[live, None])"),   # truncation
+        ("codes = np.rint(W[live] / s[live, None])", "codes = np.round(W[live] / s[live, None] + 0.5 * (W[live] > 0))"),  # ties away
+        ("amax = np.max(np.abs(W), axis=1)", "amax = np.max(np.abs(W))"),                          # one scale per tensor
+        ("s = (amax / np.float32(127.0))", "s = (amax / np.float32(128.0))"),                      # 128 levels
+        ("np.clip(codes, -127, 127)", "np.clip(codes, -128, 126)"),                                # asymmetric clip
+    ]
+    for old, new in mistakes:
+        assert not _xq_pins_pass(variant(old, new)), new
