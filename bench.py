@@ -202,6 +202,72 @@ def oracle_step(inp: I.LayerInputs, W0p, n_tok: int):
     O.backward_chain(X, dY, W0p, inp.theta_R, inp.theta_P, inp.pi_L, inp.pi_R, s.b, s.k)
 
 
+def measure_xq(s, src, X, dY, flush, stream, world, dev, use_graph, Kx):
+    """POET-XQ beside POET-Xmem on the same layer state: one mem-mode layer with the bf16 W0' and
+    one with W0' quantised to int8 codes and per-row scales (the W0' GEMMs dequantise in shared
+    memory).  Each step is captured and timed like the headline step (L2 flushed between steps,
+    outside the intervals), then replayed once more with the library's per-launch events to get
+    the W0' GEMM launch times."""
+    import torch
+
+    import orthogonal_equivalence_cnp_b200 as P
+    from orthogonal_equivalence_cnp_b200.layer import PoetxLayer, make_desc
+    res = {}
+    for name in ("mem_bf16", "xq"):
+        L = PoetxLayer(make_desc(s.d_in, s.d_out, s.b, s.k, "bf16", "mem"), s.n_tokens, device=dev)
+        L.W0p.copy_(src.W0p)
+        L.theta.copy_(src.theta)
+        L.perm_L.copy_(src.perm_L)
+        L.perm_R.copy_(src.perm_R)
+        if name == "xq":
+            L.quantize()
+        for _ in range(3):
+            L.step(X, dY)
+        torch.cuda.synchronize()
+        g = None
+        if use_graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                L.step(X, dY)
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(Kx)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(Kx)]
+        for i in range(Kx):
+            flush.zero_()
+            e0[i].record(stream)
+            if g is not None:
+                g.replay()
+            else:
+                L.step(X, dY)
+            e1[i].record(stream)
+        torch.cuda.synchronize()
+        res[f"{name}_ms_per_step"] = round(max_over_ranks(sum(e0[i].elapsed_time(e1[i]) for i in range(Kx)),
+                                                          world, dev) / Kx, 4)
+        prof = {}
+        for i in range(min(Kx, 50)):
+            flush.zero_()
+            P.poetx_profile_enable(True)
+            L.step(X, dY)
+            P.poetx_profile_enable(False)
+            torch.cuda.synchronize()
+            for k, (n, ms) in P.poetx_profile_summary().items():
+                c = prof.get(k, (0, 0.0))
+                prof[k] = (c[0] + n, c[1] + ms)
+        for cls, tag in (("w_gemm", "w_gemm_launch_ms"), ("w_gemm_adj", "w_gemm_adj_launch_ms")):
+            n, ms = prof.get(cls, (0, 0.0))
+            res[f"{name}_{tag}"] = round(ms / max(n, 1), 4)
+        st, det = P.poetx_device_status()
+        if st != 0:
+            raise RuntimeError(f"device-side timeout in the POET-XQ measurement ({det:#x})")
+        del g, L
+    res["w0p_bytes_bf16"] = 2 * s.d_out * s.d_in
+    res["w0p_bytes_xq"] = s.d_out * s.d_in + 4 * s.d_out
+    res["xq_over_mem_bf16_time"] = round(res["xq_ms_per_step"] / res["mem_bf16_ms_per_step"], 3)
+    res["what"] = ("POET-Xmem step (CNP, forward, backward with recompute) with W0' in bf16 vs. int8 codes + "
+                   "per-row fp32 scales dequantised inside the W0' GEMMs (three W0' launches per step: forward, "
+                   "recompute, adjoint)")
+    return res
+
+
 def cpu_baseline(inp: I.LayerInputs, budget_s: float = 20.0) -> dict:
     import oracle as O
     W0p = O.absorb(inp.W0, inp.pi_L, inp.pi_R)
@@ -449,6 +515,10 @@ def run_poetx(args):
         wc_ms = max_over_ranks(sum(we0[i].elapsed_time(we1[i]) for i in range(Kc)), world, dev) / Kc
         del wgraph
 
+    xq = None
+    if args.xq and s.dtype == "bf16" and s.d_in % 256 == 0 and s.d_out % 256 == 0:
+        xq = measure_xq(s, layer, X, dY, flush, stream, world, dev, graph is not None, min(K, 200))
+
     fl = step_flops(s)
     value = world * s.n_tokens * K / (t_ms / 1e3)
     tflops = world * fl["total"] * K / (t_ms / 1e3) / 1e12
@@ -509,6 +579,7 @@ def run_poetx(args):
                         "what": "same layer step with W = R W0 P formed first (original POET order): "
                                 "T = W0' BD_P, M = BD_R T, W permuted to the original basis, Y = X W^T; "
                                 "dX = dY W, dW = dY^T X, dM, gradients of Q from dM, CNP adjoint"}),
+        "xq": xq,
         "optimizer": {"kernel": "adamw_kernel (packed theta_R + theta_P, one launch)", "params": int(n_par),
                       "us_per_launch": round(opt_ms * 1e3, 2),
                       "achieved": round(28 * n_par / (opt_ms / 1e3) / 1e9, 1), "unit": "GB/s",
@@ -614,6 +685,8 @@ def main():
     ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
     ap.add_argument("--workload", choices=sorted(I.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-xq", dest="xq", action="store_false",
+                    help="skip timing the POET-XQ (int8 W0') mem-mode step beside the bf16 mem-mode step")
     ap.add_argument("--no-comparator", dest="comparator", action="store_false",
                     help="skip timing the weight-centric comparator")
     ap.add_argument("--no-graph", action="store_true", help="launch every step directly instead of replaying a CUDA graph")

@@ -189,6 +189,47 @@ poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, con
                          const int32_t* perm_L_new, const int32_t* perm_R_new, float* theta_R,
                          float* theta_P, void* workspace, size_t ws_bytes, poetx_stream stream);
 
+/* ------------------------------------------------------------------------------- POET-XQ
+ * The quantised variant (replication review, "Summary": POET-XQ is possible because POET-Xmem
+ * never keeps a high-precision weight resident; "Strengths": it runs through POET-Xmem, whose
+ * recompute means the dequantised W is never stored, and it is set against 8-bit baselines;
+ * agidaily.cc article, the section on how POET-X differs from existing methods: POET-X has a
+ * quantised version).  The pages give no format; this library's reading is 8-bit symmetric
+ * with one scale per row of W0':
+ *   s_o = max_i |W0'[o, i]| / 127,  q[o, i] = round(W0'[o, i] / s_o) (nearest, ties to even,
+ *   clipped to [-127, 127]; a zero row has s_o = 0, q = 0), both in float32 with IEEE division;
+ *   the layer uses W0'[o, i] = s_o * q[o, i].
+ *   W0q int8 [d_out, d_in], W0s float32 [d_out] (caller-owned device memory, 16-byte aligned).
+ * Only POETX_MEM mode and POETX_BF16 (INVALID_ARG otherwise), d_in and d_out multiples of 256
+ * (UNSUPPORTED_SHAPE otherwise).  The W0' GEMMs of forward and backward read the codes and
+ * dequantise each tile in shared memory; no bf16 W0' exists at any time.  Workspace:
+ * poetx_workspace_size(desc, n_tokens) covers every call below.  Other arguments and errors
+ * as for the bf16 calls above (poetx_xq_backward: no `saved`, no `powers`).
+ *
+ * poetx_xq_quantize:   W0p bf16 [d_out, d_in] (in) -> W0q, W0s (out).
+ * poetx_xq_dequantize: W0q, W0s (in) -> W0p bf16 (out) = bf16(s_o * q) (for inspection).
+ * poetx_xq_merge:      the merge of poetx_merge on W0' = s * q, then the new W0' quantised
+ *                      again into W0q, W0s (in/out); the bf16 weight lives only in the workspace
+ *                      during the call; theta_R, theta_P zeroed. */
+poetx_status poetx_xq_quantize(const poetx_desc* desc, const void* W0p, int8_t* W0q, float* W0s,
+                               poetx_stream stream);
+poetx_status poetx_xq_dequantize(const poetx_desc* desc, const int8_t* W0q, const float* W0s,
+                                 void* W0p, poetx_stream stream);
+poetx_status poetx_xq_forward(const poetx_desc* desc, int n_tokens, const void* X,
+                              const int8_t* W0q, const float* W0s, const int32_t* perm_L,
+                              const int32_t* perm_R, const void* Q_R, const void* Q_P, void* Y,
+                              void* workspace, size_t ws_bytes, poetx_stream stream);
+poetx_status poetx_xq_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
+                               const int8_t* W0q, const float* W0s, const int32_t* perm_L,
+                               const int32_t* perm_R, const void* Q_R, const void* Q_P,
+                               const float* theta_R, const float* theta_P, void* dX,
+                               float* grad_theta_R, float* grad_theta_P, void* workspace,
+                               size_t ws_bytes, poetx_stream stream);
+poetx_status poetx_xq_merge(const poetx_desc* desc, int8_t* W0q, float* W0s, const void* Q_R,
+                            const void* Q_P, const int32_t* perm_L_old, const int32_t* perm_R_old,
+                            const int32_t* perm_L_new, const int32_t* perm_R_new, float* theta_R,
+                            float* theta_P, void* workspace, size_t ws_bytes, poetx_stream stream);
+
 /* ------------------------------------------------------ weight-centric comparator (not the path)
  * The original POET order of evaluation, for comparison with the input-centric path above
  * (replication review, "Summary": POET-X's speed-ups are measured against forming the

@@ -19,6 +19,7 @@ __all__ = [
     "poetx_launch_count", "poetx_profile_enable", "poetx_profile_summary", "KERNEL_CLASSES",
     "poetx_cnp_blocks_noalloc", "poetx_cnp_powers_size", "poetx_adamw_cfg", "poetx_adamw_step",
     "poetx_adamw_reset", "poetx_wc_saved_size", "poetx_wc_workspace_size", "poetx_wc_forward", "poetx_wc_backward",
+    "poetx_xq_quantize", "poetx_xq_dequantize", "poetx_xq_forward", "poetx_xq_backward", "poetx_xq_merge",
 ]
 
 POETX_F32, POETX_BF16 = 0, 1
@@ -81,6 +82,11 @@ _SIGNATURES = {
     "poetx_wc_workspace_size": (_SZ, [_D]),
     "poetx_wc_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_wc_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_xq_quantize": (_I, [_D, _P, _P, _P, _P]),
+    "poetx_xq_dequantize": (_I, [_D, _P, _P, _P, _P]),
+    "poetx_xq_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_xq_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_xq_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_status_string": (ctypes.c_char_p, [_I]),
     "poetx_device_status": (_I, [ctypes.POINTER(ctypes.c_int)]),
     "poetx_launch_count": (ctypes.c_ulonglong, []),
@@ -234,6 +240,41 @@ def poetx_merge(desc, W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_
     _check(lib().poetx_merge(ctypes.byref(desc), _ptr(W0p), _ptr(Q_R), _ptr(Q_P), _ptr(perm_L_old),
                              _ptr(perm_R_old), _ptr(perm_L_new), _ptr(perm_R_new), _ptr(theta_R), _ptr(theta_P),
                              _ptr(workspace), ws_bytes, _stream(stream)), "poetx_merge")
+
+
+def poetx_xq_quantize(desc, W0p, W0q, W0s, stream=None):
+    _check(lib().poetx_xq_quantize(ctypes.byref(desc), _ptr(W0p), _ptr(W0q), _ptr(W0s), _stream(stream)),
+           "poetx_xq_quantize")
+
+
+def poetx_xq_dequantize(desc, W0q, W0s, W0p, stream=None):
+    _check(lib().poetx_xq_dequantize(ctypes.byref(desc), _ptr(W0q), _ptr(W0s), _ptr(W0p), _stream(stream)),
+           "poetx_xq_dequantize")
+
+
+def poetx_xq_forward(desc, n_tokens, X, W0q, W0s, perm_L, perm_R, Q_R, Q_P, Y, workspace, ws_bytes=None,
+                     stream=None):
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_xq_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0q), _ptr(W0s), _ptr(perm_L),
+                                  _ptr(perm_R), _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "poetx_xq_forward")
+
+
+def poetx_xq_backward(desc, n_tokens, dY, X, W0q, W0s, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, dX,
+                      grad_theta_R, grad_theta_P, workspace, ws_bytes=None, stream=None):
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_xq_backward(ctypes.byref(desc), n_tokens, _ptr(dY), _ptr(X), _ptr(W0q), _ptr(W0s),
+                                   _ptr(perm_L), _ptr(perm_R), _ptr(Q_R), _ptr(Q_P), _ptr(theta_R), _ptr(theta_P),
+                                   _ptr(dX), _ptr(grad_theta_R), _ptr(grad_theta_P), _ptr(workspace), ws_bytes,
+                                   _stream(stream)), "poetx_xq_backward")
+
+
+def poetx_xq_merge(desc, W0q, W0s, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P,
+                   workspace, ws_bytes=None, stream=None):
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_xq_merge(ctypes.byref(desc), _ptr(W0q), _ptr(W0s), _ptr(Q_R), _ptr(Q_P), _ptr(perm_L_old),
+                                _ptr(perm_R_old), _ptr(perm_L_new), _ptr(perm_R_new), _ptr(theta_R),
+                                _ptr(theta_P), _ptr(workspace), ws_bytes, _stream(stream)), "poetx_xq_merge")
 
 
 def poetx_device_status():

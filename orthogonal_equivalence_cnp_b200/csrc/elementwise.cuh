@@ -429,4 +429,58 @@ __global__ void perm_compose_kernel(const int32_t* __restrict__ inv_old, const i
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) sigma[i] = inv_old[pnew[i]];
 }
 
+// ------------------------------------------------------------ POET-XQ weight format
+// Per row o of a bf16 W0' [rows, cols] (cols % 8 == 0): s_o = max_i |w| / 127 and
+// q[o, i] = round(w / s_o) to nearest, ties to even, clipped to [-127, 127]; a zero row gets
+// s_o = 0 and q = 0.  Both decisions are taken in float32 with IEEE division, so the codes are
+// a deterministic function of the bf16 input.  One warp per row: the first pass finds the
+// absmax, the second (from L2) writes 8 codes per 16-byte load.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* __restrict__ W, long ld, long rows,
+                                                            int cols, int8_t* __restrict__ q, long ldq,
+                                                            float* __restrict__ scale) {
+  sm100::griddep_wait();
+  const int lane = threadIdx.x & 31, chunks = cols / 8;
+  for (long r = (long)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += (long)gridDim.x * 8) {
+    const uint4* src = reinterpret_cast<const uint4*>(W + r * ld);
+    float amax = 0.f;
+    for (int c = lane; c < chunks; c += 32) {
+      const uint4 u = src[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[t] << 16)), fabsf(__uint_as_float(w[t] & 0xFFFF0000u))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = __fdiv_rn(amax, 127.f);
+    if (lane == 0) scale[r] = s;
+    uint2* dst = reinterpret_cast<uint2*>(q + r * ldq);
+    for (int c = lane; c < chunks; c += 32) {
+      const uint4 u = src[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float v = __uint_as_float(e & 1 ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+        const int code = s > 0.f ? min(127, max(-127, __float2int_rn(__fdiv_rn(v, s)))) : 0;
+        packed[e >> 2] |= (uint32_t)(code & 0xff) << (8 * (e & 3));
+      }
+      dst[c] = make_uint2(packed[0], packed[1]);
+    }
+  }
+}
+
+// W0'[o, i] = bf16(s_o * q[o, i]) for [rows, cols] (cols % 8 == 0), eight codes per thread step.
+__global__ void __launch_bounds__(256) dequantize_rows_kernel(const int8_t* __restrict__ q, long ldq,
+                                                              const float* __restrict__ scale, long rows, int cols,
+                                                              uint16_t* __restrict__ W, long ld) {
+  sm100::griddep_wait();
+  const long chunks = cols / 8, total = rows * chunks;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (long)gridDim.x * blockDim.x) {
+    const long r = idx / chunks, c = idx - r * chunks;
+    const uint2 w = *reinterpret_cast<const uint2*>(q + r * ldq + c * 8);
+    *reinterpret_cast<uint4*>(W + r * ld + c * 8) = dequant8_bf16(w, scale[r]);
+  }
+}
+
 }  // namespace poetx

@@ -51,6 +51,7 @@ struct GemmDesc {
   Operand A, B;
   bool a_mn = false, b_mn = false;
   Epilogue epi;
+  const float* b_scale = nullptr;  // set: B is int8 codes, B row r scaled by b_scale[r] (W0' GEMM only)
 };
 
 // Kernel ids recorded in the device error word.
@@ -556,21 +557,30 @@ __global__ void __launch_bounds__(128, 1)
 // MN-major: D . Q, adjoint of BD_P), reusing the half's own TMEM columns once drained.  Q's
 // four 64-wide K chunks follow the K loop through the ring (two per stage); the D half uses the
 // third stage.  All waits bounded; every thread reaches every barrier.
+//
+// Q8 (POET-XQ, the replication review of POET-X, "Summary" and "Strengths": the quantised
+// variant works through POET-Xmem, so no dequantised weight is ever stored): B is int8 codes
+// with one fp32 scale per row of the B array (bscale).  TMA brings each k step's 16 KiB of codes
+// into one of two staging slots; four more warps (threads 128..255) turn them into bf16
+// scale * code, written straight into the stage's swizzled B tile, and signal the MMA issuer.
 struct WideArgs {
   int M, N, K;
   void* d1;    // bf16 [M, N] store of D (may be null when out2 is set)
   long ld1;
   void* out2;  // bf16 [M, N] block-factor result, or null (plain GEMM)
   long ld2;
+  const float* bscale;  // Q8 only: scale of each row of the int8 B array
 };
 
 constexpr int TCW_BM = 256, TCW_BN = 256, TCW_STAGES = 3;
+constexpr uint32_t TCW_Q8_TILE = 256 * TC_BK;  // int8 codes of one k step's B tile
+template <bool Q8 = false>
 __host__ __device__ constexpr size_t tcw_smem_bytes() {
-  return (size_t)TCW_STAGES * (TCW_BM * TC_BK * 2 + TCW_BN * TC_BK * 2) + 1024 + 256;
+  return (size_t)TCW_STAGES * (TCW_BM * TC_BK * 2 + TCW_BN * TC_BK * 2) + (Q8 ? 2 * TCW_Q8_TILE : 0) + 1024 + 256;
 }
 
-template <bool B_MN, bool Q_MN>
-__global__ void __launch_bounds__(128, 1)
+template <bool B_MN, bool Q_MN, bool Q8 = false>
+__global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
     gemm_w256_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmD,
                  const WideArgs args) {
@@ -585,7 +595,8 @@ __global__ void __launch_bounds__(128, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  constexpr uint32_t STG_OFF = STAGES * STAGE_BYTES;  // Q8: two int8 staging slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STG_OFF + (Q8 ? 2 * TCW_Q8_TILE : 0));
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
   const uint32_t smem0 = smem_u32(smem);
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -593,6 +604,9 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
   const uint32_t q_full = smem_u32(bars + 2 * STAGES + 1);
   const uint32_t acc2_bar = smem_u32(bars + 2 * STAGES + 2);
+  // Q8: B tile of stage s converted (one arrival per converter warp); staging slot j free again.
+  auto conv_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + 4 + s); };
+  auto sfree_bar = [&](int j) { return smem_u32(bars + 3 * STAGES + 4 + j); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * TCW_BM, n0 = blockIdx.x * BN;
@@ -610,6 +624,10 @@ __global__ void __launch_bounds__(128, 1)
     mbar_init(accum_bar, 1);
     mbar_init(q_full, 1);
     mbar_init(acc2_bar, 1);
+    if (Q8) {
+      for (int s = 0; s < STAGES; ++s) mbar_init(conv_bar(s), 4);
+      for (int j = 0; j < 2; ++j) mbar_init(sfree_bar(j), 4);
+    }
     fence_mbar_init();
     fence_proxy_async_smem();
     prefetch_tmap(&tmA);
@@ -633,9 +651,20 @@ __global__ void __launch_bounds__(128, 1)
       const int s = i % STAGES;
       const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
       if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 11)) { ok = false; break; }
-      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
       const int k0 = i * TC_BK;
       const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+      if (Q8) {
+        // Codes of step i into staging slot i % 2, once the converters are done with step i - 2.
+        const int j = i & 1;
+        if (!mbar_wait(sfree_bar(j), ((uint32_t)(i >> 1) & 1u) ^ 1u, KID_GEMM_TC, 17)) { ok = false; break; }
+        mbar_arrive_expect_tx(full_bar(s), A_BYTES + TCW_Q8_TILE);
+        tma_load_2d(sa, &tmA, full_bar(s), k0, m0);
+        const uint32_t stg = smem0 + STG_OFF + j * TCW_Q8_TILE;
+        if (!B_MN) tma_load_2d(stg, &tmB, full_bar(s), k0, n0);  // box 64 (k) x 256 (n) codes
+        else tma_load_2d(stg, &tmB, full_bar(s), n0, k0);        // box 256 (n) x 64 (k) codes
+        continue;
+      }
+      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
       tma_load_2d(sa, &tmA, full_bar(s), k0, m0);  // box 64 x 256: both halves
       if (!B_MN) {
         tma_load_2d(sb, &tmB, full_bar(s), k0, n0);
@@ -671,6 +700,7 @@ __global__ void __launch_bounds__(128, 1)
       const int s = i % STAGES;
       const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
       if (!mbar_wait(full_bar(s), ph, KID_GEMM_TC, 13)) break;
+      if (Q8 && !mbar_wait(conv_bar(s), ph, KID_GEMM_TC, 19)) break;
       tc_fence_after();
       const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
 #pragma unroll
@@ -684,6 +714,53 @@ __global__ void __launch_bounds__(128, 1)
       mma_commit(empty_bar(s));
     }
     mma_commit(accum_bar);
+  } else if (Q8 && warp >= 4) {
+    // ---------------- converters: codes -> bf16 scale * code in the stage's swizzled B tile.
+    // Thread t converts chunks c = 128 j + t (j < 16) of 8 codes each.  K-major B (rows n, 64
+    // codes each): chunk c is row c / 8, 16-byte chunk c % 8.  MN-major B (rows k, 256 codes
+    // each): chunk c is row k = c / 32, columns 8 (c % 32) .. +7, i.e. 64-column sub-tile
+    // (c % 32) / 8, chunk c % 8.  Either way the scale belongs to the code's row of B.
+    const int t = threadIdx.x - 128;
+    float sc[16], scn[16];
+    auto load_scales = [&](int i, float (&dst)[16]) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int row = B_MN ? i * TC_BK + j * 4 + (t >> 5) : n0 + j * 16 + (t >> 3);
+        dst[j] = row < (B_MN ? args.K : args.N) ? __ldg(args.bscale + row) : 0.f;
+      }
+    };
+    load_scales(0, scn);
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) sc[j] = scn[j];
+      if (B_MN && i + 1 < nkt) load_scales(i + 1, scn);  // K-major: the same rows every step
+      if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, KID_GEMM_TC, 18))) break;  // warp-uniform exit
+      const uint8_t* stg = smem + STG_OFF + (i & 1) * TCW_Q8_TILE;
+      uint8_t* tile = smem + s * STAGE_BYTES + A_BYTES;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int c = j * 128 + t;
+        int src, dst;
+        if (!B_MN) {
+          const int row = c >> 3, ch = c & 7;
+          src = row * 64 + ch * 8;
+          dst = row * 128 + ((ch ^ (row & 7)) << 4);
+        } else {
+          const int row = c >> 5, nc = c & 31;
+          src = row * 256 + nc * 8;
+          dst = (nc >> 3) * 8192 + row * 128 + (((nc & 7) ^ (row & 7)) << 4);
+        }
+        *reinterpret_cast<uint4*>(tile + dst) = dequant8_bf16(*reinterpret_cast<const uint2*>(stg + src), sc[j]);
+      }
+      fence_proxy_async_smem();  // the tensor core reads what the threads wrote
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(conv_bar(s));
+        mbar_arrive(sfree_bar(i & 1));
+      }
+    }
   }
   __syncwarp();
 
@@ -693,6 +770,7 @@ __global__ void __launch_bounds__(128, 1)
   griddep_launch();
   const int r = warp * 32 + lane;  // TMEM lane = row within a half
   const uint32_t tl = tmem_d + ((uint32_t)(warp * 32) << 16);
+  const bool epi_warp = !Q8 || warp < 4;  // the four warps that own the TMEM lanes drain them
 
   // Drains 256 columns of TMEM at column offset col0 (row m of the output): bf16 to global
   // `dst` (if set) and, if stage >= 0, into that ring stage as four swizzled K-major 128 x 64
@@ -738,7 +816,7 @@ __global__ void __launch_bounds__(128, 1)
     }
   };
   if (!fuse) {
-    if (ok) {
+    if (ok && epi_warp) {
       drain(0, m0 + r, nullptr, 0, 0);
       drain(BN, m0 + TC_BM + r, nullptr, 0, 1);
     }
@@ -759,7 +837,7 @@ __global__ void __launch_bounds__(128, 1)
         if (threadIdx.x == 0) bulk_wait_read<0>();
         __syncthreads();
       }
-      if (ok2) {
+      if (ok2 && epi_warp) {
         if (h == 1) drain(0, m0 + r, args.out2, args.ld2, -1);  // first half's result
         drain((uint32_t)(h * BN), m0 + h * TC_BM + r, nullptr, 0, sdh);
       }
@@ -790,7 +868,7 @@ __global__ void __launch_bounds__(128, 1)
       ok2 = __all_sync(0xffffffffu, ok2);
       tc_fence_after();
     }
-    if (ok2) drain(BN, m0 + TC_BM + r, args.out2, args.ld2, -1);
+    if (ok2 && epi_warp) drain(BN, m0 + TC_BM + r, args.out2, args.ld2, -1);
   }
   // Shared memory stays valid until the stores have read it (the writes complete with the grid).
   if (threadIdx.x == 0) bulk_wait_read<0>();

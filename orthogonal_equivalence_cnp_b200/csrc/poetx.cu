@@ -203,18 +203,21 @@ Operand view(const void* base, long rows, long cols, long ld, long zrow = 0, lon
 }
 
 // 2-D tensor map of a row-major bf16 (or fp32) array, 128-byte swizzle; box_inner elements must
-// span 128 bytes (64 bf16 / 32 fp32).
+// span 128 bytes (64 bf16 / 32 fp32).  Int8 codes (dt = U8) are mapped unswizzled (the
+// converter warps read them row by row), any box up to 256 x 256.
 bool make_tmap(CUtensorMap* m, const Operand& op, uint32_t box_inner, uint32_t box_outer, int dt = BF16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
-  const uint64_t es = dt == F32 ? 4 : 2;
+  const uint64_t es = dt == F32 ? 4 : dt == U8 ? 1 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)op.cols, (cuuint64_t)op.rows};
   cuuint64_t strides[1] = {(cuuint64_t)op.ld * es};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt == F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-            const_cast<void*>(op.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  const CUtensorMapDataType type = dt == F32  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : dt == U8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return fn(m, type, 2, const_cast<void*>(op.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            dt == U8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -428,21 +431,26 @@ bool w256_ok(int dt, const GemmDesc& g) {
          4L * ((g.M + TCW_BM - 1) / TCW_BM) * (g.N / TCW_BN) >= 3L * kNumSms;
 }
 
-template <bool BMN, bool QMN>
+template <bool BMN, bool QMN, bool Q8 = false>
 poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* out2, long ld2, cudaStream_t st,
                          int cls) {
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
-  constexpr size_t smem = tcw_smem_bytes();
-  auto kern = gemm_w256_tc<BMN, QMN>;
+  constexpr size_t smem = tcw_smem_bytes<Q8>();
+  auto kern = gemm_w256_tc<BMN, QMN, Q8>;
   if (!attr_done[dev]) {
     if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
   CUtensorMap ta, tb, tq, td;
   if (!make_tmap(&ta, g.A, 64, TCW_BM)) return POETX_ERR_CUDA;
-  if (!make_tmap(&tb, g.B, 64, BMN ? 64 : TCW_BN)) return POETX_ERR_CUDA;
+  if (Q8) {
+    // int8 codes: a 64 (k) x 256 (n) box of the K-major array, or 256 (n) x 64 (k) of the MN-major one.
+    if (!make_tmap(&tb, g.B, BMN ? TCW_BN : 64, BMN ? 64 : TCW_BN, U8)) return POETX_ERR_CUDA;
+  } else if (!make_tmap(&tb, g.B, 64, BMN ? 64 : TCW_BN)) {
+    return POETX_ERR_CUDA;
+  }
   // Store boxes of D: 64 columns x 128 rows (one half's K chunk).
   if (!make_tmap(&td, view(g.epi.d1, g.M, g.N, g.epi.ld1), 64, TC_BM)) return POETX_ERR_CUDA;
   if (out2 != nullptr) {
@@ -454,15 +462,41 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.M = g.M; a.N = g.N; a.K = g.K;
   a.d1 = g.epi.d1; a.ld1 = g.epi.ld1;
   a.out2 = out2; a.ld2 = ld2;
+  a.bscale = g.b_scale;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(cls, st);
-  if (launch_pdl(kern, grid, dim3(128), smem, st, ta, tb, tq, td, a) != cudaSuccess) return POETX_ERR_CUDA;
+  if (launch_pdl(kern, grid, dim3(Q8 ? 256 : 128), smem, st, ta, tb, tq, td, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
+}
+
+// POET-XQ W0' GEMM: B is int8 codes with per-row scales (g.b_scale), dequantised in the kernel.
+// Always the 256 x 256 kernel (its converter warps are the only dequantising path): N in whole
+// 256-column tiles, rows of codes 16-byte aligned.
+poetx_status run_w_gemm_q8(const GemmDesc& g, const void* Q, long q_rows, bool q_mn, void* out2, long ld2,
+                           cudaStream_t st, int cls) {
+  const Epilogue& e = g.epi;
+  if (g.M <= 0 || g.K <= 0 || g.a_mn || g.batch != 1 || g.splits != 1 || g.N % TCW_BN) return POETX_ERR_UNSUPPORTED_SHAPE;
+  if (!e.d1 || e.d1_dtype != BF16 || e.alpha1 != 1.f || e.beta1 != 0.f || e.c || e.d2 || e.diag1 || e.split_stride1)
+    return POETX_ERR_INVALID_ARG;
+  if (!view_fits(g.A, false, g.M, g.K, 1) || !view_fits(g.B, g.b_mn, g.N, g.K, 1)) return POETX_ERR_INVALID_ARG;
+  if (!aligned16(g.A.base) || g.A.ld % 8 || !aligned16(g.B.base) || g.B.ld % 16 || !aligned16(e.d1) || e.ld1 % 8 ||
+      !aligned16(g.b_scale))
+    return POETX_ERR_ALIGNMENT;
+  if (out2 == nullptr) {
+    return g.b_mn ? launch_w256<true, false, true>(g, nullptr, 0, nullptr, 0, st, cls)
+                  : launch_w256<false, false, true>(g, nullptr, 0, nullptr, 0, st, cls);
+  }
+  if (q_rows < g.N || !aligned16(Q) || !aligned16(out2) || ld2 % 8) return POETX_ERR_ALIGNMENT;
+  if (!g.b_mn && !q_mn) return launch_w256<false, false, true>(g, Q, q_rows, out2, ld2, st, cls);
+  if (!g.b_mn && q_mn) return launch_w256<false, true, true>(g, Q, q_rows, out2, ld2, st, cls);
+  if (g.b_mn && !q_mn) return launch_w256<true, false, true>(g, Q, q_rows, out2, ld2, st, cls);
+  return launch_w256<true, true, true>(g, Q, q_rows, out2, ld2, st, cls);
 }
 
 // The W0' GEMM D = A . B^T -> d1, and (out2 != null, b = 256) out2 = D . Q^T or D . Q.
 poetx_status run_w_gemm(int dt, const GemmDesc& g, const void* Q, long q_rows, bool q_mn, void* out2, long ld2,
                         cudaStream_t st, int cls = POETX_KC_W_GEMM) {
+  if (g.b_scale != nullptr) return dt == BF16 ? run_w_gemm_q8(g, Q, q_rows, q_mn, out2, ld2, st, cls) : POETX_ERR_INVALID_ARG;
   if (out2 == nullptr) {
     if (!w256_ok(dt, g)) return run_gemm(dt, g, st, cls);
     POETX_TRY(check_gemm(g, BF16));
@@ -1073,9 +1107,9 @@ poetx_status check_ws(const void* ws, size_t have, size_t need) {
 }
 
 // Forward chain into caller buffers; `Z` receives the W0'-GEMM output.
-poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const void* W0p, const int32_t* pL,
-                           const int32_t* pR, const void* QR, const void* QP, void* Y, void* Z, char* U, char* V,
-                           char* Yp, cudaStream_t st) {
+poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const void* W0p, const float* W0s,
+                           const int32_t* pL, const int32_t* pR, const void* QR, const void* QP, void* Y, void* Z,
+                           char* U, char* V, char* Yp, cudaStream_t st) {
   const int dt = d->dtype, b = d->b;
   POETX_TRY(permute_cols(dt, X, d->d_in, U, d->d_in, n, d->d_in, pR, nullptr, false, st));
   POETX_TRY(bd_forward(dt, n, d->d_in, b, U, QP, V, st));
@@ -1083,6 +1117,7 @@ poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const voi
   g.M = (int)n; g.N = d->d_out; g.K = d->d_in;
   g.A = view(V, n, d->d_in, d->d_in);
   g.B = view(W0p, d->d_out, d->d_in, d->d_in);
+  g.b_scale = W0s;  // POET-XQ: W0' is int8 codes with per-row scales
   g.epi.d1 = Z; g.epi.d1_dtype = dt; g.epi.ld1 = d->d_out;
   if (Y == nullptr) return run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, st);  // recompute only (mem-mode backward)
   if (bd_fusable(dt, b, g)) {
@@ -1247,9 +1282,10 @@ poetx_status poetx_absorb(const poetx_desc* desc, const void* W0, const int32_t*
                       stream);
 }
 
-poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
-                           const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P, void* Y,
-                           void* saved, void* workspace, size_t ws_bytes, poetx_stream stream) {
+static poetx_status forward_impl(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                                 const float* W0s, const int32_t* perm_L, const int32_t* perm_R, const void* Q_R,
+                                 const void* Q_P, void* Y, void* saved, void* workspace, size_t ws_bytes,
+                                 poetx_stream stream) {
   POETX_TRY(check_desc(desc));
   if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
   if (n_tokens == 0) return POETX_OK;
@@ -1264,7 +1300,14 @@ poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, 
   const size_t zbytes = (size_t)n_tokens * desc->d_out * esize(desc->dtype);
   void* Z = desc->mode == POETX_FAST ? saved : ws + f.Z;
   char* U = desc->mode == POETX_FAST ? static_cast<char*>(saved) + zbytes : ws + f.U;
-  return forward_chain(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, Z, U, ws + f.V, ws + f.Yp, stream);
+  return forward_chain(desc, n_tokens, X, W0p, W0s, perm_L, perm_R, Q_R, Q_P, Y, Z, U, ws + f.V, ws + f.Yp, stream);
+}
+
+poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                           const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P, void* Y,
+                           void* saved, void* workspace, size_t ws_bytes, poetx_stream stream) {
+  return forward_impl(desc, n_tokens, X, W0p, nullptr, perm_L, perm_R, Q_R, Q_P, Y, saved, workspace, ws_bytes,
+                      stream);
 }
 
 // Side stream of the backward pass.  Two chains of the backward are independent: the
@@ -1311,11 +1354,11 @@ struct SideJoin {
   }
 };
 
-poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X, const void* W0p,
-                            const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
-                            const float* theta_R, const float* theta_P, const void* saved, const void* powers,
-                            void* dX, float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
-                            poetx_stream stream) {
+static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
+                                  const void* W0p, const float* W0s, const int32_t* perm_L, const int32_t* perm_R,
+                                  const void* Q_R, const void* Q_P, const float* theta_R, const float* theta_P,
+                                  const void* saved, const void* powers, void* dX, float* grad_theta_R,
+                                  float* grad_theta_P, void* workspace, size_t ws_bytes, poetx_stream stream) {
   POETX_TRY(check_desc(desc));
   POETX_TRY(check_powers(desc, powers));
   if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
@@ -1341,7 +1384,7 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
   const char* U = desc->mode == POETX_FAST ? static_cast<const char*>(saved) + (size_t)n * dout * esize(dt) : ws + w.U;
   if (desc->mode == POETX_MEM) {
     // POET-Xmem: recompute U = X[:, pi_R], V = BD_P.U and Z = V.W0'^T from X.
-    POETX_TRY(forward_chain(desc, n, X, W0p, perm_L, perm_R, Q_R, Q_P, nullptr, ws + w.Z, ws + w.U, ws + w.V,
+    POETX_TRY(forward_chain(desc, n, X, W0p, W0s, perm_L, perm_R, Q_R, Q_P, nullptr, ws + w.Z, ws + w.U, ws + w.V,
                             nullptr, stream));
     Z = ws + w.Z;
   }
@@ -1362,6 +1405,7 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
   g.M = (int)n; g.N = din; g.K = dout;
   g.A = view(ws + w.dZ, n, dout, dout);
   g.B = view(W0p, dout, din, din); g.b_mn = true;
+  g.b_scale = W0s;
   g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
   const bool fused_du = bd_fusable(dt, b, g);
   if (fused_du) POETX_TRY(run_w_gemm(dt, g, Q_P, din, true, ws + w.dU, din, stream, POETX_KC_W_GEMM_ADJ));
@@ -1387,6 +1431,15 @@ poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY
                             grad_theta_R, ws + w.cnpR, stream));
   return cnp_bwd_generic(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + w.GpP), w.sP,
                          grad_theta_P, ws + w.cnpP, stream);
+}
+
+poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X, const void* W0p,
+                            const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
+                            const float* theta_R, const float* theta_P, const void* saved, const void* powers,
+                            void* dX, float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
+                            poetx_stream stream) {
+  return backward_impl(desc, n_tokens, dY, X, W0p, nullptr, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved,
+                       powers, dX, grad_theta_R, grad_theta_P, workspace, ws_bytes, stream);
 }
 
 size_t poetx_wc_saved_size(const poetx_desc* desc) {
@@ -1515,21 +1568,19 @@ poetx_status poetx_wc_backward(const poetx_desc* desc, int n_tokens, const void*
                          ws + m.cnpP, stream);
 }
 
-poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, const void* Q_P,
-                         const int32_t* perm_L_old, const int32_t* perm_R_old, const int32_t* perm_L_new,
-                         const int32_t* perm_R_new, float* theta_R, float* theta_P, void* workspace, size_t ws_bytes,
-                         poetx_stream stream) {
-  POETX_TRY(check_desc(desc));
-  POETX_TRY(check_ptrs({W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P}));
+// The merge with W0' read from W_in and the new W0' written to W_out (the same array, or for
+// POET-XQ the dequantised weight in the M2 region and the result in the T region).
+static poetx_status merge_impl(const poetx_desc* desc, const void* W_in, void* W_out, const void* Q_R,
+                               const void* Q_P, const int32_t* perm_L_old, const int32_t* perm_R_old,
+                               const int32_t* perm_L_new, const int32_t* perm_R_new, float* theta_R, float* theta_P,
+                               char* ws, poetx_stream stream) {
   const MergePlan m = merge_plan(desc);
-  POETX_TRY(check_ws(workspace, ws_bytes, m.total));
-  char* ws = static_cast<char*>(workspace);
   const int dt = desc->dtype, b = desc->b, din = desc->d_in, dout = desc->d_out;
   // T = W0' . BD_P   (column blocks: T[:, blk z] = W0'[:, blk z] . Q_P,z)
   {
     GemmDesc g;
     g.M = dout; g.N = b; g.K = b; g.batch = din / b;
-    g.A = view(W0p, dout, din, din, 0, b);
+    g.A = view(W_in, dout, din, din, 0, b);
     g.B = view(Q_P, din, b, b, b, 0); g.b_mn = true;
     g.epi.d1 = ws + m.T; g.epi.d1_dtype = dt; g.epi.ld1 = din; g.epi.zcol1 = b;
     POETX_TRY(run_gemm(dt, g, stream, POETX_KC_MERGE_GEMM));
@@ -1564,11 +1615,100 @@ poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, con
     perm_compose_kernel<<<ew_grid(din), 256, 0, stream>>>(inv, perm_R_new, din, sR);
   }
   POETX_TRY(last_launch());
-  POETX_TRY(permute_cols(dt, ws + m.M2, din, W0p, din, dout, din, sR, sL, false, stream));
+  POETX_TRY(permute_cols(dt, ws + m.M2, din, W_out, din, dout, din, sR, sL, false, stream));
   const size_t P = (size_t)b * (b - 1) / 2;
   if (cudaMemsetAsync(theta_R, 0, (size_t)(dout / b) * P * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
   if (cudaMemsetAsync(theta_P, 0, (size_t)(din / b) * P * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
   return POETX_OK;
+}
+
+poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, const void* Q_P,
+                         const int32_t* perm_L_old, const int32_t* perm_R_old, const int32_t* perm_L_new,
+                         const int32_t* perm_R_new, float* theta_R, float* theta_P, void* workspace, size_t ws_bytes,
+                         poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  POETX_TRY(check_ptrs({W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P}));
+  POETX_TRY(check_ws(workspace, ws_bytes, merge_plan(desc).total));
+  return merge_impl(desc, W0p, W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P,
+                    static_cast<char*>(workspace), stream);
+}
+
+// ------------------------------------------------------------------------------- POET-XQ
+// POET-XQ holds W0' as int8 codes with one fp32 scale per row and runs POET-Xmem on it: the
+// W0' GEMMs dequantise their B tiles in shared memory, nothing keeps a bf16 W0'.
+static poetx_status check_xq(const poetx_desc* desc) {
+  POETX_TRY(check_desc(desc));
+  if (desc->dtype != POETX_BF16 || desc->mode != POETX_MEM) return POETX_ERR_INVALID_ARG;
+  if (desc->d_in % 256 || desc->d_out % 256) return POETX_ERR_UNSUPPORTED_SHAPE;
+  return POETX_OK;
+}
+
+static poetx_status xq_quantize(const poetx_desc* d, const void* W, int8_t* q, float* s, cudaStream_t st) {
+  const int grid = (int)std::min<long>((d->d_out + 7) / 8, (long)kNumSms * 8);
+  LaunchScope ls(POETX_KC_ELEMENTWISE, st);
+  if (launch_pdl(quantize_rows_kernel, dim3(grid), dim3(256), 0, st, static_cast<const uint16_t*>(W), (long)d->d_in,
+                 (long)d->d_out, d->d_in, q, (long)d->d_in, s) != cudaSuccess)
+    return POETX_ERR_CUDA;
+  return last_launch();
+}
+
+static poetx_status xq_dequantize(const poetx_desc* d, const int8_t* q, const float* s, void* W, cudaStream_t st) {
+  LaunchScope ls(POETX_KC_ELEMENTWISE, st);
+  if (launch_pdl(dequantize_rows_kernel, dim3(ew_grid((long)d->d_out * d->d_in / 8)), dim3(256), 0, st, q,
+                 (long)d->d_in, s, (long)d->d_out, d->d_in, static_cast<uint16_t*>(W), (long)d->d_in) != cudaSuccess)
+    return POETX_ERR_CUDA;
+  return last_launch();
+}
+
+poetx_status poetx_xq_quantize(const poetx_desc* desc, const void* W0p, int8_t* W0q, float* W0s,
+                               poetx_stream stream) {
+  POETX_TRY(check_xq(desc));
+  POETX_TRY(check_ptrs({W0p, W0q, W0s}));
+  return xq_quantize(desc, W0p, W0q, W0s, stream);
+}
+
+poetx_status poetx_xq_dequantize(const poetx_desc* desc, const int8_t* W0q, const float* W0s, void* W0p,
+                                 poetx_stream stream) {
+  POETX_TRY(check_xq(desc));
+  POETX_TRY(check_ptrs({W0p, W0q, W0s}));
+  return xq_dequantize(desc, W0q, W0s, W0p, stream);
+}
+
+poetx_status poetx_xq_forward(const poetx_desc* desc, int n_tokens, const void* X, const int8_t* W0q,
+                              const float* W0s, const int32_t* perm_L, const int32_t* perm_R, const void* Q_R,
+                              const void* Q_P, void* Y, void* workspace, size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_xq(desc));
+  POETX_TRY(check_ptrs({W0q, W0s}));
+  return forward_impl(desc, n_tokens, X, W0q, W0s, perm_L, perm_R, Q_R, Q_P, Y, nullptr, workspace, ws_bytes,
+                      stream);
+}
+
+poetx_status poetx_xq_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
+                               const int8_t* W0q, const float* W0s, const int32_t* perm_L, const int32_t* perm_R,
+                               const void* Q_R, const void* Q_P, const float* theta_R, const float* theta_P,
+                               void* dX, float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
+                               poetx_stream stream) {
+  POETX_TRY(check_xq(desc));
+  POETX_TRY(check_ptrs({W0q, W0s}));
+  return backward_impl(desc, n_tokens, dY, X, W0q, W0s, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, nullptr,
+                       nullptr, dX, grad_theta_R, grad_theta_P, workspace, ws_bytes, stream);
+}
+
+poetx_status poetx_xq_merge(const poetx_desc* desc, int8_t* W0q, float* W0s, const void* Q_R, const void* Q_P,
+                            const int32_t* perm_L_old, const int32_t* perm_R_old, const int32_t* perm_L_new,
+                            const int32_t* perm_R_new, float* theta_R, float* theta_P, void* workspace,
+                            size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_xq(desc));
+  POETX_TRY(check_ptrs({W0q, W0s, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P}));
+  const MergePlan m = merge_plan(desc);
+  POETX_TRY(check_ws(workspace, ws_bytes, m.total));
+  char* ws = static_cast<char*>(workspace);
+  // Dequantise into the M2 region (read only by the first merge product), merge into the T
+  // region, quantise back.  The bf16 weight lives only in the workspace for the call.
+  POETX_TRY(xq_dequantize(desc, W0q, W0s, ws + m.M2, stream));
+  POETX_TRY(merge_impl(desc, ws + m.M2, ws + m.T, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R,
+                       theta_P, ws, stream));
+  return xq_quantize(desc, ws + m.T, W0q, W0s, stream);
 }
 
 poetx_status poetx_device_status(int* detail) {

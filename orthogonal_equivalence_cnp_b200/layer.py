@@ -11,7 +11,7 @@ import torch
 from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_adamw_cfg, poetx_adamw_reset,
                poetx_adamw_step, poetx_backward, poetx_cnp, poetx_cnp_powers_size, poetx_desc, poetx_forward,
                poetx_merge, poetx_wc_backward, poetx_wc_forward, poetx_wc_saved_size, poetx_wc_workspace_size,
-               poetx_workspace_size)
+               poetx_workspace_size, poetx_xq_backward, poetx_xq_forward, poetx_xq_merge, poetx_xq_quantize)
 
 TORCH_DTYPE = {POETX_F32: torch.float32, POETX_BF16: torch.bfloat16}
 
@@ -34,6 +34,9 @@ class PoetxLayer:
         P = b * (b - 1) // 2
         dev = self.device
         self.W0p = torch.empty(dout, din, dtype=dt, device=dev)
+        # POET-XQ (after quantize()): W0' as int8 codes W0q [d_out, d_in] and scales W0s [d_out].
+        self.xq = False
+        self.W0q = self.W0s = None
         # theta_R and theta_P (and their gradients and AdamW moments) are stored back to back so
         # that one optimiser launch covers both sides.
         nbo, nbi = dout // b, din // b
@@ -78,14 +81,32 @@ class PoetxLayer:
         poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.powers, self.ws)
 
     def forward(self, X: torch.Tensor):
-        poetx_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
-                      self.saved, self.ws)
+        if self.xq:
+            poetx_xq_forward(self.desc, self.n, X, self.W0q, self.W0s, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
+                             self.Y, self.ws)
+        else:
+            poetx_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
+                          self.saved, self.ws)
         return self.Y
 
     def backward(self, dY: torch.Tensor, X: torch.Tensor):
-        poetx_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
-                       self.theta_R, self.theta_P, self.saved, self.powers, self.dX, self.g_R, self.g_P, self.ws)
+        if self.xq:
+            poetx_xq_backward(self.desc, self.n, dY, X, self.W0q, self.W0s, self.perm_L, self.perm_R, self.Q_R,
+                              self.Q_P, self.theta_R, self.theta_P, self.dX, self.g_R, self.g_P, self.ws)
+        else:
+            poetx_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
+                           self.theta_R, self.theta_P, self.saved, self.powers, self.dX, self.g_R, self.g_P, self.ws)
         return self.dX, self.g_R, self.g_P
+
+    def quantize(self):
+        """Switches the layer to POET-XQ (mem mode, bf16): W0' becomes int8 codes with one scale
+        per row, and the bf16 W0' is released."""
+        d = self.desc
+        self.W0q = torch.empty(d.d_out, d.d_in, dtype=torch.int8, device=self.device)
+        self.W0s = torch.empty(d.d_out, dtype=torch.float32, device=self.device)
+        poetx_xq_quantize(d, self.W0p, self.W0q, self.W0s)
+        self.W0p = None  # stream-ordered release: the quantiser has been enqueued before it
+        self.xq = True
 
     def step(self, X: torch.Tensor, dY: torch.Tensor):
         """CNP forward + layer forward + layer backward (incl. the CNP adjoint)."""
@@ -131,7 +152,11 @@ class PoetxLayer:
 
     def merge(self, pi_L_new: torch.Tensor, pi_R_new: torch.Tensor):
         """Folds R and P into W0', absorbs the new permutations and resets theta (Q must be current)."""
-        poetx_merge(self.desc, self.W0p, self.Q_R, self.Q_P, self.perm_L, self.perm_R, pi_L_new, pi_R_new,
-                    self.theta_R, self.theta_P, self.ws)
+        if self.xq:
+            poetx_xq_merge(self.desc, self.W0q, self.W0s, self.Q_R, self.Q_P, self.perm_L, self.perm_R, pi_L_new,
+                           pi_R_new, self.theta_R, self.theta_P, self.ws)
+        else:
+            poetx_merge(self.desc, self.W0p, self.Q_R, self.Q_P, self.perm_L, self.perm_R, pi_L_new, pi_R_new,
+                        self.theta_R, self.theta_P, self.ws)
         self.perm_L.copy_(pi_L_new)
         self.perm_R.copy_(pi_R_new)

@@ -128,3 +128,31 @@ def test_adamw_host_validation():
                 P.poetx_adamw_cfg(-1.0, 0.5, 0.9, 0.999, 1e-8, 0.0), P.poetx_adamw_cfg(1e-3, 0.5, 0.9, 0.999, 1e-8, -1.0)):
         assert L.poetx_adamw_step(ctypes.byref(bad), 16, 1, A, A, A, A, None) == 1
     assert L.poetx_adamw_reset(-1, A, A, None) == 1 and L.poetx_adamw_reset(0, None, None, None) == 0
+
+
+def test_xq_host_validation():
+    # POET-XQ: bf16 and mem mode only, d_in and d_out multiples of 256, pointers checked before
+    # anything is launched.
+    L = P.lib()
+    A = 1 << 20
+    good = P.poetx_desc(512, 768, 256, 3, P.POETX_BF16, P.POETX_MEM)
+    fast = P.poetx_desc(512, 768, 256, 3, P.POETX_BF16, P.POETX_FAST)
+    f32 = P.poetx_desc(512, 768, 256, 3, P.POETX_F32, P.POETX_MEM)
+    odd = P.poetx_desc(384, 768, 128, 3, P.POETX_BF16, P.POETX_MEM)
+
+    def fwd(d, codes=A, scales=A, ws_bytes=16):
+        return L.poetx_xq_forward(ctypes.byref(d), 64, A, codes, scales, A, A, A, A, A, A, ws_bytes, None)
+
+    assert fwd(fast) == 1 and fwd(f32) == 1 and fwd(odd) == 2
+    assert fwd(good) == 4                      # workspace too small
+    assert fwd(good, codes=None) == 1 and fwd(good, scales=A + 4) == 3
+    assert L.poetx_xq_forward(ctypes.byref(good), 0, None, A, A, None, None, None, None, None, None, 0, None) == 0
+    bwd = lambda d, ws_bytes=16: L.poetx_xq_backward(ctypes.byref(d), 64, A, A, A, A, A, A, A, A, A, A, A, A, A, A,
+                                                     ws_bytes, None)
+    assert bwd(fast) == 1 and bwd(odd) == 2 and bwd(good) == 4
+    assert L.poetx_xq_quantize(ctypes.byref(fast), A, A, A, None) == 1
+    assert L.poetx_xq_quantize(ctypes.byref(good), None, A, A, None) == 1
+    assert L.poetx_xq_quantize(ctypes.byref(good), A, A, A + 8, None) == 3
+    assert L.poetx_xq_dequantize(ctypes.byref(odd), A, A, A, None) == 2
+    assert L.poetx_xq_merge(ctypes.byref(good), A, A, A, A, A, A, A, A, A, A, A, 16, None) == 4
+    assert L.poetx_xq_merge(ctypes.byref(f32), A, A, A, A, A, A, A, A, A, A, A, 1 << 30, None) == 1
