@@ -561,8 +561,10 @@ __global__ void __launch_bounds__(128, 1)
 // Q8 (POET-XQ, the replication review of POET-X, "Summary" and "Strengths": the quantised
 // variant works through POET-Xmem, so no dequantised weight is ever stored): B is int8 codes
 // with one fp32 scale per row of the B array (bscale).  TMA brings each k step's 16 KiB of codes
-// into one of two staging slots; four more warps (threads 128..255) turn them into bf16
-// scale * code, written straight into the stage's swizzled B tile, and signal the MMA issuer.
+// into the first half of the stage's B region (so the codes ride the same 3-deep ring as A);
+// eight more warps (threads 128..383) read all of them into registers, meet on a named barrier,
+// then expand them in place into the stage's swizzled bf16 B tile (scale * code) and signal the
+// MMA issuer.
 struct WideArgs {
   int M, N, K;
   void* d1;    // bf16 [M, N] store of D (may be null when out2 is set)
@@ -574,13 +576,29 @@ struct WideArgs {
 
 constexpr int TCW_BM = 256, TCW_BN = 256, TCW_STAGES = 3;
 constexpr uint32_t TCW_Q8_TILE = 256 * TC_BK;  // int8 codes of one k step's B tile
-template <bool Q8 = false>
+constexpr int TCW_CONV_THREADS = 256;           // Q8 converter warps 4..11
+constexpr int TCW_CONV_CHUNKS = 2048 / TCW_CONV_THREADS;  // 8-code chunks per converter thread per k step
 __host__ __device__ constexpr size_t tcw_smem_bytes() {
-  return (size_t)TCW_STAGES * (TCW_BM * TC_BK * 2 + TCW_BN * TC_BK * 2) + (Q8 ? 2 * TCW_Q8_TILE : 0) + 1024 + 256;
+  return (size_t)TCW_STAGES * (TCW_BM * TC_BK * 2 + TCW_BN * TC_BK * 2) + 1024 + 256;
+}
+
+// Named barrier 1 over the `count` threads of the converter warps, ANDing p across them: every
+// participant gets the same answer, so a bounded wait that gave up anywhere ends all of them.
+__device__ __forceinline__ bool converters_all(bool p, int count) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, 1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 template <bool B_MN, bool Q_MN, bool Q8 = false>
-__global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
+__global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
     gemm_w256_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmD,
                  const WideArgs args) {
@@ -595,8 +613,7 @@ __global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr uint32_t STG_OFF = STAGES * STAGE_BYTES;  // Q8: two int8 staging slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STG_OFF + (Q8 ? 2 * TCW_Q8_TILE : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
   const uint32_t smem0 = smem_u32(smem);
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -604,9 +621,8 @@ __global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
   const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
   const uint32_t q_full = smem_u32(bars + 2 * STAGES + 1);
   const uint32_t acc2_bar = smem_u32(bars + 2 * STAGES + 2);
-  // Q8: B tile of stage s converted (one arrival per converter warp); staging slot j free again.
+  // Q8: B tile of stage s converted (one arrival per converter warp).
   auto conv_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + 4 + s); };
-  auto sfree_bar = [&](int j) { return smem_u32(bars + 3 * STAGES + 4 + j); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * TCW_BM, n0 = blockIdx.x * BN;
@@ -624,10 +640,8 @@ __global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
     mbar_init(accum_bar, 1);
     mbar_init(q_full, 1);
     mbar_init(acc2_bar, 1);
-    if (Q8) {
-      for (int s = 0; s < STAGES; ++s) mbar_init(conv_bar(s), 4);
-      for (int j = 0; j < 2; ++j) mbar_init(sfree_bar(j), 4);
-    }
+    if (Q8)
+      for (int s = 0; s < STAGES; ++s) mbar_init(conv_bar(s), TCW_CONV_THREADS / 32);
     fence_mbar_init();
     fence_proxy_async_smem();
     prefetch_tmap(&tmA);
@@ -654,14 +668,11 @@ __global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
       const int k0 = i * TC_BK;
       const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
       if (Q8) {
-        // Codes of step i into staging slot i % 2, once the converters are done with step i - 2.
-        const int j = i & 1;
-        if (!mbar_wait(sfree_bar(j), ((uint32_t)(i >> 1) & 1u) ^ 1u, KID_GEMM_TC, 17)) { ok = false; break; }
+        // Codes of step i into the first 16 KiB of the stage's B region.
         mbar_arrive_expect_tx(full_bar(s), A_BYTES + TCW_Q8_TILE);
         tma_load_2d(sa, &tmA, full_bar(s), k0, m0);
-        const uint32_t stg = smem0 + STG_OFF + j * TCW_Q8_TILE;
-        if (!B_MN) tma_load_2d(stg, &tmB, full_bar(s), k0, n0);  // box 64 (k) x 256 (n) codes
-        else tma_load_2d(stg, &tmB, full_bar(s), n0, k0);        // box 256 (n) x 64 (k) codes
+        if (!B_MN) tma_load_2d(sb, &tmB, full_bar(s), k0, n0);  // box 64 (k) x 256 (n) codes
+        else tma_load_2d(sb, &tmB, full_bar(s), n0, k0);        // box 256 (n) x 64 (k) codes
         continue;
       }
       mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
@@ -716,16 +727,19 @@ __global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
     mma_commit(accum_bar);
   } else if (Q8 && warp >= 4) {
     // ---------------- converters: codes -> bf16 scale * code in the stage's swizzled B tile.
-    // Thread t converts chunks c = 128 j + t (j < 16) of 8 codes each.  K-major B (rows n, 64
-    // codes each): chunk c is row c / 8, 16-byte chunk c % 8.  MN-major B (rows k, 256 codes
-    // each): chunk c is row k = c / 32, columns 8 (c % 32) .. +7, i.e. 64-column sub-tile
-    // (c % 32) / 8, chunk c % 8.  Either way the scale belongs to the code's row of B.
+    // Thread t converts chunks c = CT j + t (CT converter threads, j < 2048 / CT) of 8 codes each.
+    // K-major B (rows n, 64 codes each): chunk c is row c / 8, 16-byte chunk c % 8.  MN-major B
+    // (rows k, 256 codes each): chunk c is row k = c / 32, columns 8 (c % 32) .. +7, i.e.
+    // 64-column sub-tile (c % 32) / 8, chunk c % 8.  Either way the scale belongs to the code's
+    // row of B.
+    constexpr int CT = TCW_CONV_THREADS, NCH = TCW_CONV_CHUNKS;
     const int t = threadIdx.x - 128;
-    float sc[16], scn[16];
-    auto load_scales = [&](int i, float (&dst)[16]) {
+    float sc[NCH], scn[NCH];
+    auto load_scales = [&](int i, float (&dst)[NCH]) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int row = B_MN ? i * TC_BK + j * 4 + (t >> 5) : n0 + j * 16 + (t >> 3);
+      for (int j = 0; j < NCH; ++j) {
+        const int c = j * CT + t;
+        const int row = B_MN ? i * TC_BK + (c >> 5) : n0 + (c >> 3);
         dst[j] = row < (B_MN ? args.K : args.N) ? __ldg(args.bscale + row) : 0.f;
       }
     };
@@ -734,32 +748,35 @@ __global__ void __launch_bounds__(Q8 ? 256 : 128, 1)
       const int s = i % STAGES;
       const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) sc[j] = scn[j];
+      for (int j = 0; j < NCH; ++j) sc[j] = scn[j];
       if (B_MN && i + 1 < nkt) load_scales(i + 1, scn);  // K-major: the same rows every step
-      if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, KID_GEMM_TC, 18))) break;  // warp-uniform exit
-      const uint8_t* stg = smem + STG_OFF + (i & 1) * TCW_Q8_TILE;
+      // All converter warps agree (named barrier) before anyone reads, so a timeout ends all of them.
+      if (!converters_all(mbar_wait(full_bar(s), ph, KID_GEMM_TC, 18), CT)) break;
       uint8_t* tile = smem + s * STAGE_BYTES + A_BYTES;
+      uint2 code[NCH];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int c = j * 128 + t;
-        int src, dst;
+      for (int j = 0; j < NCH; ++j) {
+        const int c = j * CT + t;
+        code[j] = *reinterpret_cast<const uint2*>(tile + (!B_MN ? (c >> 3) * 64 + (c & 7) * 8
+                                                                 : (c >> 5) * 256 + (c & 31) * 8));
+      }
+      converters_all(true, CT);  // every code of the stage is in registers before the expansion
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        const int c = j * CT + t;
+        int dst;
         if (!B_MN) {
           const int row = c >> 3, ch = c & 7;
-          src = row * 64 + ch * 8;
           dst = row * 128 + ((ch ^ (row & 7)) << 4);
         } else {
           const int row = c >> 5, nc = c & 31;
-          src = row * 256 + nc * 8;
           dst = (nc >> 3) * 8192 + row * 128 + (((nc & 7) ^ (row & 7)) << 4);
         }
-        *reinterpret_cast<uint4*>(tile + dst) = dequant8_bf16(*reinterpret_cast<const uint2*>(stg + src), sc[j]);
+        *reinterpret_cast<uint4*>(tile + dst) = dequant8_bf16(code[j], sc[j]);
       }
       fence_proxy_async_smem();  // the tensor core reads what the threads wrote
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(conv_bar(s));
-        mbar_arrive(sfree_bar(i & 1));
-      }
+      if (lane == 0) mbar_arrive(conv_bar(s));
     }
   }
   __syncwarp();

@@ -437,7 +437,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
-  constexpr size_t smem = tcw_smem_bytes<Q8>();
+  constexpr size_t smem = tcw_smem_bytes();
   auto kern = gemm_w256_tc<BMN, QMN, Q8>;
   if (!attr_done[dev]) {
     if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
@@ -465,7 +465,8 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.bscale = g.b_scale;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(cls, st);
-  if (launch_pdl(kern, grid, dim3(Q8 ? 256 : 128), smem, st, ta, tb, tq, td, a) != cudaSuccess) return POETX_ERR_CUDA;
+  if (launch_pdl(kern, grid, dim3(Q8 ? 128 + TCW_CONV_THREADS : 128), smem, st, ta, tb, tq, td, a) != cudaSuccess)
+    return POETX_ERR_CUDA;
   return last_launch();
 }
 
@@ -1392,14 +1393,15 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   POETX_TRY(side_stream(&ss));
   std::lock_guard<std::mutex> side_lock(ss->mu);
   const cudaStream_t side = ss->st;
-  // Output side: dY' = dY[:, pi_L]; dZ = BD_R^T-adjoint; G_R partials on the side stream, beside
-  // the W0' GEMM below (which leaves SMs idle in its last wave).
+  // Output side: dY' = dY[:, pi_L]; then G_R partials on the side stream beside dZ =
+  // BD_R^T-adjoint (both read dY', so it is shared through L2), leaving the W0' GEMM below the
+  // whole GPU.
   POETX_TRY(permute_cols(dt, dY, dout, ws + w.dYp, dout, n, dout, perm_L, nullptr, false, stream));
-  POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
   POETX_TRY(stream_edge(stream, side, ss->ev[0]));
   SideJoin join{stream, side, ss->ev[3], true};
   POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, side));
   if (cudaEventRecord(ss->ev[1], side) != cudaSuccess) return POETX_ERR_CUDA;  // G_R partials done
+  POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
   // dV = dZ . W0' (and, for b = 256, dU_i = dV_i . Q_P,i in the same kernel)
   GemmDesc g;
   g.M = (int)n; g.N = din; g.K = dout;
