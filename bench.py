@@ -56,9 +56,9 @@ def step_flops(s: I.LayerShape) -> dict:
 
 
 # DRAM bytes (read + write) of one W0' launch, from the ncu capture summarised in
-# profiles/gemm_w256_fwd_2048x4096x4096_b256_ncu.md (bench workload, forward launch).  Only valid
-# for that workload and that kernel build; None otherwise.
-W_GEMM_TRAFFIC = {"llama8b_attn_4096_b256_bf16": 52.461056e6 + 3.457792e6}
+# profiles/gemm_w256_bf16_2048x4096x4096_b256_traffic.md (bench workload, mean of two forward and
+# two adjoint launches).  Only valid for that workload and that kernel build; None otherwise.
+W_GEMM_TRAFFIC = {"llama8b_attn_4096_b256_bf16": 52.469e6 + 0.750e6}
 
 
 def w_gemm_flops(s: I.LayerShape) -> int:
@@ -560,8 +560,8 @@ def run_poetx(args):
                      "kernel": "w0_gemm (Z = V W0'^T with Y' = BD_R Z; dV = dZ W0' with dU = BD_P^T dV)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": W_GEMM_TRAFFIC.get(args.workload),
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one forward launch "
-                                       "(profiles/gemm_w256_fwd_2048x4096x4096_b256_ncu.md)",
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean of two forward and "
+                                       "two adjoint launches (profiles/gemm_w256_bf16_2048x4096x4096_b256_traffic.md)",
                      "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                      "frac_of_sustained": round(achieved / float(peaks["bf16_tflops_sustained"]), 4),
                      "launch_ms": round(w_avg_ms, 4), "launches": wcnt,
