@@ -284,6 +284,14 @@ poetx_status poetx_adamw_step(const poetx_adamw_cfg* cfg, long long n, int t, fl
  * restarts the moments with the parameters (their step count t starts again at 1). */
 poetx_status poetx_adamw_reset(long long n, float* m, float* v, poetx_stream stream);
 
+/* Host check of a permutation (HOST memory): POETX_OK if perm holds every value of [0, n)
+ * exactly once, else POETX_ERR_INVALID_ARG.  The layer calls assume bijections and do not check
+ * them; with the environment variable POETX_DEBUG set (and not "0") when the library first looks
+ * at it, poetx_absorb, poetx_forward, poetx_backward and poetx_merge copy their permutations to
+ * the host in stream order and return POETX_ERR_INVALID_ARG, launching nothing, when one is not
+ * a bijection (skipped while the stream is being captured). */
+poetx_status poetx_check_permutation(const int32_t* perm, int n);
+
 /* Human-readable name of a status code (static storage). */
 const char* poetx_status_string(poetx_status s);
 

@@ -20,6 +20,7 @@ __all__ = [
     "poetx_cnp_blocks_noalloc", "poetx_cnp_powers_size", "poetx_adamw_cfg", "poetx_adamw_step",
     "poetx_adamw_reset", "poetx_wc_saved_size", "poetx_wc_workspace_size", "poetx_wc_forward", "poetx_wc_backward",
     "poetx_xq_quantize", "poetx_xq_dequantize", "poetx_xq_forward", "poetx_xq_backward", "poetx_xq_merge",
+    "poetx_check_permutation",
 ]
 
 POETX_F32, POETX_BF16 = 0, 1
@@ -87,6 +88,7 @@ _SIGNATURES = {
     "poetx_xq_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_xq_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_xq_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_check_permutation": (_I, [_P, _I]),
     "poetx_status_string": (ctypes.c_char_p, [_I]),
     "poetx_device_status": (_I, [ctypes.POINTER(ctypes.c_int)]),
     "poetx_launch_count": (ctypes.c_ulonglong, []),
@@ -275,6 +277,18 @@ def poetx_xq_merge(desc, W0q, W0s, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new,
     _check(lib().poetx_xq_merge(ctypes.byref(desc), _ptr(W0q), _ptr(W0s), _ptr(Q_R), _ptr(Q_P), _ptr(perm_L_old),
                                 _ptr(perm_R_old), _ptr(perm_L_new), _ptr(perm_R_new), _ptr(theta_R),
                                 _ptr(theta_P), _ptr(workspace), ws_bytes, _stream(stream)), "poetx_xq_merge")
+
+
+def poetx_check_permutation(perm, n=None):
+    """perm: a HOST int32 array (numpy or CPU tensor) or a raw host address; raises unless it is a
+    bijection of [0, n)."""
+    import numpy as np
+    if isinstance(perm, int):
+        addr, n = perm, n
+    else:
+        arr = np.ascontiguousarray(np.asarray(perm), dtype=np.int32)
+        perm, addr, n = arr, arr.ctypes.data, arr.size if n is None else n
+    _check(lib().poetx_check_permutation(addr, n), "poetx_check_permutation")
 
 
 def poetx_device_status():

@@ -9,6 +9,8 @@
 #include <vector>
 #include <initializer_list>
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/poetx_testing.h"
@@ -1092,6 +1094,45 @@ WcPlan wc_plan(const poetx_desc* d) {
   return m;
 }
 
+// Every value in [0, n) exactly once.
+bool is_bijection(const int32_t* p, int n) {
+  std::vector<unsigned char> seen((size_t)std::max(n, 0), 0);
+  for (int i = 0; i < n; ++i) {
+    const int32_t v = p[i];
+    if (v < 0 || v >= n || seen[v]) return false;
+    seen[v] = 1;
+  }
+  return true;
+}
+
+// With POETX_DEBUG set (and not "0") in the environment, read once per process, the entry points
+// that take permutations copy them to the host in stream order and check that they are
+// bijections before anything is launched.  Skipped while the stream is being captured, where a
+// synchronising copy is not allowed.
+bool debug_checks() {
+  static const bool on = [] {
+    const char* e = std::getenv("POETX_DEBUG");
+    return e != nullptr && *e != 0 && std::strcmp(e, "0") != 0;
+  }();
+  return on;
+}
+
+poetx_status debug_check_perms(cudaStream_t st, std::initializer_list<std::pair<const int32_t*, int>> perms) {
+  if (!debug_checks()) return POETX_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return POETX_ERR_CUDA;
+  if (cs != cudaStreamCaptureStatusNone) return POETX_OK;
+  for (const auto& pr : perms) {
+    std::vector<int32_t> h((size_t)std::max(pr.second, 0));
+    if (pr.second > 0 &&
+        cudaMemcpyAsync(h.data(), pr.first, (size_t)pr.second * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return POETX_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return POETX_ERR_CUDA;
+    if (!is_bijection(h.data(), pr.second)) return POETX_ERR_INVALID_ARG;
+  }
+  return POETX_OK;
+}
+
 poetx_status check_ptrs(std::initializer_list<const void*> ps) {
   for (const void* p : ps) {
     if (p == nullptr) return POETX_ERR_INVALID_ARG;
@@ -1199,6 +1240,11 @@ poetx_status poetx_adamw_reset(long long n, float* m, float* v, poetx_stream str
   return cudaMemsetAsync(v, 0, (size_t)n * 4, stream) == cudaSuccess ? POETX_OK : POETX_ERR_CUDA;
 }
 
+poetx_status poetx_check_permutation(const int32_t* perm, int n) {
+  if (n < 0 || (n > 0 && perm == nullptr)) return POETX_ERR_INVALID_ARG;
+  return is_bijection(perm, n) ? POETX_OK : POETX_ERR_INVALID_ARG;
+}
+
 const char* poetx_status_string(poetx_status s) {
   switch (s) {
     case POETX_OK: return "POETX_OK";
@@ -1279,6 +1325,7 @@ poetx_status poetx_absorb(const poetx_desc* desc, const void* W0, const int32_t*
   POETX_TRY(check_desc(desc));
   POETX_TRY(check_ptrs({W0, perm_L, perm_R, W0p}));
   if (W0 == W0p) return POETX_ERR_INVALID_ARG;
+  POETX_TRY(debug_check_perms(stream, {{perm_L, desc->d_out}, {perm_R, desc->d_in}}));
   return permute_cols(desc->dtype, W0, desc->d_in, W0p, desc->d_in, desc->d_out, desc->d_in, perm_R, perm_L, false,
                       stream);
 }
@@ -1296,6 +1343,7 @@ static poetx_status forward_impl(const poetx_desc* desc, int n_tokens, const voi
   if (saved != nullptr && !aligned16(saved)) return POETX_ERR_ALIGNMENT;
   const FwdPlan f = fwd_plan(desc, n_tokens);
   POETX_TRY(check_ws(workspace, ws_bytes, f.total));
+  POETX_TRY(debug_check_perms(stream, {{perm_L, desc->d_out}, {perm_R, desc->d_in}}));
   char* ws = static_cast<char*>(workspace);
   // POET-Xfast keeps Z = V.W0'^T and U = X[:, pi_R] for the backward pass (in `saved`).
   const size_t zbytes = (size_t)n_tokens * desc->d_out * esize(desc->dtype);
@@ -1377,6 +1425,7 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   if (saved != nullptr && !aligned16(saved)) return POETX_ERR_ALIGNMENT;
   const BwdPlan w = bwd_plan(desc, n_tokens);
   POETX_TRY(check_ws(workspace, ws_bytes, w.total));
+  POETX_TRY(debug_check_perms(stream, {{perm_L, desc->d_out}, {perm_R, desc->d_in}}));
   char* ws = static_cast<char*>(workspace);
   const long n = n_tokens;
   const int din = desc->d_in, dout = desc->d_out;
@@ -1631,6 +1680,8 @@ poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, con
   POETX_TRY(check_desc(desc));
   POETX_TRY(check_ptrs({W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P}));
   POETX_TRY(check_ws(workspace, ws_bytes, merge_plan(desc).total));
+  POETX_TRY(debug_check_perms(stream, {{perm_L_old, desc->d_out}, {perm_R_old, desc->d_in},
+                                       {perm_L_new, desc->d_out}, {perm_R_new, desc->d_in}}));
   return merge_impl(desc, W0p, W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P,
                     static_cast<char*>(workspace), stream);
 }

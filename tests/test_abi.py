@@ -156,3 +156,14 @@ def test_xq_host_validation():
     assert L.poetx_xq_dequantize(ctypes.byref(odd), A, A, A, None) == 2
     assert L.poetx_xq_merge(ctypes.byref(good), A, A, A, A, A, A, A, A, A, A, A, 16, None) == 4
     assert L.poetx_xq_merge(ctypes.byref(f32), A, A, A, A, A, A, A, A, A, A, A, 1 << 30, None) == 1
+
+
+def test_check_permutation_on_the_host():
+    import numpy as np
+    P.poetx_check_permutation(np.random.default_rng(0).permutation(1000).astype(np.int32))
+    P.poetx_check_permutation(np.zeros(0, np.int32))  # the bijection of the empty set
+    for bad in ([0, 0, 2], [0, 1, 3], [-1, 0, 1], [2, 1]):
+        with pytest.raises(P.PoetxError):
+            P.poetx_check_permutation(np.array(bad, np.int32))
+    assert P.lib().poetx_check_permutation(None, 3) == 1 and P.lib().poetx_check_permutation(None, 0) == 0
+    assert P.lib().poetx_check_permutation(None, -1) == 1
