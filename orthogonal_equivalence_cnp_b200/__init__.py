@@ -284,7 +284,9 @@ def poetx_check_permutation(perm, n=None):
     bijection of [0, n)."""
     import numpy as np
     if isinstance(perm, int):
-        addr, n = perm, n
+        if n is None:
+            raise ValueError("a raw host address needs its length n")
+        addr = perm
     else:
         arr = np.ascontiguousarray(np.asarray(perm), dtype=np.int32)
         perm, addr, n = arr, arr.ctypes.data, arr.size if n is None else n
