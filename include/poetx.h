@@ -82,28 +82,18 @@ typedef struct {
  * descriptor. */
 size_t poetx_workspace_size(const poetx_desc* desc, int n_tokens);
 
-/* Bytes of the CNP powers that poetx_cnp can keep for poetx_backward: the Horner terms
- * M_j = S + S.M_{j-1} (M_1 = S), j = 1..k, of every block of both sides, bf16.  Keeping them
- * spares the adjoint k-1 of its chained products (the same trade as POET-Xfast's kept
- * activations; replication review, "Summary": the CNP kernel reuses the lower powers).
- * Returns 0 where nothing is kept (F32, b = 512, k = 0, invalid descriptor); then `powers`
- * must be NULL in both calls.  Layout: R side [d_out, k*b] (row z*b+i of block z holds
- * [M_k | ... | M_1] row i), then P side [d_in, k*b]. */
-size_t poetx_cnp_powers_size(const poetx_desc* desc);
-
 /* CNP forward for both sides of one layer (replication review, "Summary": fused
  * Cayley–Neumann series; "Reproducibility & code": k = 3, n_elements = b(b-1)/2).
  *   theta_R  float32 [d_out/b, b(b-1)/2]   packed skew parameters of R's blocks (in)
  *   theta_P  float32 [d_in/b,  b(b-1)/2]   packed skew parameters of P's blocks (in)
  *   Q_R      dtype   [d_out/b, b, b]       Q_i = (I + S_i) Σ_{j<=k} S_i^j, row-major (out)
  *   Q_P      dtype   [d_in/b,  b, b]       (out)
- *   powers   poetx_cnp_powers_size(desc) bytes (out, optional): NULL, or the buffer to pass
- *            to poetx_backward with the same theta.
- * Errors: INVALID_ARG (also: powers given where the size is 0), UNSUPPORTED_SHAPE, ALIGNMENT,
- * WORKSPACE, CUDA. */
+ * For BF16 and b <= 256 the whole computation stays on chip (one launch for both sides, no
+ * workspace is touched); F32 and b = 512 go through the library's GEMM kernels and use the
+ * workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, WORKSPACE, CUDA. */
 poetx_status poetx_cnp(const poetx_desc* desc, const float* theta_R, const float* theta_P,
-                       void* Q_R, void* Q_P, void* powers, void* workspace, size_t ws_bytes,
-                       poetx_stream stream);
+                       void* Q_R, void* Q_P, void* workspace, size_t ws_bytes, poetx_stream stream);
 
 /* CNP forward over a flat batch of n_blocks blocks that share b and k (e.g. every block of
  * every layer of a model in one launch).  Uses desc->b, desc->k, desc->dtype only.
@@ -161,8 +151,6 @@ poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, 
  *   dY dtype [N, d_out], X dtype [N, d_in], W0p, perm_L, perm_R, Q_R, Q_P as in forward (in)
  *   theta_R, theta_P float32 packed (in; the CNP adjoint needs S)
  *   saved   dtype [N*(d_out + d_in)] (in, FAST: as written by poetx_forward) or NULL (MEM)
- *   powers  (in, optional) NULL (the adjoint recomputes the CNP powers) or the buffer that
- *           poetx_cnp filled for these theta
  *   dX dtype [N, d_in] (out); grad_theta_R float32 [d_out/b, b(b-1)/2] (out);
  *   grad_theta_P float32 [d_in/b, b(b-1)/2] (out).
  * The call may order part of its work on a library-owned side stream of the current device;
@@ -173,8 +161,7 @@ poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, 
 poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
                             const void* W0p, const int32_t* perm_L, const int32_t* perm_R,
                             const void* Q_R, const void* Q_P, const float* theta_R,
-                            const float* theta_P, const void* saved, const void* powers,
-                            void* dX, float* grad_theta_R, float* grad_theta_P, void* workspace,
+                            const float* theta_P, const void* saved, void* dX, float* grad_theta_R, float* grad_theta_P, void* workspace,
                             size_t ws_bytes, poetx_stream stream);
 
 /* Merge-then-reinitialise (agidaily.cc article: transforms are merged into the weight and
@@ -204,7 +191,7 @@ poetx_status poetx_merge(const poetx_desc* desc, void* W0p, const void* Q_R, con
  * (UNSUPPORTED_SHAPE otherwise).  The W0' GEMMs of forward and backward read the codes and
  * dequantise each tile in shared memory; no bf16 W0' exists at any time.  Workspace:
  * poetx_workspace_size(desc, n_tokens) covers every call below.  Other arguments and errors
- * as for the bf16 calls above (poetx_xq_backward: no `saved`, no `powers`).
+ * as for the bf16 calls above (poetx_xq_backward: no `saved`).
  *
  * poetx_xq_quantize:   W0p bf16 [d_out, d_in] (in) -> W0q, W0s (out).
  * poetx_xq_dequantize: W0q, W0s (in) -> W0p bf16 (out) = bf16(s_o * q) (for inspection).

@@ -17,7 +17,7 @@ __all__ = [
     "poetx_cnp_blocks_workspace_size", "poetx_absorb", "poetx_forward", "poetx_backward",
     "poetx_merge", "poetx_status_string", "poetx_device_status", "poetx_test_gemm",
     "poetx_launch_count", "poetx_profile_enable", "poetx_profile_summary", "KERNEL_CLASSES",
-    "poetx_cnp_blocks_noalloc", "poetx_cnp_powers_size", "poetx_adamw_cfg", "poetx_adamw_step",
+    "poetx_cnp_blocks_noalloc", "poetx_adamw_cfg", "poetx_adamw_step",
     "poetx_adamw_reset", "poetx_wc_saved_size", "poetx_wc_workspace_size", "poetx_wc_forward", "poetx_wc_backward",
     "poetx_xq_quantize", "poetx_xq_dequantize", "poetx_xq_forward", "poetx_xq_backward", "poetx_xq_merge",
     "poetx_check_permutation",
@@ -69,13 +69,12 @@ _D = ctypes.POINTER(poetx_desc)
 _SIGNATURES = {
     "poetx_workspace_size": (_SZ, [_D, _I]),
     "poetx_cnp_blocks_workspace_size": (_SZ, [_D, _I]),
-    "poetx_cnp_powers_size": (_SZ, [_D]),
-    "poetx_cnp": (_I, [_D, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_cnp": (_I, [_D, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_cnp_blocks": (_I, [_D, _I, _P, _P, _P, _SZ, _P]),
     "poetx_cnp_blocks_noalloc": (_I, [_D, _I, _P, _P, _P]),
     "poetx_absorb": (_I, [_D, _P, _P, _P, _P, _P]),
     "poetx_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
-    "poetx_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_adamw_step": (_I, [ctypes.POINTER(poetx_adamw_cfg), _LL, _I, _P, _P, _P, _P, _P]),
     "poetx_adamw_reset": (_I, [_LL, _P, _P, _P]),
@@ -164,13 +163,9 @@ def poetx_cnp_blocks_workspace_size(desc: poetx_desc, n_blocks: int) -> int:
     return lib().poetx_cnp_blocks_workspace_size(ctypes.byref(desc), n_blocks)
 
 
-def poetx_cnp_powers_size(desc: poetx_desc) -> int:
-    return lib().poetx_cnp_powers_size(ctypes.byref(desc))
-
-
-def poetx_cnp(desc, theta_R, theta_P, Q_R, Q_P, powers, workspace, ws_bytes=None, stream=None):
+def poetx_cnp(desc, theta_R, theta_P, Q_R, Q_P, workspace, ws_bytes=None, stream=None):
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
-    _check(lib().poetx_cnp(ctypes.byref(desc), _ptr(theta_R), _ptr(theta_P), _ptr(Q_R), _ptr(Q_P), _ptr(powers),
+    _check(lib().poetx_cnp(ctypes.byref(desc), _ptr(theta_R), _ptr(theta_P), _ptr(Q_R), _ptr(Q_P),
                            _ptr(workspace), ws_bytes, _stream(stream)), "poetx_cnp")
 
 
@@ -193,12 +188,12 @@ def poetx_forward(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, saved, wo
                                _stream(stream)), "poetx_forward")
 
 
-def poetx_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved, powers, dX,
+def poetx_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved, dX,
                    grad_theta_R, grad_theta_P, workspace, ws_bytes=None, stream=None):
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_backward(ctypes.byref(desc), n_tokens, _ptr(dY), _ptr(X), _ptr(W0p), _ptr(perm_L),
                                 _ptr(perm_R), _ptr(Q_R), _ptr(Q_P), _ptr(theta_R), _ptr(theta_P), _ptr(saved),
-                                _ptr(powers), _ptr(dX), _ptr(grad_theta_R), _ptr(grad_theta_P), _ptr(workspace),
+                                _ptr(dX), _ptr(grad_theta_R), _ptr(grad_theta_P), _ptr(workspace),
                                 ws_bytes, _stream(stream)), "poetx_backward")
 
 

@@ -18,7 +18,7 @@
 #include "elementwise.cuh"
 #include "gemm.cuh"
 #include "sm100.cuh"
-#include "cnp_fused.cuh"
+#include "cnp_onchip.cuh"
 
 using namespace poetx;
 
@@ -717,33 +717,14 @@ poetx_status cnp_bwd_generic(int b, int k, int dt, long nb, const float* theta, 
   return pack(E, nb, b, grad, st);
 }
 
-// ----------------------------------------------------------------- fused CNP (bf16 path)
+// ----------------------------------------------------------------- on-chip CNP (bf16 path)
 // One launch runs the whole CNP forward (or adjoint) of up to two block sets (the R and P sides
-// of a layer) as a cluster program; see cnp_fused.cuh.  Used for bf16 and b <= 256.
-bool cnp_fused_ok(int b, int dt) { return dt == BF16 && b >= 64 && b <= 256; }
-int cnp_bn(int b) { return b >= 128 ? 128 : 64; }
+// of a layer) with every operand on chip; see cnp_onchip.cuh.  Used for bf16 and b <= 256; it
+// needs no global scratch.
+bool cnp_fused_ok(int b, int dt) { return dt == BF16 && (b == 64 || b == 128 || b == 256); }
 
-// Global scratch of the fused programs (per side): the bf16 operands the peer CTAs read.
-size_t cnp_fwd_fused_ws(int b, int k, long nb) {
-  if (k == 0 || nb == 0) return 0;
-  const size_t blk = (size_t)nb * b * b;
-  Plan p;
-  p.take(blk * 2);                                  // S (bf16)
-  if (k >= 2) { p.take(blk * 2); p.take(blk * 2); }  // M_j ping-pong (bf16)
-  return p.total;
-}
-size_t cnp_bwd_fused_ws(int b, int k, long nb) {
-  if (nb == 0) return 0;
-  const size_t blk = (size_t)nb * b * b;
-  Plan p;
-  p.take(blk * 4);  // E = G_S (f32), read transposed by PACK (G itself when k = 0)
-  if (k >= 1) {
-    p.take(blk * 2);               // S (bf16)
-    p.take(blk * (size_t)k * 2);   // A-stack [G | Gbar_k | ... | Gbar_2]
-    p.take(blk * (size_t)k * 2);   // B-stack [M_k | ... | M_1]
-  }
-  return p.total;
-}
+size_t cnp_fwd_fused_ws(int, int, long) { return 0; }
+size_t cnp_bwd_fused_ws(int, int, long) { return 0; }
 
 struct CnpSide {
   long nb = 0;
@@ -752,240 +733,83 @@ struct CnpSide {
   const float* part = nullptr;      // adjoint: split-K partials of G
   int splits = 1;
   float* grad = nullptr;            // adjoint output
-  char* ws = nullptr;               // this side's scratch
-  char* powers = nullptr;           // [nb*b, k*b] bf16 stack [M_k | ... | M_1] kept by the forward (or null)
 };
 
-CnpStageDesc stage_desc(int kind) {
-  CnpStageDesc d;
-  d.kind = kind; d.b_mn = 0; d.c_reg = CNP_NONE; d.alpha1 = 1.f; d.beta1 = 0.f; d.diag1 = 0; d.r1 = CNP_NONE;
-  d.g1_dtype = BF16; d.r2 = CNP_NONE; d.alpha2 = 1.f; d.beta2 = 0.f; d.accum2 = 0;
-  return d;
-}
-
-// Operand maps, K and global output of GEMM stage s for one segment.  A is K-major [rows, lda]
-// (block z at row z*b); B is MN-major (B[n][k] = mem[z*b+k][n]) or K-major (B[n][k] = mem[z*b+n][k]).
-poetx_status set_seg_gemm(CnpProgram& pr, int s, int q, long nb, const void* A, long lda, const void* B, long ldb,
-                          bool b_mn, int K, void* g1, long g1_ld) {
-  const int b = pr.b, BN = cnp_bn(b);
-  GemmDesc g;
-  g.M = b; g.N = b; g.K = K; g.batch = (int)nb;
-  g.A = view(A, nb * b, K, lda, b, 0);
-  g.B = view(B, nb * b, b_mn ? b : K, ldb, b, 0); g.b_mn = b_mn;
-  POETX_TRY(check_gemm(g, BF16));
-  CnpSegStage& G = pr.g[s][q];
-  if (!make_tmap(&G.tmA, g.A, 64, TC_BM)) return POETX_ERR_CUDA;
-  if (!make_tmap(&G.tmB, g.B, 64, b_mn ? 64 : BN)) return POETX_ERR_CUDA;
-  G.K = K; G.a_zrow = b; G.b_zrow = b; G.b_zcol = 0;
-  G.g1 = g1; G.g1_ld = g1_ld;
-  if (g1 && (!aligned16(g1) || g1_ld % 8)) return POETX_ERR_ALIGNMENT;
-  if (g1) {
-    // The stage's output leaves through TMA stores of 32-row boxes (128-byte rows).
-    const bool f32 = pr.st[s].g1_dtype == F32;
-    if (!make_tmap(&G.tmD, view(g1, nb * b, b, g1_ld), f32 ? 32 : 64, 32, f32 ? F32 : BF16)) return POETX_ERR_CUDA;
-  }
-  pr.st[s].b_mn = b_mn ? 1 : 0;
-  return POETX_OK;
-}
-
-static_assert(sizeof(CnpProgram) <= 32764, "the CNP program is passed as one kernel parameter");
-
-template <int BN>
-poetx_status launch_cnp_program(const CnpProgram& pr, long nb_total, cudaStream_t st) {
-  constexpr int ST = 6;  // ring depth: the long-K product of the adjoint (K = k b) streams in two rounds
+template <int B, bool ADJ>
+poetx_status launch_cnp_chip(int k, const CnpSide* sides, int nsides, cudaStream_t st) {
+  using C = ChipCfg<B>;
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return POETX_ERR_CUDA;
-  constexpr size_t smem = cnp_smem_bytes<BN, ST>();
-  auto kern = cnp_program_kernel<BN, ST>;
+  auto kern = cnp_chip_kernel<B, ADJ>;
   if (!attr_done[dev]) {
-    if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
+    if (!set_smem(kern, C::SMEM)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
-  if (nb_total > 65535) return POETX_ERR_UNSUPPORTED_SHAPE;
-  const int b = pr.b, nt = b / BN, mt = (b + TC_BM - 1) / TC_BM;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(nt, mt, (unsigned)nb_total);
-  cfg.blockDim = dim3(CNP_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = nt;
-  attr[0].val.clusterDim.y = mt;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  LaunchScope ls(POETX_KC_CNP_GEMM, st);
-  if (cudaLaunchKernelEx(&cfg, kern, pr) != cudaSuccess) return POETX_ERR_CUDA;
-  return last_launch();
-}
-
-poetx_status run_cnp_program(CnpProgram& pr, long nb_total, cudaStream_t st) {
-  // Store maps of the S copies written by the UNPACK stage (64-column x 32-row bf16 boxes).
-  for (int q = 0; q < pr.nseg; ++q) {
-    CnpSegment& S = pr.seg[q];
-    const long rows = (long)S.nb * pr.b;
-    if (S.Sb0 && !make_tmap(&S.tmS0, view(S.Sb0, rows, pr.b, S.ld0), 64, 32)) return POETX_ERR_CUDA;
-    if (S.Sb1 && !make_tmap(&S.tmS1, view(S.Sb1, rows, pr.b, S.ld1), 64, 32)) return POETX_ERR_CUDA;
-  }
-  return cnp_bn(pr.b) == 128 ? launch_cnp_program<128>(pr, nb_total, st) : launch_cnp_program<64>(pr, nb_total, st);
-}
-
-std::mutex g_cnp_prog_mu;
-CnpProgram g_cnp_prog;  // large; rebuilt on the host for every launch (guarded by the mutex)
-
-// Forward: Q = (I + S)(I + S + ... + S^k) per block by the Horner recursion on M_j = N_j - I:
-//   R1 = S;  M_j = S.M_{j-1} + R1 (bf16 to global);  at j = k also R2 = T = S.M_{k-1} + 2 R1;
-//   Q = S.M_k + R2 + I   (k = 1: Q = S.S + 2 R1 + I;  k = 0: Q = I + S directly).
-poetx_status cnp_fwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaStream_t st) {
-  std::lock_guard<std::mutex> lock(g_cnp_prog_mu);
-  CnpProgram& pr = g_cnp_prog;
-  pr = CnpProgram();
-  pr.b = b;
-  pr.nseg = nsides;
+  CnpChipArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.nseg = nsides;
+  a.k = k;
   long nb_total = 0;
-  for (int q = 0; q < nsides; ++q) nb_total += sides[q].nb;
-  if (nb_total == 0) return POETX_OK;
-  pr.st[0] = stage_desc(CNP_UNPACK);
-  int ns = 1;
-  if (k >= 1) {
-    for (int j = 2; j <= k + 1; ++j, ++ns) {
-      CnpStageDesc d = stage_desc(CNP_GEMM);
-      d.c_reg = CNP_R1;
-      d.beta1 = 1.f;
-      if (j == k && j <= k) { d.r2 = CNP_R2; d.alpha2 = 1.f; d.beta2 = 2.f; }
-      if (j == k + 1) {
-        d.diag1 = 1;
-        if (k == 1) d.beta1 = 2.f; else d.c_reg = CNP_R2;
-      }
-      pr.st[ns] = d;
-    }
-  }
-  pr.nstages = ns;
   for (int q = 0; q < nsides; ++q) {
     const CnpSide& sd = sides[q];
-    CnpSegment& S = pr.seg[q];
-    S.nb = (int)sd.nb;
-    S.theta = sd.theta;
-    S.splits = 1;
-    if (k == 0) {
-      S.no_sreg = 1; S.Sb0 = sd.Q; S.ld0 = b; S.add_identity = 1;
-      continue;
-    }
-    const size_t blk = (size_t)sd.nb * b * b;
-    Plan p;
-    char* Sop = sd.ws + p.take(blk * 2);
-    char* Mbuf[2] = {nullptr, nullptr};
-    if (k >= 2 && sd.powers == nullptr) { Mbuf[0] = sd.ws + p.take(blk * 2); Mbuf[1] = sd.ws + p.take(blk * 2); }
-    const long kb = (long)k * b;
-    // Kept powers: M_j goes to slot k - j of the stack, and M_1 = S is written there once by
-    // the UNPACK stage and read back from there as the A operand of every product.
-    auto slot = [&](int j) { return static_cast<void*>(sd.powers + (size_t)(k - j) * b * 2); };
-    const void* Sa = sd.powers ? slot(1) : Sop;
-    const long lds = sd.powers ? kb : b;
-    S.Sb0 = const_cast<void*>(Sa); S.ld0 = lds;
-    const void* Mprev = Sa;
-    long ldprev = lds;
-    int s = 1;
-    for (int j = 2; j <= k + 1; ++j, ++s) {
-      const bool last = (j == k + 1);
-      void* out = last ? sd.Q : (sd.powers ? slot(j) : Mbuf[j & 1]);
-      const long ldout = (last || !sd.powers) ? b : kb;
-      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sa, lds, Mprev, ldprev, true, b, out, ldout));
-      Mprev = out;
-      ldprev = ldout;
-    }
-  }
-  return run_cnp_program(pr, nb_total, st);
-}
-
-// Adjoint (packed gradients) from the split-K partials of G = dL/dQ, by the Horner adjoint:
-//   G_S = G.N_k^T + sum_{j=1..k} Gbar_j.N_{j-1}^T,  Gbar_k = (I + S^T).G,  Gbar_{j-1} = S^T.Gbar_j,
-//   = E + [G | Gbar_k | ... | Gbar_2] . [M_k | ... | M_1]^T,  E = G + sum_j Gbar_j (f32, in TMEM R3).
-poetx_status cnp_bwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaStream_t st) {
-  std::lock_guard<std::mutex> lock(g_cnp_prog_mu);
-  CnpProgram& pr = g_cnp_prog;
-  pr = CnpProgram();
-  pr.b = b;
-  pr.nseg = nsides;
-  long nb_total = 0;
-  for (int q = 0; q < nsides; ++q) nb_total += sides[q].nb;
-  if (nb_total == 0) return POETX_OK;
-  const long kb = (long)k * b;
-  // The power stages are skipped when the forward kept M_1..M_k (all sides or none).
-  const bool kept = sides[0].powers != nullptr;
-  for (int q = 1; q < nsides; ++q)
-    if ((sides[q].powers != nullptr) != kept) return POETX_ERR_INVALID_ARG;
-  // stage list (same for both segments)
-  int ns = 0;
-  pr.st[ns++] = stage_desc(CNP_REDUCE_UNPACK);
-  if (k >= 1) {
-    for (int j = 2; j <= k && !kept; ++j) {  // M_j = S.M_{j-1} + S
-      CnpStageDesc d = stage_desc(CNP_GEMM);
-      d.c_reg = CNP_R1; d.beta1 = 1.f;
-      pr.st[ns++] = d;
-    }
-    {  // Gbar_k = G - S.G (bf16 out, k >= 2);  E = 2G - S.G
-      CnpStageDesc d = stage_desc(CNP_GEMM);
-      d.c_reg = CNP_R2; d.alpha1 = -1.f; d.beta1 = 1.f;
-      d.r2 = CNP_R3; d.alpha2 = -1.f; d.beta2 = 2.f;
-      pr.st[ns++] = d;
-    }
-    for (int j = k - 1; j >= 1; --j) {  // Gbar_j = -S.Gbar_{j+1};  E += Gbar_j
-      CnpStageDesc d = stage_desc(CNP_GEMM);
-      d.alpha1 = -1.f;
-      d.r2 = CNP_R3; d.alpha2 = -1.f; d.accum2 = 1;
-      pr.st[ns++] = d;
-    }
-    {  // G_S = E + A-stack . B-stack^T  -> global f32
-      CnpStageDesc d = stage_desc(CNP_GEMM);
-      d.c_reg = CNP_R3; d.beta1 = 1.f; d.g1_dtype = F32;
-      pr.st[ns++] = d;
-    }
-  }
-  pr.st[ns++] = stage_desc(CNP_PACK);
-  pr.nstages = ns;
-  for (int q = 0; q < nsides; ++q) {
-    const CnpSide& sd = sides[q];
-    CnpSegment& S = pr.seg[q];
+    CnpChipSide& S = a.seg[q];
     S.nb = (int)sd.nb;
     S.theta = sd.theta;
     S.part = sd.part;
     S.splits = sd.splits;
     S.grad = sd.grad;
-    const size_t blk = (size_t)sd.nb * b * b;
-    Plan p;
-    float* E = reinterpret_cast<float*>(sd.ws + p.take(blk * 4));
-    S.GS = E;
-    if (k == 0) {
-      S.no_sreg = 1; S.G32 = E;
-      continue;
+    nb_total += sd.nb;
+    if (!aligned16(sd.theta)) return POETX_ERR_ALIGNMENT;
+    if (!ADJ) {
+      if (!aligned16(sd.Q)) return POETX_ERR_ALIGNMENT;
+      // Q leaves through TMA stores of (64 columns x rows-per-CTA) boxes.
+      if (!make_tmap(&S.tmQ, view(sd.Q, sd.nb * B, B, B), 64, C::ROWS)) return POETX_ERR_CUDA;
+    } else if (!aligned16(sd.part) || sd.splits < 1) {
+      return POETX_ERR_ALIGNMENT;
     }
-    char* Sop = sd.ws + p.take(blk * 2);
-    char* Ast = sd.ws + p.take(blk * (size_t)k * 2);
-    char* Bst = kept ? sd.powers : sd.ws + p.take(blk * (size_t)k * 2);
-    auto aslot = [&](int t) { return static_cast<void*>(Ast + (size_t)t * b * 2); };
-    auto bslot = [&](int t) { return static_cast<void*>(Bst + (size_t)t * b * 2); };
-    S.Sb0 = Sop; S.ld0 = b;
-    if (kept) {
-      S.no_sreg = 1;  // S in TMEM only feeds the power stages
-    } else {
-      S.Sb1 = bslot(k - 1); S.ld1 = kb;
-    }
-    S.Gb = aslot(0); S.ldg = kb;
-    int s = 1;
-    for (int j = 2; j <= k && !kept; ++j, ++s)
-      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, bslot(k - j + 1), kb, true, b, bslot(k - j), kb));
-    POETX_TRY(set_seg_gemm(pr, s++, q, sd.nb, Sop, b, aslot(0), kb, true, b, k >= 2 ? aslot(1) : nullptr, kb));
-    for (int j = k - 1; j >= 1; --j, ++s)
-      POETX_TRY(set_seg_gemm(pr, s, q, sd.nb, Sop, b, aslot(k - j), kb, true, b, j >= 2 ? aslot(k - j + 1) : nullptr,
-                             kb));
-    POETX_TRY(set_seg_gemm(pr, s++, q, sd.nb, Ast, kb, Bst, kb, false, (int)kb, E, b));
   }
-  return run_cnp_program(pr, nb_total, st);
+  if (nb_total == 0) return POETX_OK;
+  if (nb_total * C::NCTA > 0x7fffffffL) return POETX_ERR_UNSUPPORTED_SHAPE;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nb_total * C::NCTA), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (C::PAIR) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  LaunchScope ls(POETX_KC_CNP_GEMM, st);
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return POETX_ERR_CUDA;
+  return last_launch();
+}
+
+template <bool ADJ>
+poetx_status run_cnp_chip(int b, int k, const CnpSide* sides, int nsides, cudaStream_t st) {
+  if (b == 256) return launch_cnp_chip<256, ADJ>(k, sides, nsides, st);
+  if (b == 128) return launch_cnp_chip<128, ADJ>(k, sides, nsides, st);
+  if (b == 64) return launch_cnp_chip<64, ADJ>(k, sides, nsides, st);
+  return POETX_ERR_UNSUPPORTED_SHAPE;
+}
+
+// Forward: Q of every block of the given sides (one launch).
+poetx_status cnp_fwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaStream_t st) {
+  return run_cnp_chip<false>(b, k, sides, nsides, st);
+}
+// Adjoint: packed gradients from the split-K partials of G = dL/dQ (one launch).
+poetx_status cnp_bwd_fused(int b, int k, const CnpSide* sides, int nsides, cudaStream_t st) {
+  return run_cnp_chip<true>(b, k, sides, nsides, st);
 }
 
 // Scratch of the CNP forward / adjoint for nb blocks (fused path for bf16 and b <= 256).
@@ -999,7 +823,7 @@ size_t cnp_bwd_ws(int b, int k, int dt, long nb) {
 poetx_status cnp_fwd_run(int b, int k, int dt, long nb, const float* theta, void* Q, char* ws, cudaStream_t st) {
   if (!cnp_fused_ok(b, dt)) return cnp_fwd_generic(b, k, dt, nb, theta, Q, ws, st);
   CnpSide sd;
-  sd.nb = nb; sd.theta = theta; sd.Q = Q; sd.ws = ws;
+  sd.nb = nb; sd.theta = theta; sd.Q = Q;
   return cnp_fwd_fused(b, k, &sd, 1, st);
 }
 
@@ -1282,38 +1106,18 @@ poetx_status poetx_cnp_blocks(const poetx_desc* desc, int n_blocks, const float*
   return cnp_fwd_run(desc->b, desc->k, desc->dtype, n_blocks, theta, Q, static_cast<char*>(workspace), stream);
 }
 
-size_t poetx_cnp_powers_size(const poetx_desc* desc) {
-  if (check_desc(desc) != POETX_OK || !cnp_fused_ok(desc->b, desc->dtype) || desc->k < 1) return 0;
-  return (size_t)desc->k * desc->b * ((size_t)desc->d_in + desc->d_out) * 2;
-}
-
-// The kept powers of the R side ([d_out, k*b] bf16), then those of the P side ([d_in, k*b]).
-static void split_powers(const poetx_desc* d, const void* powers, char** pr, char** pp) {
-  char* base = static_cast<char*>(const_cast<void*>(powers));
-  *pr = base;
-  *pp = base ? base + (size_t)d->k * d->b * d->d_out * 2 : nullptr;
-}
-
-static poetx_status check_powers(const poetx_desc* desc, const void* powers) {
-  if (powers == nullptr) return POETX_OK;
-  if (poetx_cnp_powers_size(desc) == 0) return POETX_ERR_INVALID_ARG;
-  return aligned16(powers) ? POETX_OK : POETX_ERR_ALIGNMENT;
-}
-
 poetx_status poetx_cnp(const poetx_desc* desc, const float* theta_R, const float* theta_P, void* Q_R, void* Q_P,
-                       void* powers, void* workspace, size_t ws_bytes, poetx_stream stream) {
+                       void* workspace, size_t ws_bytes, poetx_stream stream) {
   POETX_TRY(check_desc(desc));
   POETX_TRY(check_ptrs({theta_R, theta_P, Q_R, Q_P}));
-  POETX_TRY(check_powers(desc, powers));
   POETX_TRY(check_ws(workspace, ws_bytes, cnp_layer_ws(desc)));
   char* ws = static_cast<char*>(workspace);
   const int b = desc->b;
   const size_t offP = align256(cnp_fwd_ws(b, desc->k, desc->dtype, desc->d_out / b));
   if (cnp_fused_ok(b, desc->dtype)) {
     CnpSide sides[2];
-    sides[0].nb = desc->d_out / b; sides[0].theta = theta_R; sides[0].Q = Q_R; sides[0].ws = ws;
-    sides[1].nb = desc->d_in / b; sides[1].theta = theta_P; sides[1].Q = Q_P; sides[1].ws = ws + offP;
-    split_powers(desc, powers, &sides[0].powers, &sides[1].powers);
+    sides[0].nb = desc->d_out / b; sides[0].theta = theta_R; sides[0].Q = Q_R;
+    sides[1].nb = desc->d_in / b; sides[1].theta = theta_P; sides[1].Q = Q_P;
     return cnp_fwd_fused(b, desc->k, sides, 2, stream);
   }
   POETX_TRY(cnp_fwd_generic(b, desc->k, desc->dtype, desc->d_out / b, theta_R, Q_R, ws, stream));
@@ -1406,10 +1210,9 @@ struct SideJoin {
 static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
                                   const void* W0p, const float* W0s, const int32_t* perm_L, const int32_t* perm_R,
                                   const void* Q_R, const void* Q_P, const float* theta_R, const float* theta_P,
-                                  const void* saved, const void* powers, void* dX, float* grad_theta_R,
+                                  const void* saved, void* dX, float* grad_theta_R,
                                   float* grad_theta_P, void* workspace, size_t ws_bytes, poetx_stream stream) {
   POETX_TRY(check_desc(desc));
-  POETX_TRY(check_powers(desc, powers));
   if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
   if (desc->mode == POETX_FAST && saved == nullptr && n_tokens > 0) return POETX_ERR_INVALID_ARG;
   if (desc->mode == POETX_MEM && saved != nullptr) return POETX_ERR_INVALID_ARG;
@@ -1472,10 +1275,9 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   if (cnp_fused_ok(b, dt)) {
     CnpSide sides[2];
     sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + w.GpR);
-    sides[0].splits = w.sR; sides[0].grad = grad_theta_R; sides[0].ws = ws + w.cnpR;
+    sides[0].splits = w.sR; sides[0].grad = grad_theta_R;
     sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + w.GpP);
-    sides[1].splits = w.sP; sides[1].grad = grad_theta_P; sides[1].ws = ws + w.cnpP;
-    split_powers(desc, powers, &sides[0].powers, &sides[1].powers);
+    sides[1].splits = w.sP; sides[1].grad = grad_theta_P;
     return cnp_bwd_fused(b, desc->k, sides, 2, stream);
   }
   POETX_TRY(cnp_bwd_generic(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + w.GpR), w.sR,
@@ -1486,11 +1288,11 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
 
 poetx_status poetx_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* X, const void* W0p,
                             const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
-                            const float* theta_R, const float* theta_P, const void* saved, const void* powers,
+                            const float* theta_R, const float* theta_P, const void* saved,
                             void* dX, float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
                             poetx_stream stream) {
   return backward_impl(desc, n_tokens, dY, X, W0p, nullptr, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved,
-                       powers, dX, grad_theta_R, grad_theta_P, workspace, ws_bytes, stream);
+                       dX, grad_theta_R, grad_theta_P, workspace, ws_bytes, stream);
 }
 
 size_t poetx_wc_saved_size(const poetx_desc* desc) {
@@ -1608,9 +1410,9 @@ poetx_status poetx_wc_backward(const poetx_desc* desc, int n_tokens, const void*
   if (cnp_fused_ok(b, dt)) {
     CnpSide sides[2];
     sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + m.GpR);
-    sides[0].splits = 1; sides[0].grad = grad_theta_R; sides[0].ws = ws + m.cnpR;
+    sides[0].splits = 1; sides[0].grad = grad_theta_R;
     sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + m.GpP);
-    sides[1].splits = 1; sides[1].grad = grad_theta_P; sides[1].ws = ws + m.cnpP;
+    sides[1].splits = 1; sides[1].grad = grad_theta_P;
     return cnp_bwd_fused(b, desc->k, sides, 2, stream);
   }
   POETX_TRY(cnp_bwd_generic(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + m.GpR), 1, grad_theta_R,
@@ -1744,7 +1546,7 @@ poetx_status poetx_xq_backward(const poetx_desc* desc, int n_tokens, const void*
   POETX_TRY(check_xq(desc));
   POETX_TRY(check_ptrs({W0q, W0s}));
   return backward_impl(desc, n_tokens, dY, X, W0q, W0s, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, nullptr,
-                       nullptr, dX, grad_theta_R, grad_theta_P, workspace, ws_bytes, stream);
+                       dX, grad_theta_R, grad_theta_P, workspace, ws_bytes, stream);
 }
 
 poetx_status poetx_xq_merge(const poetx_desc* desc, int8_t* W0q, float* W0s, const void* Q_R, const void* Q_P,

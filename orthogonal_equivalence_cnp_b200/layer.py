@@ -9,7 +9,7 @@ import numpy as np
 import torch
 
 from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_adamw_cfg, poetx_adamw_reset,
-               poetx_adamw_step, poetx_backward, poetx_cnp, poetx_cnp_powers_size, poetx_desc, poetx_forward,
+               poetx_adamw_step, poetx_backward, poetx_cnp, poetx_desc, poetx_forward,
                poetx_merge, poetx_wc_backward, poetx_wc_forward, poetx_wc_saved_size, poetx_wc_workspace_size,
                poetx_workspace_size, poetx_xq_backward, poetx_xq_forward, poetx_xq_merge, poetx_xq_quantize)
 
@@ -49,9 +49,6 @@ class PoetxLayer:
         self.Y = torch.empty(self.n, dout, dtype=dt, device=dev)
         # POET-Xfast keeps Z [N, d_out] and U = X[:, pi_R] [N, d_in] for the backward pass.
         self.saved = torch.empty(self.n * (dout + din), dtype=dt, device=dev) if desc.mode == POETX_FAST else None
-        # POET-Xfast also keeps the CNP powers M_1..M_k for the adjoint (where the library keeps any).
-        pw = poetx_cnp_powers_size(desc) if desc.mode == POETX_FAST else 0
-        self.powers = torch.empty(pw, dtype=torch.uint8, device=dev) if pw else None
         self.dX = torch.empty(self.n, din, dtype=dt, device=dev)
         self.grad = torch.zeros_like(self.theta)
         self.g_R, self.g_P = self.grad[:nbo], self.grad[nbo:]
@@ -78,7 +75,7 @@ class PoetxLayer:
 
     # ------------------------------------------------------------------------- the step
     def cnp(self):
-        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.powers, self.ws)
+        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.ws)
 
     def forward(self, X: torch.Tensor):
         if self.xq:
@@ -95,7 +92,7 @@ class PoetxLayer:
                               self.Q_P, self.theta_R, self.theta_P, self.dX, self.g_R, self.g_P, self.ws)
         else:
             poetx_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
-                           self.theta_R, self.theta_P, self.saved, self.powers, self.dX, self.g_R, self.g_P, self.ws)
+                           self.theta_R, self.theta_P, self.saved, self.dX, self.g_R, self.g_P, self.ws)
         return self.dX, self.g_R, self.g_P
 
     def quantize(self):

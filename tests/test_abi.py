@@ -51,24 +51,25 @@ def test_invalid_descriptors_rejected(kw, code):
     assert P.poetx_workspace_size(d, 64) == 0
     L = P.lib()
     fake = 1 << 20  # aligned, never dereferenced: validation fails first
-    st = L.poetx_cnp(ctypes.byref(d), fake, fake, fake, fake, None, fake, 1 << 30, None)
+    st = L.poetx_cnp(ctypes.byref(d), fake, fake, fake, fake, fake, 1 << 30, None)
     assert st == code
 
 
-def test_kept_powers_size_and_validation():
-    bf = _desc(d_in=512, d_out=768, b=256, dtype=P.POETX_BF16)
-    assert P.poetx_cnp_powers_size(bf) == 3 * 256 * (512 + 768) * 2
-    # nothing is kept for fp32, b = 512 or k = 0: a powers buffer is then an argument error
-    f32, b512, k0 = _desc(), _desc(d_in=1024, d_out=512, b=512, dtype=P.POETX_BF16), _desc(dtype=P.POETX_BF16, b=64, k=0)
-    assert P.poetx_cnp_powers_size(f32) == P.poetx_cnp_powers_size(b512) == P.poetx_cnp_powers_size(k0) == 0
+def test_onchip_cnp_needs_no_workspace_and_checks_alignment():
+    # bf16 with b <= 256: the CNP forward and adjoint run on chip (no scratch); fp32 and b = 512
+    # run through the GEMM kernels and need scratch.
+    for b in (64, 128, 256):
+        d = _desc(d_in=512, d_out=768, b=b, dtype=P.POETX_BF16)
+        assert P.poetx_cnp_blocks_workspace_size(d, 1000) == 0
+    assert P.poetx_cnp_blocks_workspace_size(_desc(d_in=1024, d_out=512, b=512, dtype=P.POETX_BF16), 4) > 0
+    assert P.poetx_cnp_blocks_workspace_size(_desc(), 4) > 0
     L = P.lib()
     A = 1 << 20
-    ws = P.poetx_workspace_size(f32, 8)
-    assert L.poetx_cnp(ctypes.byref(f32), A, A, A, A, A, A, ws, None) == 1
-    assert L.poetx_backward(ctypes.byref(f32), 8, A, A, A, A, A, A, A, A, A, A, A, A, A, A, A, ws, None) == 1
+    bf = _desc(d_in=512, d_out=768, b=256, dtype=P.POETX_BF16)
     ws = P.poetx_workspace_size(bf, 8)
-    assert L.poetx_cnp(ctypes.byref(bf), A, A, A, A, A + 8, A, ws, None) == 3
-    assert L.poetx_backward(ctypes.byref(bf), 8, A, A, A, A, A, A, A, A, A, A, A + 8, A, A, A, A, ws, None) == 3
+    assert L.poetx_cnp(ctypes.byref(bf), A, A, A + 8, A, A, ws, None) == 3
+    assert L.poetx_cnp(ctypes.byref(bf), A, None, A, A, A, ws, None) == 1
+    assert L.poetx_cnp_blocks(ctypes.byref(bf), 3, A + 4, A, None, 0, None) == 3
 
 
 def test_null_misaligned_and_workspace_errors():
@@ -104,7 +105,6 @@ def test_workspace_grows_with_tokens_and_mem_mode():
     assert 0 < a < b
     dm = _desc(d_in=4096, d_out=4096, b=256, dtype=P.POETX_BF16, mode=P.POETX_MEM)
     assert P.poetx_workspace_size(dm, 2048) > b
-    assert P.poetx_cnp_blocks_workspace_size(d, 10240) > 0
 
 
 def test_gemm_hook_rejects_out_of_range_views():
