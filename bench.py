@@ -55,9 +55,9 @@ def step_flops(s: I.LayerShape) -> dict:
     return {"fwd": fwd, "bwd": bwd, "cnp": cnp, "total": fwd + bwd + cnp}
 
 
-# DRAM bytes (read + write) of one W0' launch, from the ncu capture summarised in
-# profiles/gemm_w256_bf16_2048x4096x4096_b256_traffic.md (bench workload, mean of two forward and
-# two adjoint launches).  Only valid for that workload and that kernel build; None otherwise.
+# DRAM bytes (read + write) of one W0' launch, from one ncu capture of this kernel build on the
+# bench workload (mean of two forward and two adjoint launches).  Only valid for that workload
+# and that kernel build; None otherwise.
 W_GEMM_TRAFFIC = {"llama8b_attn_4096_b256_bf16": 52.469e6 + 0.750e6}
 
 
@@ -533,6 +533,20 @@ def run_poetx(args):
     achieved = w_gemm_flops(s) / (w_avg_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
     total_prof_ms = sum(v[1] for v in prof.values())
+    # The CNP against HBM: algorithmic bytes per launch (forward: theta read, bf16 Q written;
+    # adjoint: G = dL/dQ read as fp32, theta read, packed gradients written).
+    nbt, Pk = s.nb_in + s.nb_out, s.b * (s.b - 1) // 2
+    cnp_bytes = {"cnp_gemm": nbt * (4 * Pk + 2 * s.b * s.b), "cnp_adj": nbt * (4 * s.b * s.b + 8 * Pk)}
+    cnp = {}
+    for cls, tag in (("cnp_gemm", "fwd"), ("cnp_adj", "adj")):
+        n_c, ms_c = prof.get(cls, (0, 0.0))
+        if n_c:
+            us = 1e3 * ms_c / n_c
+            cnp[f"{tag}_us"] = round(us, 2)
+            cnp[f"{tag}_bytes"] = cnp_bytes[cls]
+            cnp[f"{tag}_hbm_frac"] = round(cnp_bytes[cls] / (us * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 4)
+    cnp["note"] = ("per-launch CUDA-event times inside the replayed step; algorithmic bytes; both sides of the "
+                   "layer in one launch each")
     out = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -561,7 +575,7 @@ def run_poetx(args):
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": W_GEMM_TRAFFIC.get(args.workload),
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean of two forward and "
-                                       "two adjoint launches (profiles/gemm_w256_bf16_2048x4096x4096_b256_traffic.md)",
+                                       "two adjoint launches of this kernel build on this workload",
                      "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                      "frac_of_sustained": round(achieved / float(peaks["bf16_tflops_sustained"]), 4),
                      "launch_ms": round(w_avg_ms, 4), "launches": wcnt,
@@ -570,6 +584,7 @@ def run_poetx(args):
                      "forward_frac": round(w_gemm_flops(s) / (fms / max(fcnt, 1) / 1e3) / 1e12 / peak, 4)},
         "step_roofline": {"t_flop_us": round(fl["total"] / (peak * 1e12) * 1e6, 1),
                           "frac": round((fl["total"] / (peak * 1e12)) / (t_ms / K / 1e3), 4)},
+        "cnp": cnp,
         "kernel_share": {k: round(v[1] / total_prof_ms, 4) for k, v in prof.items() if v[0]},
         "kernel_ms_per_step": {k: round(v[1] / K, 4) for k, v in prof.items() if v[0]},
         "gpu_launches": int(launches),
@@ -590,9 +605,10 @@ def run_poetx(args):
         "e2e": {"value": round(world * s.n_tokens * Ke / (te_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(te_ms / Ke, 4),
-                "protocol": "pinned X, dY in and packed theta gradients out every step; copies on their "
-                            "own streams overlap the previous/next step; L2 flushed before every step "
-                            "inside the interval"},
+                "protocol": "pinned X, dY in and packed theta gradients out every step; Y and dX stay "
+                            "on the device (a training loop hands them to the neighbouring layers there); "
+                            "copies on their own streams overlap the previous/next step; L2 flushed before "
+                            "every step inside the interval"},
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -145,6 +145,17 @@ poetx_status poetx_forward(const poetx_desc* desc, int n_tokens, const void* X, 
                            const void* Q_P, void* Y, void* saved, void* workspace,
                            size_t ws_bytes, poetx_stream stream);
 
+/* poetx_cnp followed by poetx_forward in one call, with the same arguments and results (theta
+ * in, Q_R and Q_P out, then the forward pass with those Q).  The CNP of both sides may run on a
+ * library-owned side stream of the current device beside the input gather of the forward pass,
+ * which does not need Q; everything is complete when `stream` reaches the end of the call (also
+ * under stream capture).  Workspace: poetx_workspace_size(desc, n_tokens) bytes.  Errors as for
+ * the two calls. */
+poetx_status poetx_cnp_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                               const int32_t* perm_L, const int32_t* perm_R, const float* theta_R,
+                               const float* theta_P, void* Q_R, void* Q_P, void* Y, void* saved,
+                               void* workspace, size_t ws_bytes, poetx_stream stream);
+
 /* Backward pass: dX and the gradients w.r.t. the PACKED skew parameters (only the packed form
  * is written; replication review, "Summary": compact skew storage; W0 is frozen, so there is
  * no dW0).  In POETX_MEM mode `saved` must be NULL and U, V, Z are recomputed from X.
@@ -295,14 +306,15 @@ typedef enum {
   POETX_KC_W_GEMM = 0,       /* Z = V W0'^T (tensor cores; with BD_R fused for b = 256)     */
   POETX_KC_BD_GEMM = 1,      /* block-diagonal products BD_P, BD_R and their adjoints       */
   POETX_KC_GRAD_GEMM = 2,    /* per-block gradient products G = dY'^T Z, dV^T U (split-K)   */
-  POETX_KC_CNP_GEMM = 3,     /* Cayley-Neumann power products (forward and adjoint)         */
+  POETX_KC_CNP_GEMM = 3,     /* CNP forward (the on-chip kernel, or its products for F32 / b = 512) */
   POETX_KC_MERGE_GEMM = 4,   /* BD_R W0' BD_P of the merge                                  */
   POETX_KC_PERMUTE = 5,      /* feature-dimension gather / scatter                          */
   POETX_KC_ELEMENTWISE = 6,  /* unpack, pack, split-K reduction, permutation inverse        */
   POETX_KC_TEST_GEMM = 7,    /* poetx_test_gemm                                              */
   POETX_KC_OPTIMIZER = 8,    /* poetx_adamw_step                                             */
   POETX_KC_W_GEMM_ADJ = 9,   /* dV = dZ W0' (with the BD_P adjoint fused for b = 256)        */
-  POETX_KC_COUNT = 10
+  POETX_KC_CNP_ADJ = 10,     /* CNP adjoint to the packed gradients (on-chip, or its products) */
+  POETX_KC_COUNT = 11
 } poetx_kernel_class;
 
 /* Number of kernels this library has launched in the process so far. */

@@ -35,6 +35,15 @@ poetx_status poetx_test_gemm(int dtype, int M, int N, int K, int batch, int spli
                              long long c_ld, long long c_zrow, long long c_zcol, int diag,
                              poetx_stream stream);
 
+/* Failure-detection probe (the bounded device-side waits of every kernel; no GPU fault is
+ * involved).  Launches one CTA that waits on a shared-memory mbarrier nothing arrives on, with the
+ * wait bounded by limit_ns nanoseconds of the device's global timer (1 us .. 100 ms).  The wait
+ * runs out, the kernel records a device timeout (poetx_device_status() then returns
+ * POETX_ERR_DEVICE_TIMEOUT with detail (7 << 8) | 1) and writes 2 to *returned (a device int;
+ * 1 would mean that the wait completed).  Errors: INVALID_ARG (NULL, limit out of range),
+ * ALIGNMENT, CUDA. */
+poetx_status poetx_test_wait_timeout(long long limit_ns, int* returned, poetx_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

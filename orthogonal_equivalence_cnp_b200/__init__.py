@@ -20,7 +20,7 @@ __all__ = [
     "poetx_cnp_blocks_noalloc", "poetx_adamw_cfg", "poetx_adamw_step",
     "poetx_adamw_reset", "poetx_wc_saved_size", "poetx_wc_workspace_size", "poetx_wc_forward", "poetx_wc_backward",
     "poetx_xq_quantize", "poetx_xq_dequantize", "poetx_xq_forward", "poetx_xq_backward", "poetx_xq_merge",
-    "poetx_check_permutation",
+    "poetx_check_permutation", "poetx_test_wait_timeout", "poetx_cnp_forward",
 ]
 
 POETX_F32, POETX_BF16 = 0, 1
@@ -31,7 +31,7 @@ STATUS = {
 }
 
 KERNEL_CLASSES = ["w_gemm", "bd_gemm", "grad_gemm", "cnp_gemm", "merge_gemm", "permute", "elementwise", "test_gemm",
-                  "optimizer", "w_gemm_adj"]
+                  "optimizer", "w_gemm_adj", "cnp_adj"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -74,6 +74,7 @@ _SIGNATURES = {
     "poetx_cnp_blocks_noalloc": (_I, [_D, _I, _P, _P, _P]),
     "poetx_absorb": (_I, [_D, _P, _P, _P, _P, _P]),
     "poetx_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_cnp_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_adamw_step": (_I, [ctypes.POINTER(poetx_adamw_cfg), _LL, _I, _P, _P, _P, _P, _P]),
@@ -88,6 +89,7 @@ _SIGNATURES = {
     "poetx_xq_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_xq_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_check_permutation": (_I, [_P, _I]),
+    "poetx_test_wait_timeout": (_I, [_LL, _P, _P]),
     "poetx_status_string": (ctypes.c_char_p, [_I]),
     "poetx_device_status": (_I, [ctypes.POINTER(ctypes.c_int)]),
     "poetx_launch_count": (ctypes.c_ulonglong, []),
@@ -186,6 +188,14 @@ def poetx_forward(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, saved, wo
     _check(lib().poetx_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0p), _ptr(perm_L), _ptr(perm_R),
                                _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(saved), _ptr(workspace), ws_bytes,
                                _stream(stream)), "poetx_forward")
+
+
+def poetx_cnp_forward(desc, n_tokens, X, W0p, perm_L, perm_R, theta_R, theta_P, Q_R, Q_P, Y, saved, workspace,
+                      ws_bytes=None, stream=None):
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_cnp_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0p), _ptr(perm_L), _ptr(perm_R),
+                                   _ptr(theta_R), _ptr(theta_P), _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(saved),
+                                   _ptr(workspace), ws_bytes, _stream(stream)), "poetx_cnp_forward")
 
 
 def poetx_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved, dX,
@@ -326,3 +336,7 @@ def poetx_cnp_blocks_noalloc(desc, n_blocks, theta, Q, stream=None):
     """CNP forward that takes no workspace (built-in 32 MiB device scratch; see include/poetx.h)."""
     _check(lib().poetx_cnp_blocks_noalloc(ctypes.byref(desc), n_blocks, _ptr(theta), _ptr(Q), _stream(stream)),
            "poetx_cnp_blocks_noalloc")
+
+
+def poetx_test_wait_timeout(limit_ns, returned, stream=None):
+    _check(lib().poetx_test_wait_timeout(int(limit_ns), _ptr(returned), _stream(stream)), "poetx_test_wait_timeout")

@@ -42,6 +42,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "elementwise.cuh"
 #include "gemm.cuh"
 #include "sm100.cuh"
 
@@ -60,22 +61,43 @@ struct ChipCfg {
   static constexpr uint32_t REG = (B / 64) * ATOM; // one operand buffer
   static constexpr uint32_t BFORM_ATOM = B * 128;  // one 64-column atom of a B-form buffer (b rows)
   static constexpr int TCOLS = 2 * B;              // TMEM: ACC [0, b), REG2 [b, 2b)
-  static constexpr int PITCH = B + 1;              // transposed-tile pitch of PACK (floats)
-  static constexpr size_t SMEM = 3 * (size_t)REG + 1024 + 256;
+  static constexpr uint32_t GBOX = ROWS * 128;     // G staging: one 32-column fp32 box of this CTA's rows
+  static constexpr int QN = PAIR ? 128 : B;        // PACK quadrant: QN x QN fp32, rows at QPITCH floats
+  static constexpr int QPITCH = QN + 4;
+  static constexpr size_t BAR_OFF = 3 * (size_t)REG;
+  static constexpr size_t SMEM = BAR_OFF + 256 + 1024;
+  static_assert((size_t)(B / 32) * GBOX <= 2 * (size_t)REG, "G staging fits V1 + V2");
   static_assert((size_t)B * (B - 1) / 2 * 4 <= 2 * (size_t)REG, "theta staging fits V1 + V2");
-  static_assert((size_t)ROWS * PITCH * 4 <= 3 * (size_t)REG, "PACK tile fits the operand buffers");
+  static_assert((size_t)(PAIR ? 2 : 1) * QN * QPITCH * 4 <= BAR_OFF, "PACK quadrants fit below the barriers");
 };
 
 struct CnpChipSide {
   CUtensorMap tmQ;      // forward: store map of Q [nb*b, b] bf16, 128-byte swizzle, box 64 x rows
+  CUtensorMap tmG;      // adjoint: load map of the partials [splits*nb*b, b] fp32, 128-byte swizzle,
+                        //          box 32 x rows
   const float* theta;   // [nb, b(b-1)/2]
   const float* part;    // adjoint: split-K partials of G = dL/dQ, [splits][nb*b][b] fp32
   float* grad;          // adjoint: packed gradients [nb, b(b-1)/2]
   int nb;
   int splits;
 };
+// Spare blocks of a forward launch: the blocks past the CNP ones permute the columns of a bf16
+// row-major array (the input gather U = X[:, pi_R] of the layer), as permute_cols_bulk_kernel
+// does, on the SMs the CNP leaves free.
+struct CnpGather {
+  const uint16_t* in;
+  long ld_in;
+  uint16_t* out;
+  long ld_out;
+  long rows;
+  const int32_t* colmap;
+  int cols;
+  int nblk;  // number of spare blocks (0: none)
+};
 struct CnpChipArgs {
   CnpChipSide seg[2];
+  CnpGather gather;
+  int ncnp;  // blocks of the CNP proper; blocks from ncnp on run the gather
   int nseg;
   int k;
 };
@@ -99,13 +121,25 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
   using C = ChipCfg<B>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned start, derived by pointer arithmetic so that every pointer below stays in
+  // the shared address space (32-bit shared loads instead of generic ones).
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t s0 = smem_u32(smem);
   const uint32_t SC = s0, V1 = s0 + C::REG, V2 = s0 + 2 * C::REG;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 3 * C::REG);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   const uint32_t bar_mma = smem_u32(bars), bar_ready = smem_u32(bars + 1), bar_theta = smem_u32(bars + 2);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 4);
+  const uint32_t bar_g = smem_u32(bars + 3);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 5);
 
+  if constexpr (!ADJ) {
+    if ((int)blockIdx.x >= args.ncnp) {  // a spare block: gather rows (whole clusters, no TMEM)
+      griddep_wait();
+      const CnpGather& G = args.gather;
+      permute_cols_bulk_body<4>(smem, (long)blockIdx.x - args.ncnp, G.nblk, G.in, G.ld_in, G.out, G.ld_out, G.rows,
+                                G.cols, G.colmap, nullptr, 0);
+      return;
+    }
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3, half = warp >> 2;
   const int c = C::PAIR ? (int)cluster_ctarank() : 0;
@@ -127,6 +161,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     mbar_init(bar_mma, 1);
     mbar_init(bar_ready, 8 * C::NCTA);
     mbar_init(bar_theta, 1);
+    mbar_init(bar_g, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -185,8 +220,11 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     }
     ready_phase ^= 1u;
   };
+  // Every wait ends in a full-warp vote, so that the warp is converged (and agrees on `ok`)
+  // before the warp-collective TMEM accesses that follow.
   auto wait_mma = [&](int site) {
     if (ok) ok = mbar_wait(bar_mma, mma_phase, KID_CNP_CHIP, site);
+    ok = __all_sync(0xffffffffu, ok);
     mma_phase ^= 1u;
     tc_fence_after();
   };
@@ -223,7 +261,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
 #pragma unroll 1
       for (int a = 0; a < B / 64; ++a) tma_store_2d(&SD.tmQ, V2 + (uint32_t)a * C::ATOM, 64 * a, (int)(z * B + rbase));
       bulk_commit();
-      bulk_wait<0>();
+      bulk_wait_read<0>();  // the staging may be released; the stores complete with the grid
     }
   };
 
@@ -240,18 +278,38 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
         bulk_load_1d(V1 + off, reinterpret_cast<const char*>(SD.theta + z * P) + off, min(chunk, bytes - off), bar_theta);
     }
     if (ok) ok = mbar_wait(bar_theta, 0, KID_CNP_CHIP, 1);
+    ok = __all_sync(0xffffffffu, ok);
     const float* th = reinterpret_cast<const float*>(smem + C::REG);
     const int roi = ro(i);
+    const int iw = rbase + quarter * 32;  // first row of this warp: chunks are warp-uniform
 #pragma unroll 1
     for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
       float v[32];
+      if (!valid) {
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        const int j = j0 + u;
-        // one unconditional shared load per element (element 0 where nothing is read)
-        const int idx = (!valid || j == i) ? 0 : (j > i ? roi + j : ro(j) + i);
-        const float x = th[idx];
-        v[u] = (!valid || j == i) ? 0.f : (j > i ? x : -x);
+        for (int u = 0; u < 32; ++u) v[u] = 0.f;
+      } else if (j0 >= iw + 32) {
+        // above the diagonal for every lane: S[i][j] = theta[p(i, j)], contiguous in j
+        const float* src = th + roi + j0;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = src[u];
+      } else if (j0 + 32 <= iw) {
+        // below it: S[i][j] = -theta[p(j, i)]; p(j, i) = ro(j) + i with ro(j+1) = ro(j) + b - 2 - j
+        const float* src = th + ro(j0) + i;
+        const int step0 = B - 2 - j0;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = -src[u * step0 - (u * (u - 1)) / 2];
+      } else {
+        // the warp's diagonal block
+        const int roj0 = ro(j0);
+        const int step0 = B - 2 - j0;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int j = j0 + u;
+          const int idx = j > i ? roi + j : (j < i ? roj0 + u * step0 - (u * (u - 1)) / 2 + i : 0);
+          const float x = th[idx];
+          v[u] = j > i ? x : (j < i ? -x : 0.f);
+        }
       }
       chip_put_aform(SC, r, j0, v);
       if constexpr (!ADJ) tst(REG2 + j0, v);
@@ -327,29 +385,53 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------------------- adjoint
-    // Every CTA of the cluster has read its theta staging before V1 / V2 are written (the peer
-    // writes into this CTA's V2).
+    // G = sum of the split-K partials -> REG2 (fp32).  Each partial's rows of this CTA arrive as
+    // b/32 TMA boxes (32 columns x rows, 128-byte swizzle: the 16-byte chunk q of row r sits at
+    // position q ^ (r % 8)), one round per partial, so that every thread then reads its own row
+    // with conflict-free 16-byte loads.  The staging overlaps V1 / V2 (and the theta staging):
+    // every CTA of the cluster has finished its theta reads before the first round starts.
     if constexpr (C::PAIR) cluster_sync_all(); else __syncthreads();
-    const long sstride = (long)SD.nb * B * B;
 #pragma unroll 1
-    for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
-      float g[32];
+    for (int sp = 0; sp < SD.splits; ++sp) {
+      if (sp > 0) __syncthreads();  // every thread has read the previous round
+      if (threadIdx.x == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar_g, (uint32_t)(C::ROWS * B * 4));
+#pragma unroll 1
+        for (int a = 0; a < B / 32; ++a)
+          tma_load_2d(V1 + (uint32_t)a * C::GBOX, &SD.tmG, bar_g, 32 * a, (int)(((long)sp * SD.nb + z) * B + rbase));
+      }
+      if (ok) ok = mbar_wait(bar_g, (uint32_t)(sp & 1), KID_CNP_CHIP, 10);
+      ok = __all_sync(0xffffffffu, ok);
+#pragma unroll 1
+      for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
+        float g[32];
+        if (sp > 0) tld(REG2 + j0, g);
+        const uint8_t* row = smem + C::REG + (j0 / 32) * C::GBOX + r * 128;
 #pragma unroll
-      for (int u = 0; u < 32; ++u) g[u] = 0.f;
-      if (valid) {
-        for (int sp = 0; sp < SD.splits; ++sp) {
-          const float4* src = reinterpret_cast<const float4*>(SD.part + sp * sstride + (z * B + i) * B + j0);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 f = __ldg(src + u);
+        for (int u = 0; u < 8; ++u) {
+          const float4 f = valid ? *reinterpret_cast<const float4*>(row + ((u ^ (r & 7)) * 16))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+          if (sp > 0) {
             g[4 * u] += f.x; g[4 * u + 1] += f.y; g[4 * u + 2] += f.z; g[4 * u + 3] += f.w;
+          } else {
+            g[4 * u] = f.x; g[4 * u + 1] = f.y; g[4 * u + 2] = f.z; g[4 * u + 3] = f.w;
           }
         }
+        tst(REG2 + j0, g);
       }
-      tst(REG2 + j0, g);
-      if (k >= 1) {
-        chip_put_aform(V1, r, j0, g);  // R_k = G
-        if (valid) put_bform(V2, j0, g);  // L_k = G
+      tmem_wait_st();
+    }
+    // R_k = G (A form in V1) and L_k = G (B form in V2, the peer's quadrant in the peer): every
+    // CTA of the cluster has finished reading its G staging.
+    if constexpr (C::PAIR) cluster_sync_all(); else __syncthreads();
+    if (k >= 1) {
+#pragma unroll 1
+      for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
+        float g[32];
+        tld(REG2 + j0, g);
+        chip_put_aform(V1, r, j0, g);
+        if (valid) put_bform(V2, j0, g);
       }
     }
     uint32_t fcol = REG2;  // the TMEM columns holding G_S for PACK
@@ -387,46 +469,56 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     }
     griddep_launch();
     // ---------------------------------------------------------------------------- PACK
-    // TT[i - rbase][j] = G_S[j][i] for this CTA's rows i and every j (pitch b + 1 floats).  A pair's
-    // CTA 1 also sends CTA 0 the quadrant G_S[O_1][O_0]; CTA 0 keeps G_S[O_0][O_1] to itself
-    // (CTA 1's packed rows only reach columns of O_1).
+    // g[p(i,j)] = G_S[i][j] - G_S[j][i] for i < j, computed by the thread that owns row j of G_S
+    // (it holds G_S[j][i] in TMEM) from a row-major copy of the rows i in shared memory, so that
+    // each packed row p(i, .) leaves as coalesced stores along j.  Quadrants (QN x QN, rows of
+    // QPITCH floats, written with 16-byte stores): Qd = G_S[O_c][O_c] of this CTA; for a pair,
+    // CTA 1 also receives Qx = G_S[O_0][O_1] from CTA 0 and handles the packed entries of that
+    // quadrant (rows i in O_0, columns j in O_1).
     {
-      const int ct = C::PAIR ? c0 / 128 : 0;
-      const bool send = !(C::PAIR && c == 0 && ct == 1) && valid;
-      const uint32_t tt = (C::PAIR && ct != c) ? mapa_shared(s0, (uint32_t)ct) : s0;
+      const uint32_t QD = s0, QX = s0 + (uint32_t)(C::QN * C::QPITCH * 4);
+      const int own0 = C::PAIR ? 128 * c : 0;  // first column of this CTA's own quadrant
+      const bool own_cols = !C::PAIR || half == c;
+      const bool to_peer = C::PAIR && c == 0 && half == 1;  // G_S[O_0][O_1] -> CTA 1's Qx
+      uint32_t dst = 0;
+      if (own_cols) dst = QD + (uint32_t)(r * C::QPITCH * 4);
+      if (to_peer) dst = mapa_shared(QX + (uint32_t)(r * C::QPITCH * 4), 1);
 #pragma unroll 1
       for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
         float f[32];
         tld(fcol + j0, f);
-        if (send) {
+        if (valid && (own_cols || to_peer)) {
+          const uint32_t at = dst + (uint32_t)((j0 - (own_cols ? own0 : 128)) * 4);
 #pragma unroll
-          for (int u = 0; u < 32; ++u)
-            st_cluster_f32(tt + (uint32_t)(((j0 + u - 128 * ct) * C::PITCH + i) * 4), f[u]);
+          for (int u = 0; u < 8; ++u)
+            st_cluster_v4(at + 16 * u, make_uint4(__float_as_uint(f[4 * u]), __float_as_uint(f[4 * u + 1]),
+                                                  __float_as_uint(f[4 * u + 2]), __float_as_uint(f[4 * u + 3])));
         }
       }
-    }
-    if constexpr (C::PAIR) cluster_sync_all(); else __syncthreads();
-    float* TT = reinterpret_cast<float*>(smem);
+      if constexpr (C::PAIR) cluster_sync_all(); else __syncthreads();
+      // Thread (row j, half h): the entries (i, j) with i < j and i in the columns of its half.
+      // The TMEM loads are warp-collective: the chunk loop runs to the warp's first row (the
+      // same bound for every lane) and the per-entry test i < j only guards the stores.
+      const int j = i;
+      const bool diag = !C::PAIR || half == c;            // i in O_c: quadrant Qd
+      const bool cross = C::PAIR && c == 1 && half == 0;  // i in O_0, j in O_1: quadrant Qx
+      if (diag || cross) {
+        const float* Q = reinterpret_cast<const float*>(smem + (diag ? 0 : C::QN * C::QPITCH * 4));
+        const int jq = j - own0;                  // column of j in the quadrant
+        const int qrow0 = diag ? own0 : 0;        // block row of the quadrant's first row
+        const int jwarp = rbase + quarter * 32;   // first row of this warp
+        const bool store = ok && valid;
+        float* out = SD.grad + z * P;
 #pragma unroll 1
-    for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
-      float f[32];
-      tld(fcol + j0, f);
-      if (valid) {
+        for (int i0 = c0; i0 < c0 + C::HALF && i0 <= jwarp; i0 += 32) {
+          float f[32];
+          tld(fcol + i0, f);  // G_S[j][i0 .. i0 + 31]
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const int j = j0 + u;
-          if (j > i) TT[r * C::PITCH + j] = f[u] - TT[r * C::PITCH + j];
+          for (int u = 0; u < 32; ++u) {
+            const int ii = i0 + u;
+            if (store && ii < j) out[ro(ii) + j] = Q[(ii - qrow0) * C::QPITCH + jq] - f[u];
+          }
         }
-      }
-    }
-    __syncthreads();
-    if (ok) {
-      float* out = SD.grad + z * P;
-#pragma unroll 1
-      for (int rr = warp; rr < C::ROWS; rr += 8) {
-        const int ii = rbase + rr;
-        const int base = ro(ii);
-        for (int j = ii + 1 + lane; j < B; j += 32) out[base + j] = TT[rr * C::PITCH + j];
       }
     }
   }

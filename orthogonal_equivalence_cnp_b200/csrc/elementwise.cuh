@@ -173,14 +173,16 @@ __host__ __device__ constexpr size_t permute_bulk_smem_bytes(int cols) {
          + 64;                               // two mbarriers (+ padding)
 }
 
+// The body of the kernel below as a device function: block `bid` of `nblk` blocks (256 threads)
+// permutes its share of the row groups, staging in `smem_bulk` (permute_bulk_smem_bytes<ROWS>(cols)
+// bytes, 128-byte aligned).  It also serves the spare blocks of a CNP launch (cnp_onchip.cuh).
 template <int ROWS>
-__global__ void __launch_bounds__(256, 2)
-    permute_cols_bulk_kernel(const uint16_t* __restrict__ in, long ld_in, uint16_t* __restrict__ out, long ld_out,
-                             long rows, int cols, const int32_t* __restrict__ colmap,
-                             const int32_t* __restrict__ rowmap, int scatter) {
-  sm100::griddep_wait();
+__device__ __forceinline__ void permute_cols_bulk_body(uint8_t* smem_bulk, long bid, long nblk,
+                                                       const uint16_t* __restrict__ in, long ld_in,
+                                                       uint16_t* __restrict__ out, long ld_out, long rows, int cols,
+                                                       const int32_t* __restrict__ colmap,
+                                                       const int32_t* __restrict__ rowmap, int scatter) {
   using Word = typename std::conditional<ROWS == 4, uint64_t, uint32_t>::type;
-  extern __shared__ __align__(128) uint8_t smem_bulk[];
   const size_t slot_bytes = (size_t)ROWS * cols * 2;
   uint8_t* ring = smem_bulk;
   Word* W = reinterpret_cast<Word*>(smem_bulk + 2 * slot_bytes);
@@ -208,8 +210,8 @@ __global__ void __launch_bounds__(256, 2)
     sm100::mbar_init(sm100::smem_u32(bars + 0), 1);
     sm100::mbar_init(sm100::smem_u32(bars + 1), 1);
     sm100::fence_mbar_init();
-    if (blockIdx.x < ngroups) request(blockIdx.x, 0);
-    if (blockIdx.x + gridDim.x < ngroups) request(blockIdx.x + gridDim.x, 1);
+    if (bid < ngroups) request(bid, 0);
+    if (bid + nblk < ngroups) request(bid + nblk, 1);
   }
   // Source map (overlaps the first copies).
   {
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(256, 2)
   bool ok = true;
   int i = 0;
 #pragma unroll 1
-  for (long g = blockIdx.x; g < ngroups; g += gridDim.x, ++i) {
+  for (long g = bid; g < ngroups; g += nblk, ++i) {
     const int slot = i & 1;
     const long r0 = g * ROWS;
     const int nr = (int)min((long)ROWS, rows - r0);
@@ -265,9 +267,9 @@ __global__ void __launch_bounds__(256, 2)
       }
     }
     __syncthreads();  // W complete; the slot has been read by every thread
-    if (threadIdx.x == 0 && g + 2 * (long)gridDim.x < ngroups) {
+    if (threadIdx.x == 0 && g + 2 * nblk < ngroups) {
       sm100::fence_proxy_async_smem();  // the copy engine overwrites what the threads just read
-      request(g + 2 * (long)gridDim.x, slot);
+      request(g + 2 * nblk, slot);
     }
     {
       for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
@@ -291,11 +293,22 @@ __global__ void __launch_bounds__(256, 2)
   // A block that gave up (at its group i) waits, bounded, for the copies it still has in flight
   // (groups i and i + 1) before its shared memory is released.
   if (!ok && threadIdx.x == 0) {
-    long g = blockIdx.x + (long)i * gridDim.x;
-    for (int k = i; k < i + 2 && g < ngroups; ++k, g += gridDim.x)
+    long g = bid + (long)i * nblk;
+    for (int k = i; k < i + 2 && g < ngroups; ++k, g += nblk)
       sm100::mbar_wait(sm100::smem_u32(bars + (k & 1)), (uint32_t)(k >> 1) & 1u, KID_PERMUTE, 2);
   }
   __syncthreads();
+}
+
+template <int ROWS>
+__global__ void __launch_bounds__(256, 2)
+    permute_cols_bulk_kernel(const uint16_t* __restrict__ in, long ld_in, uint16_t* __restrict__ out, long ld_out,
+                             long rows, int cols, const int32_t* __restrict__ colmap,
+                             const int32_t* __restrict__ rowmap, int scatter) {
+  sm100::griddep_wait();
+  extern __shared__ __align__(128) uint8_t smem_bulk[];
+  permute_cols_bulk_body<ROWS>(smem_bulk, blockIdx.x, gridDim.x, in, ld_in, out, ld_out, rows, cols, colmap, rowmap,
+                               scatter);
 }
 
 // AdamW on packed parameters (decoupled weight decay), fp32: per parameter 16 bytes read

@@ -681,7 +681,7 @@ poetx_status cnp_bwd_generic(int b, int k, int dt, long nb, const float* theta, 
     g.epi.d1 = bslot(k - j); g.epi.d1_dtype = dt; g.epi.ld1 = kb; g.epi.zrow1 = b;
     g.epi.alpha1 = 1.f; g.epi.beta1 = 1.f;
     g.epi.c = S32; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
-    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_ADJ));
   }
   // Gbar_k = G - S.G into A-slot 1 (k >= 2);  E = 2G - S.G.
   {
@@ -692,7 +692,7 @@ poetx_status cnp_bwd_generic(int b, int k, int dt, long nb, const float* theta, 
     }
     g.epi.c = G32; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
     g.epi.d2 = E; g.epi.ld2 = b; g.epi.zrow2 = b; g.epi.alpha2 = -1.f; g.epi.beta2 = 2.f; g.epi.accum2 = 0;
-    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_ADJ));
   }
   // Gbar_j = -S.Gbar_{j+1} (Gbar_{j+1} in A-slot k-j) into A-slot k-j+1 (j >= 2);  E += Gbar_j.
   for (int j = k - 1; j >= 1; --j) {
@@ -702,7 +702,7 @@ poetx_status cnp_bwd_generic(int b, int k, int dt, long nb, const float* theta, 
       g.epi.alpha1 = -1.f; g.epi.beta1 = 0.f;
     }
     g.epi.d2 = E; g.epi.ld2 = b; g.epi.zrow2 = b; g.epi.alpha2 = -1.f; g.epi.beta2 = 0.f; g.epi.accum2 = 1;
-    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_ADJ));
   }
   // G_S = E + A-stack . B-stack^T  (K = k.b), written over E.
   {
@@ -712,7 +712,7 @@ poetx_status cnp_bwd_generic(int b, int k, int dt, long nb, const float* theta, 
     g.B = view(Bst, rows, kb, kb, b, 0);
     g.epi.d1 = E; g.epi.d1_dtype = F32; g.epi.ld1 = b; g.epi.zrow1 = b; g.epi.alpha1 = 1.f; g.epi.beta1 = 1.f;
     g.epi.c = E; g.epi.c_dtype = F32; g.epi.ldc = b; g.epi.zrowc = b;
-    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_GEMM));
+    POETX_TRY(run_gemm(dt, g, st, POETX_KC_CNP_ADJ));
   }
   return pack(E, nb, b, grad, st);
 }
@@ -736,7 +736,8 @@ struct CnpSide {
 };
 
 template <int B, bool ADJ>
-poetx_status launch_cnp_chip(int k, const CnpSide* sides, int nsides, cudaStream_t st) {
+poetx_status launch_cnp_chip(int k, const CnpSide* sides, int nsides, cudaStream_t st,
+                             const CnpGather* gather = nullptr) {
   using C = ChipCfg<B>;
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
@@ -765,14 +766,19 @@ poetx_status launch_cnp_chip(int k, const CnpSide* sides, int nsides, cudaStream
       if (!aligned16(sd.Q)) return POETX_ERR_ALIGNMENT;
       // Q leaves through TMA stores of (64 columns x rows-per-CTA) boxes.
       if (!make_tmap(&S.tmQ, view(sd.Q, sd.nb * B, B, B), 64, C::ROWS)) return POETX_ERR_CUDA;
-    } else if (!aligned16(sd.part) || sd.splits < 1) {
-      return POETX_ERR_ALIGNMENT;
+    } else {
+      if (!aligned16(sd.part) || sd.splits < 1) return POETX_ERR_ALIGNMENT;
+      // G partials arrive through TMA loads of (32 columns x rows-per-CTA) fp32 boxes.
+      if (!make_tmap(&S.tmG, view(sd.part, (long)sd.splits * sd.nb * B, B, B), 32, C::ROWS, F32))
+        return POETX_ERR_CUDA;
     }
   }
   if (nb_total == 0) return POETX_OK;
-  if (nb_total * C::NCTA > 0x7fffffffL) return POETX_ERR_UNSUPPORTED_SHAPE;
+  if (nb_total * C::NCTA > 0x7fffffffL - 1024) return POETX_ERR_UNSUPPORTED_SHAPE;
+  a.ncnp = (int)(nb_total * C::NCTA);
+  if (gather != nullptr) a.gather = *gather;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(nb_total * C::NCTA), 1, 1);
+  cfg.gridDim = dim3((unsigned)(a.ncnp + a.gather.nblk), 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
@@ -790,9 +796,42 @@ poetx_status launch_cnp_chip(int k, const CnpSide* sides, int nsides, cudaStream
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  LaunchScope ls(POETX_KC_CNP_GEMM, st);
+  LaunchScope ls(ADJ ? POETX_KC_CNP_ADJ : POETX_KC_CNP_GEMM, st);
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return POETX_ERR_CUDA;
   return last_launch();
+}
+
+// SMs of the current device (cached per device).
+int device_sms() {
+  static int sms[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return kNumSms;
+  if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms[dev] = kNumSms;
+  return sms[dev];
+}
+
+// Forward CNP of both sides of a b = 256 layer (one SM pair per block) with the input gather
+// U = X[:, pi_R] on the SMs the pairs leave free, in the same launch.  Returns false (nothing
+// launched) where that does not fit: other block sizes, too few free SMs, rows too wide for the
+// launch's shared memory.
+bool cnp_fwd_with_gather(int b, int k, const CnpSide* sides, int nsides, const void* X, long ld_x, void* U, long ld_u,
+                         long rows, int cols, const int32_t* colmap, cudaStream_t st, poetx_status* status) {
+  if (b != 256 || rows <= 0) return false;
+  long nb_total = 0;
+  for (int q = 0; q < nsides; ++q) nb_total += sides[q].nb;
+  const long free_sms = (long)device_sms() - 2 * nb_total;
+  if (free_sms < 16 || cols > 8192 || cols % 8 || permute_bulk_smem_bytes<4>(cols) + 1024 > ChipCfg<256>::SMEM ||
+      !aligned16(X) || !aligned16(U) || !aligned16(colmap) || ld_x % 8 || ld_u % 8)
+    return false;
+  CnpGather g;
+  g.in = static_cast<const uint16_t*>(X); g.ld_in = ld_x;
+  g.out = static_cast<uint16_t*>(U); g.ld_out = ld_u;
+  g.rows = rows; g.cols = cols; g.colmap = colmap;
+  const long groups = (rows + 3) / 4;
+  g.nblk = (int)std::min<long>(free_sms & ~1L, (groups + 1) & ~1L);  // whole clusters of two
+  *status = launch_cnp_chip<256, false>(k, sides, nsides, st, &g);
+  return true;
 }
 
 template <bool ADJ>
@@ -975,9 +1014,9 @@ poetx_status check_ws(const void* ws, size_t have, size_t need) {
 // Forward chain into caller buffers; `Z` receives the W0'-GEMM output.
 poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const void* W0p, const float* W0s,
                            const int32_t* pL, const int32_t* pR, const void* QR, const void* QP, void* Y, void* Z,
-                           char* U, char* V, char* Yp, cudaStream_t st) {
+                           char* U, char* V, char* Yp, cudaStream_t st, bool gathered = false) {
   const int dt = d->dtype, b = d->b;
-  POETX_TRY(permute_cols(dt, X, d->d_in, U, d->d_in, n, d->d_in, pR, nullptr, false, st));
+  if (!gathered) POETX_TRY(permute_cols(dt, X, d->d_in, U, d->d_in, n, d->d_in, pR, nullptr, false, st));
   POETX_TRY(bd_forward(dt, n, d->d_in, b, U, QP, V, st));
   GemmDesc g;
   g.M = (int)n; g.N = d->d_out; g.K = d->d_in;
@@ -1206,6 +1245,50 @@ struct SideJoin {
     if (armed) stream_edge(side, main, e);
   }
 };
+
+// CNP and forward pass in one call.  The CNP and the input gather U = X[:, pi_R] are independent
+// and neither fills the GPU (the on-chip CNP takes one SM pair per 256-block), so for b = 256
+// they run in one launch: the blocks past the CNP pairs gather rows on the remaining SMs.  The
+// block-diagonal product, which needs Q_P and U, follows.  Elsewhere the parts run one after
+// the other.
+poetx_status poetx_cnp_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0p,
+                               const int32_t* perm_L, const int32_t* perm_R, const float* theta_R,
+                               const float* theta_P, void* Q_R, void* Q_P, void* Y, void* saved, void* workspace,
+                               size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  POETX_TRY(check_ptrs({theta_R, theta_P, Q_R, Q_P}));
+  const int b = desc->b, dt = desc->dtype;
+  if (n_tokens <= 0 || !cnp_fused_ok(b, dt)) {
+    if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
+    POETX_TRY(poetx_cnp(desc, theta_R, theta_P, Q_R, Q_P, workspace, ws_bytes, stream));
+    return forward_impl(desc, n_tokens, X, W0p, nullptr, perm_L, perm_R, Q_R, Q_P, Y, saved, workspace, ws_bytes,
+                        stream);
+  }
+  if (desc->mode == POETX_FAST && saved == nullptr) return POETX_ERR_INVALID_ARG;
+  if (desc->mode == POETX_MEM && saved != nullptr) return POETX_ERR_INVALID_ARG;
+  POETX_TRY(check_ptrs({X, W0p, perm_L, perm_R, Y}));
+  if (saved != nullptr && !aligned16(saved)) return POETX_ERR_ALIGNMENT;
+  const FwdPlan f = fwd_plan(desc, n_tokens);
+  POETX_TRY(check_ws(workspace, ws_bytes, f.total));
+  POETX_TRY(debug_check_perms(stream, {{perm_L, desc->d_out}, {perm_R, desc->d_in}}));
+  char* ws = static_cast<char*>(workspace);
+  const size_t zbytes = (size_t)n_tokens * desc->d_out * esize(dt);
+  void* Z = desc->mode == POETX_FAST ? saved : ws + f.Z;
+  char* U = desc->mode == POETX_FAST ? static_cast<char*>(saved) + zbytes : ws + f.U;
+  CnpSide sides[2];
+  sides[0].nb = desc->d_out / b; sides[0].theta = theta_R; sides[0].Q = Q_R;
+  sides[1].nb = desc->d_in / b; sides[1].theta = theta_P; sides[1].Q = Q_P;
+  poetx_status st = POETX_OK;
+  if (cnp_fwd_with_gather(b, desc->k, sides, 2, X, desc->d_in, U, desc->d_in, n_tokens, desc->d_in, perm_R, stream,
+                          &st)) {
+    POETX_TRY(st);
+  } else {
+    POETX_TRY(cnp_fwd_fused(b, desc->k, sides, 2, stream));
+    POETX_TRY(permute_cols(dt, X, desc->d_in, U, desc->d_in, n_tokens, desc->d_in, perm_R, nullptr, false, stream));
+  }
+  return forward_chain(desc, n_tokens, X, W0p, nullptr, perm_L, perm_R, Q_R, Q_P, Y, Z, U, ws + f.V, ws + f.Yp,
+                       stream, true);
+}
 
 static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const void* dY, const void* X,
                                   const void* W0p, const float* W0s, const int32_t* perm_L, const int32_t* perm_R,
@@ -1573,6 +1656,32 @@ poetx_status poetx_device_status(int* detail) {
   if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return POETX_ERR_CUDA;
   if (detail) *detail = v;
   return v ? POETX_ERR_DEVICE_TIMEOUT : POETX_OK;
+}
+
+// Failure-detection probe: one CTA waits on a shared-memory mbarrier that nothing ever arrives
+// on, bounded by limit_ns.  The bounded wait gives up, records (KID_WAIT_PROBE, 1) in the device
+// error word and returns; the kernel then writes 2 to *returned (1 would mean the wait completed).
+enum : int { KID_WAIT_PROBE = 7 };
+__global__ void wait_probe_kernel(unsigned long long limit_ns, int* returned) {
+  using namespace sm100;
+  __shared__ uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool done = mbar_wait_limit(b, 0, limit_ns, KID_WAIT_PROBE, 1);
+  __syncthreads();
+  if (threadIdx.x == 0) *returned = done ? 1 : 2;
+}
+
+poetx_status poetx_test_wait_timeout(long long limit_ns, int* returned, poetx_stream stream) {
+  if (returned == nullptr || limit_ns < 1000 || limit_ns > 100000000LL) return POETX_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(returned) & 3u) != 0) return POETX_ERR_ALIGNMENT;
+  LaunchScope ls(POETX_KC_ELEMENTWISE, stream);
+  wait_probe_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns, returned);
+  return last_launch();
 }
 
 poetx_status poetx_test_gemm(int dtype, int M, int N, int K, int batch, int splits, const void* a, long long a_rows,

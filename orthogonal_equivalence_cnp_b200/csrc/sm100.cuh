@@ -40,20 +40,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits for the phase of parity `parity` to complete.  Gives up after kWaitLimitNs, records
-// (kernel_id, site) in the device error word and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int kernel_id, int site) {
+// Waits for the phase of parity `parity` to complete.  Gives up after limit_ns nanoseconds,
+// records (kernel_id, site) in the device error word and returns false.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
+                                                int kernel_id, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       record_device_error(kernel_id, site);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int kernel_id, int site) {
+  return mbar_wait_limit(bar, parity, kWaitLimitNs, kernel_id, site);
 }
 
 // ---------------------------------------------------------------------------------------- TMA

@@ -9,7 +9,7 @@ import numpy as np
 import torch
 
 from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_adamw_cfg, poetx_adamw_reset,
-               poetx_adamw_step, poetx_backward, poetx_cnp, poetx_desc, poetx_forward,
+               poetx_adamw_step, poetx_backward, poetx_cnp, poetx_cnp_forward, poetx_desc, poetx_forward,
                poetx_merge, poetx_wc_backward, poetx_wc_forward, poetx_wc_saved_size, poetx_wc_workspace_size,
                poetx_workspace_size, poetx_xq_backward, poetx_xq_forward, poetx_xq_merge, poetx_xq_quantize)
 
@@ -105,10 +105,19 @@ class PoetxLayer:
         self.W0p = None  # stream-ordered release: the quantiser has been enqueued before it
         self.xq = True
 
+    def cnp_forward(self, X: torch.Tensor):
+        """CNP and layer forward in one library call (the CNP overlaps the input gather)."""
+        poetx_cnp_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.theta_R, self.theta_P,
+                          self.Q_R, self.Q_P, self.Y, self.saved, self.ws)
+        return self.Y
+
     def step(self, X: torch.Tensor, dY: torch.Tensor):
         """CNP forward + layer forward + layer backward (incl. the CNP adjoint)."""
-        self.cnp()
-        self.forward(X)
+        if self.xq:
+            self.cnp()
+            self.forward(X)
+        else:
+            self.cnp_forward(X)
         self.backward(dY, X)
 
     def optimizer_step(self, cfg: poetx_adamw_cfg):
@@ -141,7 +150,7 @@ class PoetxLayer:
             self.wc_saved = torch.empty(poetx_wc_saved_size(self.desc), dtype=torch.uint8, device=self.device)
             self.wc_ws = torch.empty(max(poetx_wc_workspace_size(self.desc), 256), dtype=torch.uint8,
                                      device=self.device)
-        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, None, self.wc_ws)
+        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.wc_ws)
         poetx_wc_forward(self.desc, self.n, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
                          self.wc_saved, self.wc_ws)
         poetx_wc_backward(self.desc, self.n, dY, X, self.W0p, self.perm_L, self.perm_R, self.Q_R, self.theta_R,

@@ -167,3 +167,12 @@ def test_check_permutation_on_the_host():
             P.poetx_check_permutation(np.array(bad, np.int32))
     assert P.lib().poetx_check_permutation(None, 3) == 1 and P.lib().poetx_check_permutation(None, 0) == 0
     assert P.lib().poetx_check_permutation(None, -1) == 1
+
+
+def test_wait_probe_host_validation():
+    L = P.lib()
+    A = 1 << 20
+    assert L.poetx_test_wait_timeout(1_000_000, None, None) == 1
+    assert L.poetx_test_wait_timeout(10, A, None) == 1            # below 1 us
+    assert L.poetx_test_wait_timeout(10 ** 9, A, None) == 1       # above 100 ms
+    assert L.poetx_test_wait_timeout(1_000_000, A + 2, None) == 3

@@ -186,6 +186,31 @@ def test_layer_bf16_orders(k):
     _check_all(g, oracle_layer(inp), TOL["bf16"])
 
 
+@pytest.mark.parametrize("dtype,b,mode", [("bf16", 256, "fast"), ("bf16", 64, "mem"), ("f32", 32, "fast")])
+def test_cnp_forward_call_equals_the_two_calls(dtype, b, mode):
+    # poetx_cnp_forward runs the CNP beside the input gather; the results are the same kernels'
+    # results, so they must equal poetx_cnp followed by poetx_forward bit for bit.
+    s = I.small_shape(4 * b, 2 * b, b, 3, 200, dtype, theta_std=0.005 if dtype == "bf16" else 0.05, w_std=0.02)
+    inp = I.make_layer(s, 17 + b)
+    L = PoetxLayer(make_desc(4 * b, 2 * b, b, 3, dtype, mode), 200)
+    L.load_state(inp.W0, inp.theta_R, inp.theta_P, inp.pi_L, inp.pi_R)
+    X = L.to_dev(inp.X)
+    L.cnp()
+    L.forward(X)
+    torch.cuda.synchronize()
+    ref = {k: t.clone() for k, t in (("Q_R", L.Q_R), ("Q_P", L.Q_P), ("Y", L.Y))}
+    saved_ref = L.saved.clone() if L.saved is not None else None
+    for t in (L.Q_R, L.Q_P, L.Y):
+        t.fill_(float("nan"))
+    L.cnp_forward(X)
+    torch.cuda.synchronize()
+    device_clean()
+    for k, t in (("Q_R", L.Q_R), ("Q_P", L.Q_P), ("Y", L.Y)):
+        assert torch.equal(t, ref[k]), k
+    if saved_ref is not None:
+        assert torch.equal(L.saved, saved_ref)
+
+
 def test_fast_and_mem_agree():
     s = I.small_shape(512, 512, 128, 3, 200, "bf16", theta_std=0.005, w_std=0.02)
     inp = I.make_layer(s, 77)
