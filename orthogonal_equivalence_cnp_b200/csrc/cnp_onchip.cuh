@@ -64,7 +64,10 @@ struct ChipCfg {
   static constexpr uint32_t GBOX = ROWS * 128;     // G staging: one 32-column fp32 box of this CTA's rows
   static constexpr int QN = PAIR ? 128 : B;        // PACK quadrant: QN x QN fp32, rows at QPITCH floats
   static constexpr int QPITCH = QN + 4;
-  static constexpr size_t BAR_OFF = 3 * (size_t)REG;
+  // Pair only: XS, the staging of the quadrant sent to the peer's B form (two 16 KiB atoms).
+  static constexpr uint32_t XS_OFF = 3 * REG;
+  static constexpr uint32_t XS_BYTES = PAIR ? 2 * 128 * 128 : 0;
+  static constexpr size_t BAR_OFF = 3 * (size_t)REG + XS_BYTES;
   static constexpr size_t SMEM = BAR_OFF + 256 + 1024;
   static_assert((size_t)(B / 32) * GBOX <= 2 * (size_t)REG, "G staging fits V1 + V2");
   static_assert((size_t)B * (B - 1) / 2 * 4 <= 2 * (size_t)REG, "theta staging fits V1 + V2");
@@ -81,9 +84,11 @@ struct CnpChipSide {
   int nb;
   int splits;
 };
-// Spare blocks of a forward launch: the blocks past the CNP ones permute the columns of a bf16
-// row-major array (the input gather U = X[:, pi_R] of the layer), as permute_cols_bulk_kernel
-// does, on the SMs the CNP leaves free.
+// Spare blocks of a launch: the blocks past the CNP ones permute the columns of a bf16 row-major
+// array, as permute_cols_bulk_kernel does, on the SMs the CNP leaves free (the forward's input
+// gather U = X[:, pi_R], the adjoint's scatter of dU into dX), with a deeper ring (one block per
+// SM there, and the CNP's shared memory to fill).
+constexpr int kSpareSlots = 4;
 struct CnpGather {
   const uint16_t* in;
   long ld_in;
@@ -92,7 +97,8 @@ struct CnpGather {
   long rows;
   const int32_t* colmap;
   int cols;
-  int nblk;  // number of spare blocks (0: none)
+  int scatter;  // 0: out[r][j] = in[r][colmap[j]];  1: out[r][colmap[j]] = in[r][j]
+  int nblk;     // number of spare blocks (0: none)
 };
 struct CnpChipArgs {
   CnpChipSide seg[2];
@@ -129,16 +135,15 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   const uint32_t bar_mma = smem_u32(bars), bar_ready = smem_u32(bars + 1), bar_theta = smem_u32(bars + 2);
   const uint32_t bar_g = smem_u32(bars + 3);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 5);
+  const uint32_t bar_xin = smem_u32(bars + 4);  // data sent by the peer has landed here
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 6);
 
-  if constexpr (!ADJ) {
-    if ((int)blockIdx.x >= args.ncnp) {  // a spare block: gather rows (whole clusters, no TMEM)
-      griddep_wait();
-      const CnpGather& G = args.gather;
-      permute_cols_bulk_body<4>(smem, (long)blockIdx.x - args.ncnp, G.nblk, G.in, G.ld_in, G.out, G.ld_out, G.rows,
-                                G.cols, G.colmap, nullptr, 0);
-      return;
-    }
+  if ((int)blockIdx.x >= args.ncnp) {  // a spare block: permute rows (whole clusters, no TMEM)
+    griddep_wait();
+    const CnpGather& G = args.gather;
+    permute_cols_bulk_body<4, kSpareSlots>(smem, (long)blockIdx.x - args.ncnp, G.nblk, G.in, G.ld_in, G.out,
+                                           G.ld_out, G.rows, G.cols, G.colmap, nullptr, G.scatter);
+    return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3, half = warp >> 2;
@@ -162,6 +167,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     mbar_init(bar_ready, 8 * C::NCTA);
     mbar_init(bar_theta, 1);
     mbar_init(bar_g, 1);
+    mbar_init(bar_xin, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -183,25 +189,37 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
   griddep_wait();  // theta and the gradient partials come from earlier kernels
 
   bool ok = true;
-  uint32_t mma_phase = 0, ready_phase = 0;
+  uint32_t mma_phase = 0, ready_phase = 0, xin_phase = 0;
+  const uint32_t peer = (uint32_t)(c ^ 1);
 
   // All epilogue warps of the pair report that their writes for the next product are done.
-  auto arrive_ready = [&]() {
-    fence_proxy_async_all();
+  // After an exchange (xin), the odd CTA's warp 0 first waits for the peer's data to land in its
+  // own B form, so that the leader's `ready` also stands for that data.
+  auto arrive_ready = [&](bool xin = false) {
+    fence_proxy_async_smem();  // every operand write is to this CTA's own shared memory
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
-      if constexpr (C::PAIR) mbar_arrive_cluster(ready_dst); else mbar_arrive(bar_ready);
+      if constexpr (C::PAIR) {
+        if (xin && c == 1 && warp == 0 && ok) ok = mbar_wait_cluster(bar_xin, xin_phase & 1u, KID_CNP_CHIP, 11);
+        mbar_arrive_cluster(ready_dst);
+      } else {
+        mbar_arrive(bar_ready);
+      }
     }
+    if (xin) ++xin_phase;
   };
   // D = A . B^T (+ D) over K = b, A K-major (A form), B K-major (A form of its N rows) or
   // MN-major (B form); a_neg negates A.  Issued by one thread once the pair is ready.
-  auto issue = [&](uint32_t a, uint32_t b_op, bool b_mn, bool a_neg, bool accumulate, int site) {
+  // xin: the B operand is a B form just exchanged; the leader also waits for its own incoming half
+  // (the odd CTA's was folded into its `ready` arrival).  Call after arrive_ready(true).
+  auto issue = [&](uint32_t a, uint32_t b_op, bool b_mn, bool a_neg, bool accumulate, int site, bool xin = false) {
     if (leader && warp == 0) {
       if (lane == 0) {
         if (ok) ok = C::PAIR ? mbar_wait_cluster(bar_ready, ready_phase, KID_CNP_CHIP, site)
                              : mbar_wait(bar_ready, ready_phase, KID_CNP_CHIP, site);
+        if (C::PAIR && xin && ok) ok = mbar_wait_cluster(bar_xin, (xin_phase - 1) & 1u, KID_CNP_CHIP, 12);
         if (ok) {
           tc_fence_after();
           const uint32_t idesc = idesc_bf16_f32(C::M, B, false, b_mn) | (a_neg ? (1u << 13) : 0u);
@@ -236,21 +254,53 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
 #pragma unroll
     for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(w[u]);
   };
+  auto tld2 = [&](uint32_t col1, float (&v1)[32], uint32_t col2, float (&v2)[32]) {
+    uint32_t w1[32], w2[32];
+    tmem_ld_32x32b_x32(col1, w1);
+    tmem_ld_32x32b_x32(col2, w2);
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      v1[u] = __uint_as_float(w1[u]);
+      v2[u] = __uint_as_float(w2[u]);
+    }
+  };
   auto tst = [&](uint32_t col, const float (&v)[32]) {
     tmem_st_32x32b_x32(col, reinterpret_cast<const uint32_t(&)[32]>(v));
   };
   // Row i, columns j0..j0+31 of the B form: element (k = i, n = j) in the CTA owning column j.
+  // The peer's columns go to XS, laid out as the peer's B-form rows of this CTA's rows, and
+  // leave in one exchange (send_bform) once every warp has written them.
   auto put_bform = [&](uint32_t buf, int j0, const float (&v)[32]) {
     const int ct = C::PAIR ? j0 / 128 : 0;
     const int nl = j0 - 128 * ct;
-    uint32_t row = buf + (uint32_t)(nl / 64) * C::BFORM_ATOM + (uint32_t)i * 128u;
-    if (C::PAIR && ct != c) row = mapa_shared(row, (uint32_t)ct);
+    const uint32_t row = (C::PAIR && ct != c) ? s0 + C::XS_OFF + (uint32_t)(nl / 64) * (128u * 128u) + (uint32_t)r * 128u
+                                              : buf + (uint32_t)(nl / 64) * C::BFORM_ATOM + (uint32_t)i * 128u;
     const int ch0 = (nl % 64) / 8;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const uint4 w = make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
                                  pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
-      st_cluster_v4(row + (uint32_t)(((ch0 + u) ^ (i & 7)) * 16), w);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)(((ch0 + u) ^ (i & 7)) * 16)),
+                   "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w)
+                   : "memory");
+    }
+  };
+  // The exchange of a B form written by put_bform (pair only; every thread calls it): the peer
+  // expects 32 KiB on its xin barrier; this CTA's XS (rows O_c of the peer's two column atoms)
+  // goes out as two 16 KiB copies into the peer's buffer `buf`.
+  auto send_bform = [&](uint32_t buf) {
+    if constexpr (C::PAIR) {
+      if (threadIdx.x == 0) mbar_arrive_expect_tx(bar_xin, 2u * 128u * 128u);
+      fence_proxy_async_smem();  // XS was written by the generic proxy; the copy engine reads it
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const uint32_t bar_peer = mapa_shared(bar_xin, peer);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          bulk_copy_to_peer(mapa_shared(buf + (uint32_t)t * C::BFORM_ATOM + (uint32_t)(128 * c) * 128u, peer),
+                            s0 + C::XS_OFF + (uint32_t)t * (128u * 128u), 128u * 128u, bar_peer);
+      }
     }
   };
   // Q rows of this CTA leave through TMA stores of the A-form staging in V2.
@@ -300,15 +350,18 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
 #pragma unroll
         for (int u = 0; u < 32; ++u) v[u] = -src[u * step0 - (u * (u - 1)) / 2];
       } else {
-        // the warp's diagonal block
-        const int roj0 = ro(j0);
+        // The warp's diagonal block: both candidates are loaded at offsets that are the same for
+        // every lane (the one not selected is a harmless shared-memory read: at worst one float
+        // before the staging, for row 0), then selected.
+        const float* up = th + roi + j0;
+        const float* lo = th + ro(j0) + i;
         const int step0 = B - 2 - j0;
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
+          const float xu = up[u];
+          const float xl = lo[u * step0 - (u * (u - 1)) / 2];
           const int j = j0 + u;
-          const int idx = j > i ? roi + j : (j < i ? roj0 + u * step0 - (u * (u - 1)) / 2 + i : 0);
-          const float x = th[idx];
-          v[u] = j > i ? x : (j < i ? -x : 0.f);
+          v[u] = j > i ? xu : (j < i ? -xl : 0.f);
         }
       }
       chip_put_aform(SC, r, j0, v);
@@ -433,6 +486,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
         chip_put_aform(V1, r, j0, g);
         if (valid) put_bform(V2, j0, g);
       }
+      send_bform(V2);
     }
     uint32_t fcol = REG2;  // the TMEM columns holding G_S for PACK
     if (k >= 1) {
@@ -445,15 +499,14 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
 #pragma unroll 1
         for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
           float d[32], g[32];
-          tld(ACC + j0, d);
-          tld(REG2 + j0, g);
+          tld2(ACC + j0, d, REG2 + j0, g);
 #pragma unroll
           for (int u = 0; u < 32; ++u) d[u] += 2.f * g[u];  // R_a
           tst(ACC + j0, d);
           if (a > 0) chip_put_aform(V1, r, j0, d);
         }
-        arrive_ready();
-        issue(SC, V2, true, true, true, 8);  // ACC += (-S) . L_{a+1} = T L_{a+1}
+        arrive_ready(true);  // MMA_L reads V2 = L_{a+1}, the B form exchanged after its epilogue
+        issue(SC, V2, true, true, true, 8, true);  // ACC += (-S) . L_{a+1} = T L_{a+1}
         wait_mma(9);
         if (a > 0) {
 #pragma unroll 1
@@ -462,6 +515,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
             tld(ACC + j0, l);
             if (valid) put_bform(V2, j0, l);
           }
+          send_bform(V2);
         }
       }
     } else {
@@ -482,7 +536,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
       const bool to_peer = C::PAIR && c == 0 && half == 1;  // G_S[O_0][O_1] -> CTA 1's Qx
       uint32_t dst = 0;
       if (own_cols) dst = QD + (uint32_t)(r * C::QPITCH * 4);
-      if (to_peer) dst = mapa_shared(QX + (uint32_t)(r * C::QPITCH * 4), 1);
+      if (to_peer) dst = QX + (uint32_t)(r * C::QPITCH * 4);  // staged here, sent in one copy below
 #pragma unroll 1
       for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
         float f[32];
@@ -491,33 +545,50 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
           const uint32_t at = dst + (uint32_t)((j0 - (own_cols ? own0 : 128)) * 4);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            st_cluster_v4(at + 16 * u, make_uint4(__float_as_uint(f[4 * u]), __float_as_uint(f[4 * u + 1]),
-                                                  __float_as_uint(f[4 * u + 2]), __float_as_uint(f[4 * u + 3])));
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(at + 16 * u), "r"(__float_as_uint(f[4 * u])),
+                         "r"(__float_as_uint(f[4 * u + 1])), "r"(__float_as_uint(f[4 * u + 2])),
+                         "r"(__float_as_uint(f[4 * u + 3]))
+                         : "memory");
         }
       }
-      if constexpr (C::PAIR) cluster_sync_all(); else __syncthreads();
-      // Thread (row j, half h): the entries (i, j) with i < j and i in the columns of its half.
-      // The TMEM loads are warp-collective: the chunk loop runs to the warp's first row (the
-      // same bound for every lane) and the per-entry test i < j only guards the stores.
+      constexpr uint32_t QBYTES = C::QN * C::QPITCH * 4;
+      if (C::PAIR && c == 1 && threadIdx.x == 0) mbar_arrive_expect_tx(bar_xin, QBYTES);
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (C::PAIR && c == 0 && threadIdx.x == 0)
+        bulk_copy_to_peer(mapa_shared(QX, 1), QX, QBYTES, mapa_shared(bar_xin, 1));
+      if (C::PAIR && c == 1) {  // both warps of a quarter read G_S[O_0][O_1], sent by CTA 0
+        if (ok) ok = mbar_wait(bar_xin, xin_phase & 1u, KID_CNP_CHIP, 13);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      ++xin_phase;
+      // Thread (row j): the entries (i, j), i < j, of 32-column chunks of i.  A lane quarter's
+      // chunks are Qd's chunks below its rows (and, in a pair's CTA 1, the four chunks of Qx);
+      // the two warps of the quarter take them in turn.  The TMEM loads are warp-collective: the
+      // chunk list is the same for every lane, and i < j only guards the stores.
       const int j = i;
-      const bool diag = !C::PAIR || half == c;            // i in O_c: quadrant Qd
-      const bool cross = C::PAIR && c == 1 && half == 0;  // i in O_0, j in O_1: quadrant Qx
-      if (diag || cross) {
-        const float* Q = reinterpret_cast<const float*>(smem + (diag ? 0 : C::QN * C::QPITCH * 4));
-        const int jq = j - own0;                  // column of j in the quadrant
-        const int qrow0 = diag ? own0 : 0;        // block row of the quadrant's first row
-        const int jwarp = rbase + quarter * 32;   // first row of this warp
-        const bool store = ok && valid;
-        float* out = SD.grad + z * P;
+      const int jwarp = rbase + quarter * 32;  // first row of this warp
+      const int ndiag = jwarp < B ? (jwarp - own0) / 32 + 1 : 0;  // warps past row b - 1 (b = 64) have none
+      const int ncross = (C::PAIR && c == 1) ? 4 : 0;
+      const bool store = ok && valid;
+      float* out = SD.grad + z * P;
 #pragma unroll 1
-        for (int i0 = c0; i0 < c0 + C::HALF && i0 <= jwarp; i0 += 32) {
-          float f[32];
-          tld(fcol + i0, f);  // G_S[j][i0 .. i0 + 31]
+      for (int item = half; item < ncross + ndiag; item += 2) {
+        const bool cross = item < ncross;
+        const int i0 = cross ? 32 * item : own0 + 32 * (item - ncross);
+        float f[32];
+        tld(fcol + i0, f);  // G_S[j][i0 .. i0 + 31]
+        // G_S[i0 + u][j] at qcol[u * QPITCH]; g[p(i0 + u, j)] at o_u, with
+        // p(i + 1, j) - p(i, j) = b - 2 - i.
+        const float* qcol = reinterpret_cast<const float*>(smem + (cross ? C::QN * C::QPITCH * 4 : 0)) +
+                            (i0 - (cross ? 0 : own0)) * C::QPITCH + (j - own0);
+        float* o = out + ro(i0) + j;
+        int step = B - 2 - i0;
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int ii = i0 + u;
-            if (store && ii < j) out[ro(ii) + j] = Q[(ii - qrow0) * C::QPITCH + jq] - f[u];
-          }
+        for (int u = 0; u < 32; ++u) {
+          if (store && i0 + u < j) *o = qcol[u * C::QPITCH] - f[u];
+          o += step;
+          --step;
         }
       }
     }

@@ -165,18 +165,18 @@ __global__ void __launch_bounds__(256, ROWS == 4 ? 3 : 2)
 // id KID_PERMUTE); a block that gives up still reaches every barrier and skips its stores.
 enum : int { KID_PERMUTE = 3 };
 
-template <int ROWS>
+template <int ROWS, int SLOTS = 2>
 __host__ __device__ constexpr size_t permute_bulk_smem_bytes(int cols) {
-  return 2 * (size_t)ROWS * cols * 2        // ring: two slots of ROWS rows
+  return SLOTS * (size_t)ROWS * cols * 2    // ring: SLOTS slots of ROWS rows
          + (size_t)cols * 2 * ROWS          // W: one word of ROWS elements per column
          + ((size_t)cols * 2 + 15) / 16 * 16  // source map
-         + 64;                               // two mbarriers (+ padding)
+         + 8 * SLOTS + 48;                   // SLOTS mbarriers (+ padding)
 }
 
 // The body of the kernel below as a device function: block `bid` of `nblk` blocks (256 threads)
 // permutes its share of the row groups, staging in `smem_bulk` (permute_bulk_smem_bytes<ROWS>(cols)
 // bytes, 128-byte aligned).  It also serves the spare blocks of a CNP launch (cnp_onchip.cuh).
-template <int ROWS>
+template <int ROWS, int SLOTS = 2>
 __device__ __forceinline__ void permute_cols_bulk_body(uint8_t* smem_bulk, long bid, long nblk,
                                                        const uint16_t* __restrict__ in, long ld_in,
                                                        uint16_t* __restrict__ out, long ld_out, long rows, int cols,
@@ -185,9 +185,9 @@ __device__ __forceinline__ void permute_cols_bulk_body(uint8_t* smem_bulk, long 
   using Word = typename std::conditional<ROWS == 4, uint64_t, uint32_t>::type;
   const size_t slot_bytes = (size_t)ROWS * cols * 2;
   uint8_t* ring = smem_bulk;
-  Word* W = reinterpret_cast<Word*>(smem_bulk + 2 * slot_bytes);
-  uint16_t* src_of = reinterpret_cast<uint16_t*>(smem_bulk + 2 * slot_bytes + (size_t)cols * 2 * ROWS);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_bulk + 2 * slot_bytes + (size_t)cols * 2 * ROWS +
+  Word* W = reinterpret_cast<Word*>(smem_bulk + SLOTS * slot_bytes);
+  uint16_t* src_of = reinterpret_cast<uint16_t*>(smem_bulk + SLOTS * slot_bytes + (size_t)cols * 2 * ROWS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_bulk + SLOTS * slot_bytes + (size_t)cols * 2 * ROWS +
                                                ((size_t)cols * 2 + 15) / 16 * 16);
   const int nvec = cols / 8;
   const long ngroups = (rows + ROWS - 1) / ROWS;
@@ -207,11 +207,12 @@ __device__ __forceinline__ void permute_cols_bulk_body(uint8_t* smem_bulk, long 
   };
 
   if (threadIdx.x == 0) {
-    sm100::mbar_init(sm100::smem_u32(bars + 0), 1);
-    sm100::mbar_init(sm100::smem_u32(bars + 1), 1);
+#pragma unroll
+    for (int q = 0; q < SLOTS; ++q) sm100::mbar_init(sm100::smem_u32(bars + q), 1);
     sm100::fence_mbar_init();
-    if (bid < ngroups) request(bid, 0);
-    if (bid + nblk < ngroups) request(bid + nblk, 1);
+#pragma unroll
+    for (int q = 0; q < SLOTS; ++q)
+      if (bid + q * nblk < ngroups) request(bid + q * nblk, q);
   }
   // Source map (overlaps the first copies).
   {
@@ -243,10 +244,10 @@ __device__ __forceinline__ void permute_cols_bulk_body(uint8_t* smem_bulk, long 
   int i = 0;
 #pragma unroll 1
   for (long g = bid; g < ngroups; g += nblk, ++i) {
-    const int slot = i & 1;
+    const int slot = i % SLOTS;
     const long r0 = g * ROWS;
     const int nr = (int)min((long)ROWS, rows - r0);
-    const bool got = sm100::mbar_wait(sm100::smem_u32(bars + slot), (uint32_t)(i >> 1) & 1u, KID_PERMUTE, 1);
+    const bool got = sm100::mbar_wait(sm100::smem_u32(bars + slot), (uint32_t)(i / SLOTS) & 1u, KID_PERMUTE, 1);
     ok = __syncthreads_and(got);
     if (!ok) break;  // block-uniform
     // Interleave the slot into W (rows past nr repeat the last row).
@@ -267,9 +268,9 @@ __device__ __forceinline__ void permute_cols_bulk_body(uint8_t* smem_bulk, long 
       }
     }
     __syncthreads();  // W complete; the slot has been read by every thread
-    if (threadIdx.x == 0 && g + 2 * nblk < ngroups) {
+    if (threadIdx.x == 0 && g + SLOTS * nblk < ngroups) {
       sm100::fence_proxy_async_smem();  // the copy engine overwrites what the threads just read
-      request(g + 2 * nblk, slot);
+      request(g + SLOTS * nblk, slot);
     }
     {
       for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
@@ -291,11 +292,11 @@ __device__ __forceinline__ void permute_cols_bulk_body(uint8_t* smem_bulk, long 
     __syncthreads();  // W free again
   }
   // A block that gave up (at its group i) waits, bounded, for the copies it still has in flight
-  // (groups i and i + 1) before its shared memory is released.
+  // (groups i .. i + SLOTS - 1) before its shared memory is released.
   if (!ok && threadIdx.x == 0) {
     long g = bid + (long)i * nblk;
-    for (int k = i; k < i + 2 && g < ngroups; ++k, g += nblk)
-      sm100::mbar_wait(sm100::smem_u32(bars + (k & 1)), (uint32_t)(k >> 1) & 1u, KID_PERMUTE, 2);
+    for (int k = i; k < i + SLOTS && g < ngroups; ++k, g += nblk)
+      sm100::mbar_wait(sm100::smem_u32(bars + (k % SLOTS)), (uint32_t)(k / SLOTS) & 1u, KID_PERMUTE, 2);
   }
   __syncthreads();
 }

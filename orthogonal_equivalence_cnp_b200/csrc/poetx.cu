@@ -811,26 +811,30 @@ int device_sms() {
   return sms[dev];
 }
 
-// Forward CNP of both sides of a b = 256 layer (one SM pair per block) with the input gather
-// U = X[:, pi_R] on the SMs the pairs leave free, in the same launch.  Returns false (nothing
+// CNP (forward or adjoint) of both sides of a b = 256 layer (one SM pair per block) with a bf16
+// column permutation on the SMs the pairs leave free, in the same launch: the forward's input
+// gather U = X[:, pi_R], the adjoint's scatter dX[:, pi_R] = dU.  Returns false (nothing
 // launched) where that does not fit: other block sizes, too few free SMs, rows too wide for the
 // launch's shared memory.
-bool cnp_fwd_with_gather(int b, int k, const CnpSide* sides, int nsides, const void* X, long ld_x, void* U, long ld_u,
-                         long rows, int cols, const int32_t* colmap, cudaStream_t st, poetx_status* status) {
+template <bool ADJ>
+bool cnp_with_permute(int b, int k, const CnpSide* sides, int nsides, const void* in, long ld_in, void* out,
+                      long ld_out, long rows, int cols, const int32_t* colmap, bool scatter, cudaStream_t st,
+                      poetx_status* status) {
   if (b != 256 || rows <= 0) return false;
   long nb_total = 0;
   for (int q = 0; q < nsides; ++q) nb_total += sides[q].nb;
   const long free_sms = (long)device_sms() - 2 * nb_total;
-  if (free_sms < 16 || cols > 8192 || cols % 8 || permute_bulk_smem_bytes<4>(cols) + 1024 > ChipCfg<256>::SMEM ||
-      !aligned16(X) || !aligned16(U) || !aligned16(colmap) || ld_x % 8 || ld_u % 8)
+  if (free_sms < 16 || cols > 8192 || cols % 8 ||
+      permute_bulk_smem_bytes<4, kSpareSlots>(cols) + 1024 > ChipCfg<256>::SMEM || !aligned16(in) ||
+      !aligned16(out) || !aligned16(colmap) || ld_in % 8 || ld_out % 8)
     return false;
   CnpGather g;
-  g.in = static_cast<const uint16_t*>(X); g.ld_in = ld_x;
-  g.out = static_cast<uint16_t*>(U); g.ld_out = ld_u;
-  g.rows = rows; g.cols = cols; g.colmap = colmap;
+  g.in = static_cast<const uint16_t*>(in); g.ld_in = ld_in;
+  g.out = static_cast<uint16_t*>(out); g.ld_out = ld_out;
+  g.rows = rows; g.cols = cols; g.colmap = colmap; g.scatter = scatter ? 1 : 0;
   const long groups = (rows + 3) / 4;
   g.nblk = (int)std::min<long>(free_sms & ~1L, (groups + 1) & ~1L);  // whole clusters of two
-  *status = launch_cnp_chip<256, false>(k, sides, nsides, st, &g);
+  *status = launch_cnp_chip<256, ADJ>(k, sides, nsides, st, &g);
   return true;
 }
 
@@ -1279,8 +1283,8 @@ poetx_status poetx_cnp_forward(const poetx_desc* desc, int n_tokens, const void*
   sides[0].nb = desc->d_out / b; sides[0].theta = theta_R; sides[0].Q = Q_R;
   sides[1].nb = desc->d_in / b; sides[1].theta = theta_P; sides[1].Q = Q_P;
   poetx_status st = POETX_OK;
-  if (cnp_fwd_with_gather(b, desc->k, sides, 2, X, desc->d_in, U, desc->d_in, n_tokens, desc->d_in, perm_R, stream,
-                          &st)) {
+  if (cnp_with_permute<false>(b, desc->k, sides, 2, X, desc->d_in, U, desc->d_in, n_tokens, desc->d_in, perm_R,
+                              false, stream, &st)) {
     POETX_TRY(st);
   } else {
     POETX_TRY(cnp_fwd_fused(b, desc->k, sides, 2, stream));
@@ -1348,21 +1352,25 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   if (fused_du) POETX_TRY(run_w_gemm(dt, g, Q_P, din, true, ws + w.dU, din, stream, POETX_KC_W_GEMM_ADJ));
   else POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream, POETX_KC_W_GEMM_ADJ));
   if (!fused_du) POETX_TRY(bd_backward(dt, n, din, b, ws + w.dV, Q_P, ws + w.dU, stream));
-  // Input side: dX[:, pi_R] = dU (side stream, after G_R); G_P partials (U saved or recomputed).
-  POETX_TRY(stream_edge(stream, side, ss->ev[2]));
-  POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, side));
+  // Input side: G_P partials (U saved or recomputed), then the CNP adjoint (packed gradients
+  // only), which also needs G_R's partials from the side stream.  The scatter dX[:, pi_R] = dU
+  // runs in the adjoint's launch on the SMs its pairs leave free (b = 256), else on the side
+  // stream from the moment dU exists.
+  if (cudaEventRecord(ss->ev[2], stream) != cudaSuccess) return POETX_ERR_CUDA;  // dU done
   POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
-  // CNP adjoint, packed gradients only: it needs G_R's partials from the side stream.  The
-  // scatter may still run beside it; the join at exit waits for it.
   if (cudaStreamWaitEvent(stream, ss->ev[1], 0) != cudaSuccess) return POETX_ERR_CUDA;
-  if (cnp_fused_ok(b, dt)) {
-    CnpSide sides[2];
-    sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + w.GpR);
-    sides[0].splits = w.sR; sides[0].grad = grad_theta_R;
-    sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + w.GpP);
-    sides[1].splits = w.sP; sides[1].grad = grad_theta_P;
-    return cnp_bwd_fused(b, desc->k, sides, 2, stream);
-  }
+  CnpSide sides[2];
+  sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + w.GpR);
+  sides[0].splits = w.sR; sides[0].grad = grad_theta_R;
+  sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + w.GpP);
+  sides[1].splits = w.sP; sides[1].grad = grad_theta_P;
+  poetx_status cst = POETX_OK;
+  if (cnp_fused_ok(b, dt) &&
+      cnp_with_permute<true>(b, desc->k, sides, 2, ws + w.dU, din, dX, din, n, din, perm_R, true, stream, &cst))
+    return cst;
+  if (cudaStreamWaitEvent(side, ss->ev[2], 0) != cudaSuccess) return POETX_ERR_CUDA;
+  POETX_TRY(permute_cols(dt, ws + w.dU, din, dX, din, n, din, perm_R, nullptr, true, side));
+  if (cnp_fused_ok(b, dt)) return cnp_bwd_fused(b, desc->k, sides, 2, stream);
   POETX_TRY(cnp_bwd_generic(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + w.GpR), w.sR,
                             grad_theta_R, ws + w.cnpR, stream));
   return cnp_bwd_generic(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + w.GpP), w.sP,

@@ -122,6 +122,19 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
       : "memory");
 }
 
+// 1-D bulk copy from this CTA's shared memory to a peer CTA's shared memory (both addresses
+// 16-byte aligned, size a multiple of 16); completion counted in bytes on the mbarrier `bar` of
+// the destination CTA (shared::cluster addresses from mapa_shared).  That barrier is the only
+// completion signal: the source may be overwritten once the destination has seen it complete.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+
 // ------------------------------------------------------------------------------------ tcgen05
 // TMEM allocation: executed by one whole warp; the allocated base address is written to smem.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
