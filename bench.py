@@ -620,55 +620,260 @@ def run_poetx(args):
         dist.destroy_process_group()
 
 
+# -------------------------------------------------------------------------- stacked workloads
+def run_stack(args):
+    """A whole Llama-shaped stack as one step: one CNP launch over every block of every linear
+    (the 13B stack, b = 512, runs it per transformer block: its CNP goes through the GEMM
+    kernels and their scratch), then the forward of all linears in order, then the backward of
+    all linears in reverse order (each with its CNP adjoint); the 13B stack's step ends with the
+    merge of every linear (fresh permutations, theta reset to zero).  Weights, parameters,
+    permutations and activations are seeded draws made on the device (torch's generator; the
+    host-side draws of the single-layer workloads would need tens of GB of host memory), with the
+    distributions of the single-layer workloads.  Inputs are far larger than L2."""
+    import torch
+
+    import orthogonal_equivalence_cnp_b200 as P
+    from orthogonal_equivalence_cnp_b200.layer import make_desc
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    cfg, nblk, shapes_fn = I.STACKS[args.workload]
+    layers = I.stack_layers(args.workload)
+    sh0 = layers[0][1]
+    N, b, k = sh0.n_tokens, sh0.b, sh0.k
+    bf = torch.bfloat16
+    gen = torch.Generator(device=dev)
+
+    def randn(shape, std, seed, dtype=bf):
+        gen.manual_seed(seed)
+        return (torch.randn(shape, generator=gen, device=dev, dtype=torch.float32) * std).to(dtype)
+
+    def randperm(n, seed):
+        gen.manual_seed(seed)
+        return torch.randperm(n, generator=gen, device=dev).to(torch.int32)
+
+    descs = [make_desc(sh.d_in, sh.d_out, sh.b, sh.k, sh.dtype, sh.mode) for _, sh, _ in layers]
+    nb_of = [sh.nb_out + sh.nb_in for _, sh, _ in layers]
+    off = np.concatenate([[0], np.cumsum(nb_of)]).astype(int)
+    nb_total = int(off[-1])
+    Pk = b * (b - 1) // 2
+    theta = randn((nb_total, Pk), sh0.theta_std, 17 + cfg, torch.float32)
+    grad = torch.empty_like(theta)
+    Q = torch.empty(nb_total, b, b, dtype=bf, device=dev)
+    W = [randn((sh.d_out, sh.d_in), sh.w_std, seed) for _, sh, seed in layers]
+    perms = [[randperm(sh.d_out, seed + 1), randperm(sh.d_in, seed + 2)] for _, sh, seed in layers]
+    new_perms = [[randperm(sh.d_out, seed + 10001), randperm(sh.d_in, seed + 10002)] for _, sh, seed in layers]
+    dims_in = sorted({sh.d_in for _, sh, _ in layers})
+    dims_out = sorted({sh.d_out for _, sh, _ in layers})
+    X = {d: randn((N, d), 1.0, 7 + d) for d in dims_in}
+    dX = {d: torch.empty(N, d, dtype=bf, device=dev) for d in dims_in}
+    dY = {d: randn((N, d), 1.0, 11 + d) for d in dims_out}
+    Y = {d: torch.empty(N, d, dtype=bf, device=dev) for d in dims_out}
+    fast = sh0.mode == "fast"
+    saved = [torch.empty(N * (sh.d_in + sh.d_out), dtype=bf, device=dev) if fast else None for _, sh, _ in layers]
+    ws_bytes = max(P.poetx_workspace_size(d, N) for d in descs)
+    per_block = len(layers) // nblk
+    cnp_chunks = [(0, nb_total)] if b <= 256 else [(int(off[i]), int(off[i + per_block]) - int(off[i]))
+                                                   for i in range(0, len(layers), per_block)]
+    ws_bytes = max(ws_bytes, max(P.poetx_cnp_blocks_workspace_size(descs[0], n) for _, n in cnp_chunks))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    merge = cfg == 5
+    stream = torch.cuda.current_stream()
+    buckets = None
+    if world > 1:  # the packed gradients of each run of layers are summed while the layers below run
+        from orthogonal_equivalence_cnp_b200.ddp import GradBuckets
+        buckets = GradBuckets(grad.view(-1), [n * Pk for n in nb_of])
+
+    def sl(t, i):  # slice of the flat block arrays for linear i: R side, then P side
+        _, sh, _ = layers[i]
+        a, m = int(off[i]), sh.nb_out
+        return t[a:a + m], t[a + m:a + m + sh.nb_in]
+
+    def cnp():
+        for a, n in cnp_chunks:
+            P.poetx_cnp_blocks(descs[0], n, theta[a:a + n], Q[a:a + n], ws)
+
+    def fwd_bwd():
+        for i, (_, sh, _) in enumerate(layers):
+            QR, QP = sl(Q, i)
+            P.poetx_forward(descs[i], N, X[sh.d_in], W[i], perms[i][0], perms[i][1], QR, QP, Y[sh.d_out], saved[i], ws)
+        for i in reversed(range(len(layers))):
+            _, sh, _ = layers[i]
+            QR, QP = sl(Q, i)
+            tR, tP = sl(theta, i)
+            gR, gP = sl(grad, i)
+            P.poetx_backward(descs[i], N, dY[sh.d_out], X[sh.d_in], W[i], perms[i][0], perms[i][1], QR, QP, tR, tP,
+                             saved[i], dX[sh.d_in], gR, gP, ws)
+            if buckets is not None:
+                buckets.layer_done(i)
+        if buckets is not None:
+            buckets.finish()
+
+    def do_merge():
+        for i in range(len(layers)):
+            QR, QP = sl(Q, i)
+            tR, tP = sl(theta, i)
+            P.poetx_merge(descs[i], W[i], QR, QP, perms[i][0], perms[i][1], new_perms[i][0], new_perms[i][1], tR, tP,
+                          ws)
+            perms[i], new_perms[i] = new_perms[i], perms[i]
+
+    def step():
+        cnp()
+        fwd_bwd()
+        if merge:
+            do_merge()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, det = P.poetx_device_status()
+    if st != 0:
+        raise RuntimeError(f"device-side timeout during warm-up ({det:#x})")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler()
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = P.poetx_launch_count()
+    for i in range(K):
+        ev[i][0].record(stream)
+        cnp()
+        ev[i][1].record(stream)
+        fwd_bwd()
+        ev[i][2].record(stream)
+        if merge:
+            do_merge()
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    launches = P.poetx_launch_count() - n0
+    clk = clocks.stop(gpu_uuid(dev))
+    st, det = P.poetx_device_status()
+    if st != 0:
+        raise RuntimeError(f"device-side timeout in the timed region ({det:#x})")
+    t_step = max_over_ranks(sum(ev[i][0].elapsed_time(ev[i][3]) for i in range(K)), world, dev) / K
+    t_cnp = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K
+    t_fb = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / K
+    t_merge = sum(ev[i][2].elapsed_time(ev[i][3]) for i in range(K)) / K
+    fl = sum(step_flops(sh)["total"] for _, sh, _ in layers)
+    f_merge = sum(4 * sh.b * sh.d_in * sh.d_out for _, sh, _ in layers) if merge else 0
+    peaks = read_peaks()
+    peak, hbm = float(peaks["bf16_tflops_sustained"]), float(peaks["hbm_gbs"])
+    cnp_bytes = nb_total * (4 * Pk + 2 * b * b)
+    out = {
+        "metric": METRIC,
+        "value": round(world * N / (t_step / 1e3), 1),
+        "unit": "tokens/s",
+        "tflops": round(world * (fl + f_merge) / (t_step / 1e3) / 1e12, 2),
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(t_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded draws on the device, torch generator)",
+        "config": {"workload": args.workload, "linears": len(layers), "blocks": nb_total, "b": b, "k": k,
+                   "n_tokens_per_gpu": N, "mode": sh0.mode,
+                   "step": "one CNP launch over all blocks + forward of every linear + backward of every linear"
+                           + (" + merge of every linear" if merge else ""),
+                   "l2": "inputs larger than L2", "launch": "direct launches",
+                   "parallelism": (f"dp{world}: replicas on their own tokens; packed gradients summed over the "
+                                   f"ranks in buckets of consecutive layers during the backward pass"
+                                   if world > 1 else "dp1"),
+                   "algorithmic_gflop_per_step": round(fl / 1e9, 1),
+                   "merge_gflop_per_step": round(f_merge / 1e9, 1)},
+        "step_roofline": {"t_flop_ms": round(fl / (peak * 1e12) * 1e3, 2),
+                          "frac": round(fl / (peak * 1e12) / ((t_step - t_merge) / 1e3), 4),
+                          "peak": peak, "peak_source": f"{peaks['source']} bf16_tflops_sustained",
+                          "note": "fwd + bwd + CNP FLOPs over the step time less the merge"},
+        "cnp": {"launches_per_step": len(cnp_chunks), "ms": round(t_cnp, 3), "blocks": nb_total,
+                "bytes": cnp_bytes, "hbm_frac": round(cnp_bytes / (t_cnp / 1e3) / 1e9 / hbm, 4)},
+        "fwd_bwd_ms": round(t_fb, 3),
+        "merge_ms": round(t_merge, 3) if merge else None,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------------- reference arm
 def run_reference(args):
     """The float64 oracle on the host cores.  Each step is a bounded sample of the workload, scaled
-    to it: the activation part of the step (forward chain and the backward chain up to G = dL/dQ)
-    on the first n tokens, and the CNP forward and adjoint of one block per side; the step time of
-    the whole workload is estimated as t_act * N / n + t_cnp * (blocks of both sides) / 2, which the
-    reported tokens/s divides N by.  n is chosen so that all steps take about two minutes."""
+    to it: for every linear of the sample, the activation part of the step (forward chain and the
+    backward chain up to G = dL/dQ) on the first n tokens, and the CNP forward and adjoint of one
+    block per side; the step time of the whole workload is estimated as the sum over the sample's
+    linears of t_act * N / n + t_cnp * (blocks of both sides) / 2, which the reported tokens/s
+    divides N by.  A single-layer workload is its own sample; a stacked workload's sample is its
+    first transformer block (7 linears), scaled by the number of blocks (extrapolated).  n is
+    chosen so that all steps take about two minutes."""
     import oracle as O
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    s = I.WORKLOADS[args.workload]
-    inp = I.make_workload(args.workload)
-    n_full = s.n_tokens
-    nb = s.nb_in + s.nb_out
-    W0p = O.absorb(inp.W0, inp.pi_L, inp.pi_R)  # layer state, outside the timing
-    Q_R, Q_P = O.cnp(inp.theta_R, s.b, s.k), O.cnp(inp.theta_P, s.b, s.k)
-    _, G_R, _ = O.backward_chain_G(inp.X[:16], inp.dY[:16], W0p, Q_R, Q_P, inp.pi_L, inp.pi_R, s.b)
+    if args.workload in I.STACKS:
+        _, nblk, _ = I.STACKS[args.workload]
+        chosen = I.stack_layers(args.workload)
+        chosen = [(sh, seed) for _, sh, seed in chosen[:len(chosen) // nblk]]
+        scale = nblk
+    else:
+        chosen, scale = [(I.WORKLOADS[args.workload], I.WORKLOAD_SEEDS[args.workload])], 1
+    n_full = chosen[0][0].n_tokens
+    n_cap = 256 if args.workload in I.STACKS else n_full  # host draws of the stacks' token rows stay small
+    prepared = []
+    for sh, seed in chosen:
+        inp = I.make_layer(sh, seed, n_tokens=min(n_full, n_cap))
+        W0p = O.absorb(inp.W0, inp.pi_L, inp.pi_R)  # layer state, outside the timing
+        Q_R, Q_P = O.cnp(inp.theta_R[:1], sh.b, sh.k), O.cnp(inp.theta_P[:1], sh.b, sh.k)
+        Q_R = np.repeat(Q_R, sh.nb_out, axis=0)  # every block's Q has the same cost; one is computed
+        Q_P = np.repeat(Q_P, sh.nb_in, axis=0)
+        _, G_R, _ = O.backward_chain_G(inp.X[:8], inp.dY[:8], W0p, Q_R, Q_P, inp.pi_L, inp.pi_R, sh.b)
+        prepared.append((sh, inp, W0p, Q_R, Q_P, G_R))
 
     def sample_step(n_tok):
-        X, dY = inp.X[:n_tok], inp.dY[:n_tok]
-        t0 = time.perf_counter()
-        O.forward_chain(X, W0p, Q_R, Q_P, inp.pi_L, inp.pi_R)
-        O.backward_chain_G(X, dY, W0p, Q_R, Q_P, inp.pi_L, inp.pi_R, s.b)
-        t1 = time.perf_counter()
-        for th in (inp.theta_R[:1], inp.theta_P[:1]):  # one block per side: CNP forward + adjoint
-            O.cnp(th, s.b, s.k)
-            O.cnp_grad(th, G_R[:1], s.b, s.k)
-        t2 = time.perf_counter()
-        return t1 - t0, t2 - t1
+        """Returns (raw activation seconds, raw CNP seconds, the step estimate for the workload)."""
+        ra = rc = est = 0.0
+        for sh, inp, W0p, Q_R, Q_P, G_R in prepared:
+            X, dY = inp.X[:n_tok], inp.dY[:n_tok]
+            t0 = time.perf_counter()
+            O.forward_chain(X, W0p, Q_R, Q_P, inp.pi_L, inp.pi_R)
+            O.backward_chain_G(X, dY, W0p, Q_R, Q_P, inp.pi_L, inp.pi_R, sh.b)
+            t1 = time.perf_counter()
+            for th in (inp.theta_R[:1], inp.theta_P[:1]):  # one block per side: CNP forward + adjoint
+                O.cnp(th, sh.b, sh.k)
+                O.cnp_grad(th, G_R[:1], sh.b, sh.k)
+            t2 = time.perf_counter()
+            ra += t1 - t0
+            rc += t2 - t1
+            est += (t1 - t0) * n_full / n_tok + (t2 - t1) * (sh.nb_in + sh.nb_out) / 2
+        return ra, rc, est * scale
 
-    ta, tc = sample_step(8)
+    ra, rc, _ = sample_step(8)
     budget = 120.0 / max(1, args.steps + args.warmup)
     n_tok = 8
-    while n_tok * 2 <= n_full and tc + ta * (n_tok * 2) / 8 <= budget:
+    n_max = min(n_full, n_cap)
+    while n_tok * 2 <= n_max and ra * (n_tok * 2) / 8 + rc <= budget:
         n_tok *= 2
     for _ in range(args.warmup):
         sample_step(n_tok)
-    t_act = t_cnp = 0.0
+    t_step = 0.0
     for _ in range(args.steps):
-        a, c = sample_step(n_tok)
-        t_act += a
-        t_cnp += c
-    t_step = (t_act * n_full / n_tok + t_cnp * nb / 2) / args.steps  # whole-workload step, estimated
+        t_step += sample_step(n_tok)[2]
+    t_step /= args.steps  # whole-workload step, estimated
     value = n_full / t_step
-    fl = step_flops(s)
-    sample = (f"per step: forward + backward activation chain on the first {n_tok} of {n_full} tokens and "
-              f"the CNP forward + adjoint of 1 block per side (of {nb}), float64 numpy; scaled to the full "
-              f"step as t_act*{n_full}/{n_tok} + t_cnp*{nb}/2")
+    fl = sum(step_flops(sh)["total"] for sh, *_ in prepared) * scale
+    what = (f"{len(prepared)} linears of the first of {scale} transformer blocks, extrapolated x{scale}"
+            if scale > 1 else "the layer")
+    sample = (f"per step: {what}: forward + backward activation chain on the first {n_tok} of {n_full} tokens and "
+              f"the CNP forward + adjoint of 1 block per side, float64 numpy; scaled to the full step as "
+              f"t_act*{n_full}/{n_tok} + t_cnp*(blocks of both sides)/2 per linear")
+    s0 = prepared[0][0]
     out = {
         "impl": "reference",
         "metric": METRIC,
@@ -683,9 +888,9 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded numpy draws, see poetx_inputs.py)",
-        "config": {"workload": args.workload, "d_in": s.d_in, "d_out": s.d_out, "b": s.b, "k": s.k,
-                   "n_tokens_per_gpu": s.n_tokens, "mode": s.mode,
-                   "algorithmic_gflop_per_step": round(fl["total"] / 1e9, 2)},
+        "config": {"workload": args.workload, "d_in": s0.d_in, "d_out": s0.d_out, "b": s0.b, "k": s0.k,
+                   "n_tokens_per_gpu": n_full, "mode": s0.mode,
+                   "algorithmic_gflop_per_step": round(fl / 1e9, 2)},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -699,7 +904,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
-    ap.add_argument("--workload", choices=sorted(I.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=sorted(I.WORKLOADS) + sorted(I.STACKS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-xq", dest="xq", action="store_false",
                     help="skip timing the POET-XQ (int8 W0') mem-mode step beside the bf16 mem-mode step")
@@ -711,6 +916,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload in I.STACKS:
+        run_stack(args)
     else:
         run_poetx(args)
 

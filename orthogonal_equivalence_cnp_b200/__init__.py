@@ -126,11 +126,50 @@ def exported_symbols():
 
 
 def _ptr(x):
+    """Device address of an array argument: a CUDA tensor (contiguous; checked), a raw device
+    address (int, the caller's responsibility) or None."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if not getattr(x, "is_cuda", False):
+        raise ValueError("array arguments must be CUDA tensors (or raw device addresses)")
+    if not x.is_contiguous():
+        raise ValueError("array arguments must be contiguous")
     return x.data_ptr()
+
+
+def _need(x, name, numel, dtype=None):
+    """Checks that tensor x (if it is one) holds at least `numel` elements of `dtype`; the library
+    cannot see sizes, so a short buffer would be written past its end."""
+    if x is None or isinstance(x, int):
+        return
+    import torch
+    if dtype is not None and x.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {x.dtype}")
+    if x.numel() < numel:
+        raise ValueError(f"{name}: needs at least {numel} elements, has {x.numel()}")
+
+
+def _act_dtype(desc):
+    import torch
+    return torch.bfloat16 if desc.dtype == POETX_BF16 else torch.float32
+
+
+def _check_layer(desc, n_tokens=0, **arrays):
+    """Size and type checks of the layer arrays by name (theta_*, Q_*, X, Y, dY, dX, W0p, perm_*)."""
+    import torch
+    b, din, dout, dt = desc.b, desc.d_in, desc.d_out, _act_dtype(desc)
+    P = b * (b - 1) // 2
+    need = {"theta_R": (dout // b * P, torch.float32), "theta_P": (din // b * P, torch.float32),
+            "grad_theta_R": (dout // b * P, torch.float32), "grad_theta_P": (din // b * P, torch.float32),
+            "Q_R": (dout * b, dt), "Q_P": (din * b, dt), "W0p": (dout * din, dt),
+            "X": (n_tokens * din, dt), "dX": (n_tokens * din, dt), "Y": (n_tokens * dout, dt),
+            "dY": (n_tokens * dout, dt), "perm_L": (dout, torch.int32), "perm_R": (din, torch.int32)}
+    for name, x in arrays.items():
+        key = name.replace("_old", "").replace("_new", "")
+        if key in need:
+            _need(x, name, *need[key])
 
 
 def _nbytes(x):
@@ -166,12 +205,21 @@ def poetx_cnp_blocks_workspace_size(desc: poetx_desc, n_blocks: int) -> int:
 
 
 def poetx_cnp(desc, theta_R, theta_P, Q_R, Q_P, workspace, ws_bytes=None, stream=None):
+    _check_layer(desc, theta_R=theta_R, theta_P=theta_P, Q_R=Q_R, Q_P=Q_P)
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_cnp(ctypes.byref(desc), _ptr(theta_R), _ptr(theta_P), _ptr(Q_R), _ptr(Q_P),
                            _ptr(workspace), ws_bytes, _stream(stream)), "poetx_cnp")
 
 
+def _check_blocks(desc, n_blocks, theta, Q):
+    import torch
+    b = desc.b
+    _need(theta, "theta", n_blocks * b * (b - 1) // 2, torch.float32)
+    _need(Q, "Q", n_blocks * b * b, _act_dtype(desc))
+
+
 def poetx_cnp_blocks(desc, n_blocks, theta, Q, workspace, ws_bytes=None, stream=None):
+    _check_blocks(desc, n_blocks, theta, Q)
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_cnp_blocks(ctypes.byref(desc), n_blocks, _ptr(theta), _ptr(Q), _ptr(workspace), ws_bytes,
                                   _stream(stream)), "poetx_cnp_blocks")
@@ -184,6 +232,9 @@ def poetx_absorb(desc, W0, perm_L, perm_R, W0p, stream=None):
 
 def poetx_forward(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, saved, workspace, ws_bytes=None,
                   stream=None):
+    _check_layer(desc, n_tokens, X=X, W0p=W0p, perm_L=perm_L, perm_R=perm_R, Q_R=Q_R, Q_P=Q_P, Y=Y)
+    if saved is not None and not isinstance(saved, int):
+        _need(saved, "saved", n_tokens * (desc.d_in + desc.d_out), _act_dtype(desc))
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0p), _ptr(perm_L), _ptr(perm_R),
                                _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(saved), _ptr(workspace), ws_bytes,
@@ -192,6 +243,10 @@ def poetx_forward(desc, n_tokens, X, W0p, perm_L, perm_R, Q_R, Q_P, Y, saved, wo
 
 def poetx_cnp_forward(desc, n_tokens, X, W0p, perm_L, perm_R, theta_R, theta_P, Q_R, Q_P, Y, saved, workspace,
                       ws_bytes=None, stream=None):
+    _check_layer(desc, n_tokens, X=X, W0p=W0p, perm_L=perm_L, perm_R=perm_R, theta_R=theta_R, theta_P=theta_P,
+                 Q_R=Q_R, Q_P=Q_P, Y=Y)
+    if saved is not None and not isinstance(saved, int):
+        _need(saved, "saved", n_tokens * (desc.d_in + desc.d_out), _act_dtype(desc))
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_cnp_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0p), _ptr(perm_L), _ptr(perm_R),
                                    _ptr(theta_R), _ptr(theta_P), _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(saved),
@@ -200,6 +255,8 @@ def poetx_cnp_forward(desc, n_tokens, X, W0p, perm_L, perm_R, theta_R, theta_P, 
 
 def poetx_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved, dX,
                    grad_theta_R, grad_theta_P, workspace, ws_bytes=None, stream=None):
+    _check_layer(desc, n_tokens, dY=dY, X=X, W0p=W0p, perm_L=perm_L, perm_R=perm_R, Q_R=Q_R, Q_P=Q_P,
+                 theta_R=theta_R, theta_P=theta_P, dX=dX, grad_theta_R=grad_theta_R, grad_theta_P=grad_theta_P)
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_backward(ctypes.byref(desc), n_tokens, _ptr(dY), _ptr(X), _ptr(W0p), _ptr(perm_L),
                                 _ptr(perm_R), _ptr(Q_R), _ptr(Q_P), _ptr(theta_R), _ptr(theta_P), _ptr(saved),
@@ -243,6 +300,8 @@ def poetx_wc_backward(desc, n_tokens, dY, X, W0p, perm_L, perm_R, Q_R, theta_R, 
 
 def poetx_merge(desc, W0p, Q_R, Q_P, perm_L_old, perm_R_old, perm_L_new, perm_R_new, theta_R, theta_P, workspace,
                 ws_bytes=None, stream=None):
+    _check_layer(desc, W0p=W0p, Q_R=Q_R, Q_P=Q_P, perm_L_old=perm_L_old, perm_R_old=perm_R_old,
+                 perm_L_new=perm_L_new, perm_R_new=perm_R_new, theta_R=theta_R, theta_P=theta_P)
     ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
     _check(lib().poetx_merge(ctypes.byref(desc), _ptr(W0p), _ptr(Q_R), _ptr(Q_P), _ptr(perm_L_old),
                              _ptr(perm_R_old), _ptr(perm_L_new), _ptr(perm_R_new), _ptr(theta_R), _ptr(theta_P),
@@ -294,6 +353,8 @@ def poetx_check_permutation(perm, n=None):
         addr = perm
     else:
         arr = np.ascontiguousarray(np.asarray(perm), dtype=np.int32)
+        if n is not None and n > arr.size:
+            raise ValueError(f"n = {n} exceeds the array's {arr.size} elements")
         perm, addr, n = arr, arr.ctypes.data, arr.size if n is None else n
     _check(lib().poetx_check_permutation(addr, n), "poetx_check_permutation")
 
@@ -334,6 +395,7 @@ def poetx_profile_summary():
 
 def poetx_cnp_blocks_noalloc(desc, n_blocks, theta, Q, stream=None):
     """CNP forward that takes no workspace (built-in 32 MiB device scratch; see include/poetx.h)."""
+    _check_blocks(desc, n_blocks, theta, Q)
     _check(lib().poetx_cnp_blocks_noalloc(ctypes.byref(desc), n_blocks, _ptr(theta), _ptr(Q), _stream(stream)),
            "poetx_cnp_blocks_noalloc")
 

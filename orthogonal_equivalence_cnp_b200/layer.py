@@ -111,14 +111,18 @@ class PoetxLayer:
                           self.Q_R, self.Q_P, self.Y, self.saved, self.ws)
         return self.Y
 
-    def step(self, X: torch.Tensor, dY: torch.Tensor):
-        """CNP forward + layer forward + layer backward (incl. the CNP adjoint)."""
+    def step(self, X: torch.Tensor, dY: torch.Tensor, grad_ready=None):
+        """CNP forward + layer forward + layer backward (incl. the CNP adjoint).  grad_ready (for
+        data parallelism, e.g. GradBuckets.layer_done of this layer) is called once the backward
+        pass, which writes the packed gradients, has been enqueued."""
         if self.xq:
             self.cnp()
             self.forward(X)
         else:
             self.cnp_forward(X)
         self.backward(dY, X)
+        if grad_ready is not None:
+            grad_ready()
 
     def optimizer_step(self, cfg: poetx_adamw_cfg):
         """AdamW on the packed theta (both sides in one launch)."""

@@ -176,3 +176,40 @@ def test_wait_probe_host_validation():
     assert L.poetx_test_wait_timeout(10, A, None) == 1            # below 1 us
     assert L.poetx_test_wait_timeout(10 ** 9, A, None) == 1       # above 100 ms
     assert L.poetx_test_wait_timeout(1_000_000, A + 2, None) == 3
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor in the binding's host-side checks (never reaches the library)."""
+
+    def __init__(self, numel, dtype, contiguous=True):
+        self._n, self.dtype, self._c = numel, dtype, contiguous
+        self.is_cuda = True
+
+    def numel(self):
+        return self._n
+
+    def is_contiguous(self):
+        return self._c
+
+    def data_ptr(self):
+        return 1 << 20
+
+
+def test_binding_checks_sizes_types_and_devices_before_calling():
+    import numpy as np
+    import torch
+    d = _desc(d_in=512, d_out=256, b=256, dtype=P.POETX_BF16)
+    P_ = 256 * 255 // 2
+    good_t = _FakeCuda(P_ * 3, torch.float32)
+    with pytest.raises(ValueError, match="theta"):
+        P.poetx_cnp_blocks(d, 3, _FakeCuda(P_ * 3 - 1, torch.float32), _FakeCuda(3 * 256 * 256, torch.bfloat16), None)
+    with pytest.raises(ValueError, match="Q"):
+        P.poetx_cnp_blocks_noalloc(d, 3, good_t, _FakeCuda(3 * 256 * 256, torch.float32))
+    with pytest.raises(ValueError, match="contiguous"):
+        P.poetx_cnp_blocks(d, 3, good_t, _FakeCuda(3 * 256 * 256, torch.bfloat16, contiguous=False), None)
+    with pytest.raises(ValueError, match="CUDA"):
+        P.poetx_cnp_blocks(d, 3, torch.zeros(P_ * 3), _FakeCuda(3 * 256 * 256, torch.bfloat16), None)
+    with pytest.raises(ValueError, match="X"):
+        P.poetx_forward(d, 64, _FakeCuda(64 * 512 - 8, torch.bfloat16), None, None, None, None, None, None, None, None)
+    with pytest.raises(ValueError, match="exceeds"):
+        P.poetx_check_permutation(np.arange(4, dtype=np.int32), 5)
