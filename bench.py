@@ -491,29 +491,37 @@ def run_poetx(args):
 
     # Comparator: the same step in the weight-centric order (form W = R W0 P first, then dense
     # products), captured and timed the same way (L2 flushed between steps, outside the interval).
-    wc_ms = None
-    if args.comparator:
-        layer.wc_step(X, dY)
+    wc_ms = fp_ms = None
+
+    def time_variant(fn):
+        """A comparator step captured and timed like the headline step (L2 flushed between steps,
+        outside the intervals)."""
+        fn(X, dY)
         torch.cuda.synchronize()
-        wgraph = None
+        vgraph = None
         if graph is not None:
-            wgraph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(wgraph):
-                layer.wc_step(X, dY)
+            vgraph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(vgraph):
+                fn(X, dY)
         Kc = min(K, 200)
         we0 = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
         we1 = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
         for i in range(Kc):
             flush.zero_()
             we0[i].record(stream)
-            if wgraph is not None:
-                wgraph.replay()
+            if vgraph is not None:
+                vgraph.replay()
             else:
-                layer.wc_step(X, dY)
+                fn(X, dY)
             we1[i].record(stream)
         torch.cuda.synchronize()
-        wc_ms = max_over_ranks(sum(we0[i].elapsed_time(we1[i]) for i in range(Kc)), world, dev) / Kc
-        del wgraph
+        del vgraph
+        return max_over_ranks(sum(we0[i].elapsed_time(we1[i]) for i in range(Kc)), world, dev) / Kc
+
+    if args.comparator:
+        wc_ms = time_variant(layer.wc_step)
+        if s.mode == "fast":
+            fp_ms = time_variant(layer.fourperm_step)
 
     xq = None
     if args.xq and s.dtype == "bf16" and s.d_in % 256 == 0 and s.d_out % 256 == 0:
@@ -593,7 +601,11 @@ def run_poetx(args):
                         "input_centric_speedup": round(wc_ms / (t_ms / K), 3),
                         "what": "same layer step with W = R W0 P formed first (original POET order): "
                                 "T = W0' BD_P, M = BD_R T, W permuted to the original basis, Y = X W^T; "
-                                "dX = dY W, dW = dY^T X, dM, gradients of Q from dM, CNP adjoint"}),
+                                "dX = dY W, dW = dY^T X, dM, gradients of Q from dM, CNP adjoint",
+                        "four_permutation_ms_per_step": None if fp_ms is None else round(fp_ms, 4),
+                        "two_permutation_speedup": None if fp_ms is None else round(fp_ms / (t_ms / K), 3),
+                        "four_permutation_what": "same step with none of the permutations absorbed: R and P around "
+                                                 "the original W0, four activation permutations per pass"}),
         "xq": xq,
         "optimizer": {"kernel": "adamw_kernel (packed theta_R + theta_P, one launch)", "params": int(n_par),
                       "us_per_launch": round(opt_ms * 1e3, 2),

@@ -253,6 +253,30 @@ poetx_status poetx_wc_backward(const poetx_desc* desc, int n_tokens, const void*
                                float* grad_theta_P, void* workspace, size_t ws_bytes,
                                poetx_stream stream);
 
+/* ----------------------------------------------------- four-permutation comparator (not the path)
+ * The same layer with none of the four permutations absorbed (replication review,
+ * "Reproducibility & code": the paper's Table 2 compares the 4-permute path with the 2-permute
+ * one; "Summary": absorbing two permutations into W is one of POET-X's reductions).  R and P act
+ * around the ORIGINAL base weight W0 [d_out, d_in] (not W0'), so each pass permutes the
+ * activations four times:
+ *   forward:  U = X[:, pi_R], V_i = U_i Q_P,i^T, V scattered back to the original basis by pi_R,
+ *             Z = V W0^T, Z' = Z[:, pi_L], Y'_i = Z'_i Q_R,i^T, Y[:, pi_L] = Y'
+ *   backward: the adjoints in reverse (four permutations), then the same CNP adjoint.
+ * Results equal poetx_forward / poetx_backward on W0' = Pi_L W0 Pi_R^T up to rounding.
+ *   saved  dtype [N*(d_out + d_in)]: Z' then U, written by the forward, read by the backward.
+ * Workspace: poetx_fourperm_workspace_size(desc, n_tokens) bytes.  Errors as for poetx_forward. */
+size_t poetx_fourperm_workspace_size(const poetx_desc* desc, int n_tokens);
+poetx_status poetx_fourperm_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0,
+                                    const int32_t* perm_L, const int32_t* perm_R, const void* Q_R,
+                                    const void* Q_P, void* Y, void* saved, void* workspace,
+                                    size_t ws_bytes, poetx_stream stream);
+poetx_status poetx_fourperm_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* W0,
+                                     const int32_t* perm_L, const int32_t* perm_R, const void* Q_R,
+                                     const void* Q_P, const float* theta_R, const float* theta_P,
+                                     const void* saved, void* dX, float* grad_theta_R,
+                                     float* grad_theta_P, void* workspace, size_t ws_bytes,
+                                     poetx_stream stream);
+
 /* ------------------------------------------------------------------ optimiser (packed theta)
  * AdamW on the packed skew parameters, so that the optimiser state stays at the packed size
  * (agidaily.cc article, compact storage: gradients and optimiser state shrink with the

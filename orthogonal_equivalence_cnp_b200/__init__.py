@@ -20,7 +20,8 @@ __all__ = [
     "poetx_cnp_blocks_noalloc", "poetx_adamw_cfg", "poetx_adamw_step",
     "poetx_adamw_reset", "poetx_wc_saved_size", "poetx_wc_workspace_size", "poetx_wc_forward", "poetx_wc_backward",
     "poetx_xq_quantize", "poetx_xq_dequantize", "poetx_xq_forward", "poetx_xq_backward", "poetx_xq_merge",
-    "poetx_check_permutation", "poetx_test_wait_timeout", "poetx_cnp_forward",
+    "poetx_check_permutation", "poetx_test_wait_timeout", "poetx_cnp_forward", "poetx_fourperm_workspace_size",
+    "poetx_fourperm_forward", "poetx_fourperm_backward",
 ]
 
 POETX_F32, POETX_BF16 = 0, 1
@@ -89,6 +90,9 @@ _SIGNATURES = {
     "poetx_xq_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_xq_merge": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_check_permutation": (_I, [_P, _I]),
+    "poetx_fourperm_workspace_size": (_SZ, [_D, _I]),
+    "poetx_fourperm_forward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "poetx_fourperm_backward": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "poetx_test_wait_timeout": (_I, [_LL, _P, _P]),
     "poetx_status_string": (ctypes.c_char_p, [_I]),
     "poetx_device_status": (_I, [ctypes.POINTER(ctypes.c_int)]),
@@ -402,3 +406,28 @@ def poetx_cnp_blocks_noalloc(desc, n_blocks, theta, Q, stream=None):
 
 def poetx_test_wait_timeout(limit_ns, returned, stream=None):
     _check(lib().poetx_test_wait_timeout(int(limit_ns), _ptr(returned), _stream(stream)), "poetx_test_wait_timeout")
+
+
+def poetx_fourperm_workspace_size(desc, n_tokens):
+    return lib().poetx_fourperm_workspace_size(ctypes.byref(desc), n_tokens)
+
+
+def poetx_fourperm_forward(desc, n_tokens, X, W0, perm_L, perm_R, Q_R, Q_P, Y, saved, workspace, ws_bytes=None,
+                           stream=None):
+    _check_layer(desc, n_tokens, X=X, W0p=W0, perm_L=perm_L, perm_R=perm_R, Q_R=Q_R, Q_P=Q_P, Y=Y)
+    _need(saved, "saved", n_tokens * (desc.d_in + desc.d_out), _act_dtype(desc))
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_fourperm_forward(ctypes.byref(desc), n_tokens, _ptr(X), _ptr(W0), _ptr(perm_L), _ptr(perm_R),
+                                        _ptr(Q_R), _ptr(Q_P), _ptr(Y), _ptr(saved), _ptr(workspace), ws_bytes,
+                                        _stream(stream)), "poetx_fourperm_forward")
+
+
+def poetx_fourperm_backward(desc, n_tokens, dY, W0, perm_L, perm_R, Q_R, Q_P, theta_R, theta_P, saved, dX,
+                            grad_theta_R, grad_theta_P, workspace, ws_bytes=None, stream=None):
+    _check_layer(desc, n_tokens, dY=dY, W0p=W0, perm_L=perm_L, perm_R=perm_R, Q_R=Q_R, Q_P=Q_P, theta_R=theta_R,
+                 theta_P=theta_P, dX=dX, grad_theta_R=grad_theta_R, grad_theta_P=grad_theta_P)
+    ws_bytes = _nbytes(workspace) if ws_bytes is None else ws_bytes
+    _check(lib().poetx_fourperm_backward(ctypes.byref(desc), n_tokens, _ptr(dY), _ptr(W0), _ptr(perm_L), _ptr(perm_R),
+                                         _ptr(Q_R), _ptr(Q_P), _ptr(theta_R), _ptr(theta_P), _ptr(saved), _ptr(dX),
+                                         _ptr(grad_theta_R), _ptr(grad_theta_P), _ptr(workspace), ws_bytes,
+                                         _stream(stream)), "poetx_fourperm_backward")

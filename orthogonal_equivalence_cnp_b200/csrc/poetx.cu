@@ -1606,6 +1606,126 @@ static poetx_status xq_dequantize(const poetx_desc* d, const int8_t* q, const fl
   return last_launch();
 }
 
+// --------------------------------------------------------- four-permutation comparator
+// The un-absorbed order: R = Pi_L^T BD_R Pi_L and P = Pi_R^T BD_P Pi_R are applied around the
+// original W0, so every pass permutes the activations four times (the pages' Table 2 sets this
+// against the two-permutation form of poetx_forward / poetx_backward):
+//   forward:  U = X[:, pi_R]; V = BD_P.U; Vo[:, pi_R] = V; Z = Vo.W0^T; Z' = Z[:, pi_L];
+//             Y' = BD_R.Z'; Y[:, pi_L] = Y'
+//   backward: dY' = dY[:, pi_L]; G_R = dY'^T Z'; dZ' = dY'.Q_R; dZ[:, pi_L] = dZ'; dVo = dZ.W0;
+//             dV = dVo[:, pi_R]; G_P = dV^T U; dU = dV.Q_P; dX[:, pi_R] = dU; CNP adjoint.
+// `saved` keeps Z' then U (as POET-Xfast's `saved`) from the forward for the backward.
+struct FpPlan {
+  size_t V, Vo, Z, Yp, dYp, dZp, dZ, dVo, dV, dU, GpR, GpP, cnpR, cnpP, total;
+  int sR, sP;
+};
+FpPlan fp_plan(const poetx_desc* d, long n) {
+  const size_t e = esize(d->dtype);
+  const int b = d->b, nbo = d->d_out / b, nbi = d->d_in / b;
+  FpPlan f;
+  Plan p;
+  f.V = p.take(n * d->d_in * e);
+  f.Vo = p.take(n * d->d_in * e);
+  f.Z = p.take(n * d->d_out * e);
+  f.Yp = p.take(n * d->d_out * e);
+  f.dYp = p.take(n * d->d_out * e);
+  f.dZp = p.take(n * d->d_out * e);
+  f.dZ = p.take(n * d->d_out * e);
+  f.dVo = p.take(n * d->d_in * e);
+  f.dV = p.take(n * d->d_in * e);
+  f.dU = p.take(n * d->d_in * e);
+  f.sR = grad_splits(d->dtype, n, nbo, b);
+  f.sP = grad_splits(d->dtype, n, nbi, b);
+  f.GpR = p.take((size_t)f.sR * nbo * b * b * 4);
+  f.GpP = p.take((size_t)f.sP * nbi * b * b * 4);
+  f.cnpR = p.take(cnp_bwd_ws(b, d->k, d->dtype, nbo));
+  f.cnpP = p.take(cnp_bwd_ws(b, d->k, d->dtype, nbi));
+  f.total = p.total;
+  return f;
+}
+
+size_t poetx_fourperm_workspace_size(const poetx_desc* desc, int n_tokens) {
+  if (check_desc(desc) != POETX_OK || n_tokens < 0) return 0;
+  return std::max(fp_plan(desc, n_tokens).total, cnp_layer_ws(desc));
+}
+
+poetx_status poetx_fourperm_forward(const poetx_desc* desc, int n_tokens, const void* X, const void* W0,
+                                    const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
+                                    void* Y, void* saved, void* workspace, size_t ws_bytes, poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
+  if (n_tokens == 0) return POETX_OK;
+  POETX_TRY(check_ptrs({X, W0, perm_L, perm_R, Q_R, Q_P, Y, saved}));
+  const FpPlan f = fp_plan(desc, n_tokens);
+  POETX_TRY(check_ws(workspace, ws_bytes, f.total));
+  char* ws = static_cast<char*>(workspace);
+  const int dt = desc->dtype, b = desc->b, din = desc->d_in, dout = desc->d_out;
+  const long n = n_tokens;
+  char* Zp = static_cast<char*>(saved);
+  char* U = Zp + (size_t)n * dout * esize(dt);
+  POETX_TRY(permute_cols(dt, X, din, U, din, n, din, perm_R, nullptr, false, stream));
+  POETX_TRY(bd_forward(dt, n, din, b, U, Q_P, ws + f.V, stream));
+  POETX_TRY(permute_cols(dt, ws + f.V, din, ws + f.Vo, din, n, din, perm_R, nullptr, true, stream));
+  GemmDesc g;
+  g.M = (int)n; g.N = dout; g.K = din;
+  g.A = view(ws + f.Vo, n, din, din);
+  g.B = view(W0, dout, din, din);
+  g.epi.d1 = ws + f.Z; g.epi.d1_dtype = dt; g.epi.ld1 = dout;
+  POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream));
+  POETX_TRY(permute_cols(dt, ws + f.Z, dout, Zp, dout, n, dout, perm_L, nullptr, false, stream));
+  POETX_TRY(bd_forward(dt, n, dout, b, Zp, Q_R, ws + f.Yp, stream));
+  return permute_cols(dt, ws + f.Yp, dout, Y, dout, n, dout, perm_L, nullptr, true, stream);
+}
+
+poetx_status poetx_fourperm_backward(const poetx_desc* desc, int n_tokens, const void* dY, const void* W0,
+                                     const int32_t* perm_L, const int32_t* perm_R, const void* Q_R, const void* Q_P,
+                                     const float* theta_R, const float* theta_P, const void* saved, void* dX,
+                                     float* grad_theta_R, float* grad_theta_P, void* workspace, size_t ws_bytes,
+                                     poetx_stream stream) {
+  POETX_TRY(check_desc(desc));
+  if (n_tokens < 0) return POETX_ERR_INVALID_ARG;
+  POETX_TRY(check_ptrs({theta_R, theta_P, grad_theta_R, grad_theta_P}));
+  const int b = desc->b, dt = desc->dtype, din = desc->d_in, dout = desc->d_out, nbo = dout / b, nbi = din / b;
+  if (n_tokens == 0) {
+    const size_t P = (size_t)b * (b - 1) / 2;
+    if (cudaMemsetAsync(grad_theta_R, 0, nbo * P * 4, stream) != cudaSuccess) return POETX_ERR_CUDA;
+    return cudaMemsetAsync(grad_theta_P, 0, nbi * P * 4, stream) == cudaSuccess ? POETX_OK : POETX_ERR_CUDA;
+  }
+  POETX_TRY(check_ptrs({dY, W0, perm_L, perm_R, Q_R, Q_P, saved, dX}));
+  const FpPlan f = fp_plan(desc, n_tokens);
+  POETX_TRY(check_ws(workspace, ws_bytes, f.total));
+  char* ws = static_cast<char*>(workspace);
+  const long n = n_tokens;
+  const char* Zp = static_cast<const char*>(saved);
+  const char* U = Zp + (size_t)n * dout * esize(dt);
+  POETX_TRY(permute_cols(dt, dY, dout, ws + f.dYp, dout, n, dout, perm_L, nullptr, false, stream));
+  POETX_TRY(block_grads(dt, n, dout, b, ws + f.dYp, Zp, reinterpret_cast<float*>(ws + f.GpR), f.sR, stream));
+  POETX_TRY(bd_backward(dt, n, dout, b, ws + f.dYp, Q_R, ws + f.dZp, stream));
+  POETX_TRY(permute_cols(dt, ws + f.dZp, dout, ws + f.dZ, dout, n, dout, perm_L, nullptr, true, stream));
+  GemmDesc g;
+  g.M = (int)n; g.N = din; g.K = dout;
+  g.A = view(ws + f.dZ, n, dout, dout);
+  g.B = view(W0, dout, din, din); g.b_mn = true;
+  g.epi.d1 = ws + f.dVo; g.epi.d1_dtype = dt; g.epi.ld1 = din;
+  POETX_TRY(run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, stream, POETX_KC_W_GEMM_ADJ));
+  POETX_TRY(permute_cols(dt, ws + f.dVo, din, ws + f.dV, din, n, din, perm_R, nullptr, false, stream));
+  POETX_TRY(block_grads(dt, n, din, b, ws + f.dV, U, reinterpret_cast<float*>(ws + f.GpP), f.sP, stream));
+  POETX_TRY(bd_backward(dt, n, din, b, ws + f.dV, Q_P, ws + f.dU, stream));
+  POETX_TRY(permute_cols(dt, ws + f.dU, din, dX, din, n, din, perm_R, nullptr, true, stream));
+  if (cnp_fused_ok(b, dt)) {
+    CnpSide sides[2];
+    sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + f.GpR);
+    sides[0].splits = f.sR; sides[0].grad = grad_theta_R;
+    sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + f.GpP);
+    sides[1].splits = f.sP; sides[1].grad = grad_theta_P;
+    return cnp_bwd_fused(b, desc->k, sides, 2, stream);
+  }
+  POETX_TRY(cnp_bwd_generic(b, desc->k, dt, nbo, theta_R, reinterpret_cast<const float*>(ws + f.GpR), f.sR,
+                            grad_theta_R, ws + f.cnpR, stream));
+  return cnp_bwd_generic(b, desc->k, dt, nbi, theta_P, reinterpret_cast<const float*>(ws + f.GpP), f.sP,
+                         grad_theta_P, ws + f.cnpP, stream);
+}
+
 poetx_status poetx_xq_quantize(const poetx_desc* desc, const void* W0p, int8_t* W0q, float* W0s,
                                poetx_stream stream) {
   POETX_TRY(check_xq(desc));

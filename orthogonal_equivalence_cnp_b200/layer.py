@@ -9,7 +9,8 @@ import numpy as np
 import torch
 
 from . import (POETX_BF16, POETX_F32, POETX_FAST, POETX_MEM, poetx_absorb, poetx_adamw_cfg, poetx_adamw_reset,
-               poetx_adamw_step, poetx_backward, poetx_cnp, poetx_cnp_forward, poetx_desc, poetx_forward,
+               poetx_adamw_step, poetx_backward, poetx_cnp, poetx_cnp_forward, poetx_desc, poetx_fourperm_backward,
+               poetx_fourperm_forward, poetx_fourperm_workspace_size, poetx_forward,
                poetx_merge, poetx_wc_backward, poetx_wc_forward, poetx_wc_saved_size, poetx_wc_workspace_size,
                poetx_workspace_size, poetx_xq_backward, poetx_xq_forward, poetx_xq_merge, poetx_xq_quantize)
 
@@ -72,6 +73,7 @@ class PoetxLayer:
         self.theta_P.copy_(torch.from_numpy(np.asarray(theta_P, np.float32)))
         W0_dev = self.to_dev(W0)
         poetx_absorb(self.desc, W0_dev, self.perm_L, self.perm_R, self.W0p)
+        self.W0 = W0_dev  # the un-absorbed weight, kept for the four-permutation comparator
 
     # ------------------------------------------------------------------------- the step
     def cnp(self):
@@ -146,6 +148,20 @@ class PoetxLayer:
                        torch.from_numpy(np.asarray(pR, np.int32)).to(self.device))
             poetx_adamw_reset(self.m.numel(), self.m, self.v)
             self.t = 0
+
+    def fourperm_step(self, X: torch.Tensor, dY: torch.Tensor):
+        """The same step with none of the permutations absorbed (comparator): R and P applied around
+        the original W0, four activation permutations per pass.  Same outputs as step()."""
+        if getattr(self, "fp_saved", None) is None:
+            self.fp_saved = torch.empty(self.n * (self.desc.d_in + self.desc.d_out), dtype=self.dtype,
+                                        device=self.device)
+            self.fp_ws = torch.empty(max(poetx_fourperm_workspace_size(self.desc, self.n), 256), dtype=torch.uint8,
+                                     device=self.device)
+        poetx_cnp(self.desc, self.theta_R, self.theta_P, self.Q_R, self.Q_P, self.fp_ws)
+        poetx_fourperm_forward(self.desc, self.n, X, self.W0, self.perm_L, self.perm_R, self.Q_R, self.Q_P, self.Y,
+                               self.fp_saved, self.fp_ws)
+        poetx_fourperm_backward(self.desc, self.n, dY, self.W0, self.perm_L, self.perm_R, self.Q_R, self.Q_P,
+                                self.theta_R, self.theta_P, self.fp_saved, self.dX, self.g_R, self.g_P, self.fp_ws)
 
     def wc_step(self, X: torch.Tensor, dY: torch.Tensor):
         """The same step in the weight-centric order (comparator): CNP, form W = R W0 P, Y = X W^T,
