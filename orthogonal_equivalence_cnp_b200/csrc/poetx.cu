@@ -117,18 +117,31 @@ struct LaunchScope {
 // be scheduled while that one finishes and waits for it in griddep_wait() before touching its
 // results (every kernel of this library does).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+cudaError_t launch_pdl_prio(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool high,
+                            Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (high) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess) {
+      attr[1].id = cudaLaunchAttributePriority;
+      attr[1].val.priority = greatest;
+      cfg.numAttrs = 2;
+    }
+  }
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  return launch_pdl_prio(kern, grid, block, smem, st, false, args...);
 }
 
 poetx_status check_desc(const poetx_desc* d) {
@@ -467,7 +480,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.bscale = g.b_scale;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(cls, st);
-  if (launch_pdl(kern, grid, dim3(Q8 ? 128 + TCW_CONV_THREADS : 128), smem, st, ta, tb, tq, td, a) != cudaSuccess)
+  if (launch_pdl_prio(kern, grid, dim3(Q8 ? 128 + TCW_CONV_THREADS : 128), smem, st, true, ta, tb, tq, td, a) != cudaSuccess)
     return POETX_ERR_CUDA;
   return last_launch();
 }
@@ -550,12 +563,18 @@ int grad_splits(int dt, long n, int nb, int b) {
 }
 
 poetx_status block_grads(int dt, long n, int d, int b, const void* lhs, const void* rhs, float* part, int splits,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool few_ctas = false) {
   GemmDesc g;
   g.M = b; g.N = b; g.K = (int)n; g.batch = d / b; g.splits = splits;
   g.A = view(lhs, n, d, d, 0, b); g.a_mn = true;
   g.B = view(rhs, n, d, d, 0, b); g.b_mn = true;
   g.epi.d1 = part; g.epi.d1_dtype = F32; g.epi.ld1 = b; g.epi.zrow1 = b; g.epi.split_stride1 = (long)d * b;
+  // few_ctas: the widest tile and the deep ring whatever the CTA count, for a launch that runs
+  // beside a GEMM on the SMs that one leaves free.
+  if (few_ctas && dt == BF16 && b % 256 == 0) {
+    POETX_TRY(check_gemm(g, dt));
+    return launch_tc_major<256, 4>(g, st, POETX_KC_GRAD_GEMM);
+  }
   return run_gemm(dt, g, st, POETX_KC_GRAD_GEMM);
 }
 
@@ -902,7 +921,7 @@ BwdPlan bwd_plan(const poetx_desc* d, long n) {
   w.dU = p.take(n * d->d_in * e);
   w.V = d->mode == POETX_MEM ? p.take(n * d->d_in * e) : 0;
   w.Z = d->mode == POETX_MEM ? p.take(n * d->d_out * e) : 0;
-  w.sR = grad_splits(d->dtype, n, nbo, b);
+  w.sR = d->dtype == BF16 && b == 256 ? 1 : grad_splits(d->dtype, n, nbo, b);
   w.sP = grad_splits(d->dtype, n, nbi, b);
   w.GpR = p.take((size_t)w.sR * nbo * b * b * 4);
   w.GpP = p.take((size_t)w.sP * nbi * b * b * 4);
@@ -1336,11 +1355,11 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   // BD_R^T-adjoint (both read dY', so it is shared through L2), leaving the W0' GEMM below the
   // whole GPU.
   POETX_TRY(permute_cols(dt, dY, dout, ws + w.dYp, dout, n, dout, perm_L, nullptr, false, stream));
+  POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
   POETX_TRY(stream_edge(stream, side, ss->ev[0]));
   SideJoin join{stream, side, ss->ev[3], true};
-  POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, side));
+  POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, side, w.sR == 1));
   if (cudaEventRecord(ss->ev[1], side) != cudaSuccess) return POETX_ERR_CUDA;  // G_R partials done
-  POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
   // dV = dZ . W0' (and, for b = 256, dU_i = dV_i . Q_P,i in the same kernel)
   GemmDesc g;
   g.M = (int)n; g.N = din; g.K = dout;
