@@ -578,8 +578,11 @@ constexpr int TCW_BM = 256, TCW_BN = 256, TCW_STAGES = 3;
 constexpr uint32_t TCW_Q8_TILE = 256 * TC_BK;  // int8 codes of one k step's B tile
 constexpr int TCW_CONV_THREADS = 256;           // Q8 converter warps 4..11
 constexpr int TCW_CONV_CHUNKS = 2048 / TCW_CONV_THREADS;  // 8-code chunks per converter thread per k step
+// Past the ring: the block-factor result's store staging, two 32-row x 64-column boxes per
+// epilogue warp, so that it leaves through TMA stores while the ring still holds Q and D.
+constexpr uint32_t TCW_OUT_BYTES = 4 * 2 * 4096;
 __host__ __device__ constexpr size_t tcw_smem_bytes() {
-  return (size_t)TCW_STAGES * (TCW_BM * TC_BK * 2 + TCW_BN * TC_BK * 2) + 1024 + 256;
+  return (size_t)TCW_STAGES * (TCW_BM * TC_BK * 2 + TCW_BN * TC_BK * 2) + TCW_OUT_BYTES + 1024 + 256;
 }
 
 // Named barrier 1 over the `count` threads of the converter warps, ANDing p across them: every
@@ -601,7 +604,7 @@ template <bool B_MN, bool Q_MN, bool Q8 = false>
 __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
     gemm_w256_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmD,
-                 const WideArgs args) {
+                 const __grid_constant__ CUtensorMap tmO, const WideArgs args) {
   constexpr int BN = TCW_BN, STAGES = TCW_STAGES;
   constexpr uint32_t HALF_A = TC_BM * TC_BK * 2;     // 16 KiB: one 128-row half of an A tile
   constexpr uint32_t A_BYTES = 2 * HALF_A;
@@ -613,7 +616,7 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + TCW_OUT_BYTES);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
   const uint32_t smem0 = smem_u32(smem);
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -646,7 +649,10 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
     fence_proxy_async_smem();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (fuse) prefetch_tmap(&tmQ);
+    if (fuse) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmO);
+    }
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_holder), 2 * BN);
@@ -844,25 +850,11 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
       store_half(1, 1);
     }
   } else {
+    // Half h: D_h -> the D stage (bf16, K-major swizzled) -> global d1 by TMA, and the A operand
+    // of the block-factor product, whose result lands in the half's own TMEM columns.  The result
+    // of half 0 is drained to TMA-store boxes while the product of half 1 runs.
     bool ok2 = ok;
-#pragma unroll 1
-    for (int h = 0; h < 2; ++h) {
-      // D half h -> the D stage (free: the K loop is done, and for h = 1 the previous half's
-      // products and D stores have finished reading it) -> global d1 by TMA.  The block-factor
-      // result of half h lands in the half's own TMEM columns and is stored from registers.
-      if (h == 1) {
-        if (threadIdx.x == 0) bulk_wait_read<0>();
-        __syncthreads();
-      }
-      if (ok2 && epi_warp) {
-        if (h == 1) drain(0, m0 + r, args.out2, args.ld2, -1);  // first half's result
-        drain((uint32_t)(h * BN), m0 + h * TC_BM + r, nullptr, 0, sdh);
-      }
-      fence_proxy_async_smem();  // the tensor core and the TMA engine read what the threads wrote
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-      if (ok2) store_half(sdh, h);
+    auto block_product = [&](int h) {
       if (warp == 1 && lane == 0 && ok2) {
         if (mbar_wait(q_full, 0, KID_GEMM_TC, 15)) {
           tc_fence_after();
@@ -881,11 +873,68 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
         mma_commit(acc2_bar);
       }
       __syncwarp();
+    };
+    auto wait_product = [&](int h) {
       if (ok2) ok2 = mbar_wait(acc2_bar, (uint32_t)h, KID_GEMM_TC, 16);
       ok2 = __all_sync(0xffffffffu, ok2);
       tc_fence_after();
-    }
-    if (ok2 && epi_warp) drain(BN, m0 + TC_BM + r, args.out2, args.ld2, -1);
+    };
+    // The block-factor result of half h (TMEM columns col0..): 32-row x 64-column boxes per warp
+    // through two staging buffers, stored with TMA (rows past M clipped by the map).
+    int nbox = 0;
+    uint8_t* ostage = smem + STAGES * STAGE_BYTES + warp * 8192;
+    auto drain_out = [&](uint32_t col0, int h) {
+#pragma unroll 1
+      for (int c64 = 0; c64 < BN / 64; ++c64, ++nbox) {
+        uint8_t* buf = ostage + (nbox & 1) * 4096;
+        if (nbox >= 2) {
+          if (lane == 0) bulk_wait_read<1>();  // the store two boxes back has read this buffer
+          __syncwarp();
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(c64 * 64 + hh * 32), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = 8 * u;
+            const uint4 q = make_uint4(pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                                       pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])),
+                                       pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5])),
+                                       pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7])));
+            const int ch = hh * 4 + u;
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((ch ^ (lane & 7)) * 16)) = q;
+          }
+        }
+        fence_proxy_async_smem();  // the TMA engine reads what the threads wrote
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmO, smem_u32(buf), n0 + c64 * 64, m0 + h * TC_BM + warp * 32);
+          bulk_commit();
+        }
+      }
+    };
+    auto stage_d = [&](int h) {
+      if (ok2 && epi_warp) drain((uint32_t)(h * BN), m0 + h * TC_BM + r, nullptr, 0, sdh);
+      fence_proxy_async_smem();  // the tensor core and the TMA engine read what the threads wrote
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (ok2) store_half(sdh, h);
+    };
+    stage_d(0);
+    block_product(0);
+    wait_product(0);
+    if (threadIdx.x == 0) bulk_wait_read<0>();  // D_0's stores have read the D stage
+    __syncthreads();
+    stage_d(1);
+    block_product(1);
+    if (ok2 && epi_warp) drain_out(0, 0);  // beside the second product (other TMEM columns)
+    wait_product(1);
+    if (ok2 && epi_warp) drain_out(BN, 1);
+    if (epi_warp && lane == 0) bulk_wait_read<0>();
+    __syncwarp();
   }
   // Shared memory stays valid until the stores have read it (the writes complete with the grid).
   if (threadIdx.x == 0) bulk_wait_read<0>();

@@ -458,7 +458,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
     if (!set_smem(kern, smem)) return POETX_ERR_CUDA;
     attr_done[dev] = true;
   }
-  CUtensorMap ta, tb, tq, td;
+  CUtensorMap ta, tb, tq, td, to;
   if (!make_tmap(&ta, g.A, 64, TCW_BM)) return POETX_ERR_CUDA;
   if (Q8) {
     // int8 codes: a 64 (k) x 256 (n) box of the K-major array, or 256 (n) x 64 (k) of the MN-major one.
@@ -470,8 +470,11 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   if (!make_tmap(&td, view(g.epi.d1, g.M, g.N, g.epi.ld1), 64, TC_BM)) return POETX_ERR_CUDA;
   if (out2 != nullptr) {
     if (!make_tmap(&tq, view(Q, q_rows, 256, 256), 64, QMN ? 64 : 256)) return POETX_ERR_CUDA;
+    // Store boxes of the block-factor result: 64 columns x 32 rows (one warp's rows).
+    if (!make_tmap(&to, view(out2, g.M, g.N, ld2), 64, 32)) return POETX_ERR_CUDA;
   } else {
     tq = ta;  // unused without the block factor
+    to = ta;
   }
   WideArgs a;
   a.M = g.M; a.N = g.N; a.K = g.K;
@@ -480,7 +483,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.bscale = g.b_scale;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(cls, st);
-  if (launch_pdl_prio(kern, grid, dim3(Q8 ? 128 + TCW_CONV_THREADS : 128), smem, st, true, ta, tb, tq, td, a) != cudaSuccess)
+  if (launch_pdl_prio(kern, grid, dim3(Q8 ? 128 + TCW_CONV_THREADS : 128), smem, st, true, ta, tb, tq, td, to, a) != cudaSuccess)
     return POETX_ERR_CUDA;
   return last_launch();
 }
