@@ -32,7 +32,8 @@
 //   R_k = G, R_a = 2G + R_{a+1} T           (right factors: operands are own rows)
 //   L_k = G, L_a = R_a + T L_{a+1},  G_S = L_0   (left factor T: L in B form, quadrant exchange)
 // L_a accumulates onto R_a in the same TMEM columns.  PACK transposes G_S through shared memory
-// (the pair's off-diagonal quadrant crosses over once) and writes the packed rows coalesced.
+// (half of the pair's off-diagonal quadrant crosses over each way, so that both CTAs write the
+// same number of packed entries) and writes the packed rows coalesced.
 //
 // Synchronisation.  One thread of the (even) CTA issues every product once all epilogue warps
 // of the pair have arrived on its `ready` barrier (release at cluster scope after their shared
@@ -71,7 +72,8 @@ struct ChipCfg {
   static constexpr size_t SMEM = BAR_OFF + 256 + 1024;
   static_assert((size_t)(B / 32) * GBOX <= 2 * (size_t)REG, "G staging fits V1 + V2");
   static_assert((size_t)B * (B - 1) / 2 * 4 <= 2 * (size_t)REG, "theta staging fits V1 + V2");
-  static_assert((size_t)(PAIR ? 2 : 1) * QN * QPITCH * 4 <= BAR_OFF, "PACK quadrants fit below the barriers");
+  // PACK: Qd, and for a pair three 128 x 64 half quadrants (received, sent, kept) of 68-float rows.
+  static_assert((size_t)QN * QPITCH * 4 + (PAIR ? 3 * 128 * 68 * 4 : 0) <= BAR_OFF, "PACK staging fits below the barriers");
 };
 
 struct CnpChipSide {
@@ -162,6 +164,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
   const int c0 = half * C::HALF;              // first column of this thread's half
   auto ro = [](int x) { return x * B - (x * (x + 1)) / 2 - x - 1; };  // packed (x, y) at ro(x) + y
 
+  const bool need_s = !ADJ || k >= 1;
   if (threadIdx.x == 0) {
     mbar_init(bar_mma, 1);
     mbar_init(bar_ready, 8 * C::NCTA);
@@ -169,6 +172,17 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     mbar_init(bar_g, 1);
     mbar_init(bar_xin, 1);
     fence_mbar_init();
+    if (need_s) {
+      // The block's packed theta (8 bulk copies into V1 + V2) is requested first, so that the
+      // TMEM allocation and the cluster barrier below overlap the copy.
+      griddep_wait();  // theta may come from the previous kernel (an optimiser step)
+      const uint32_t bytes = (uint32_t)(P * 4);  // 16-byte multiple for b % 8 == 0
+      mbar_arrive_expect_tx(bar_theta, bytes);
+      const uint32_t chunk = ((bytes / 8) + 15) & ~15u;
+#pragma unroll 1
+      for (uint32_t off = 0; off < bytes; off += chunk)
+        bulk_load_1d(V1 + off, reinterpret_cast<const char*>(SD.theta + z * P) + off, min(chunk, bytes - off), bar_theta);
+    }
   }
   if (warp == 0) {
     if constexpr (C::PAIR) {
@@ -316,17 +330,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
   };
 
   // ---------------------------------------------------------------- theta -> S (Sc, REG2)
-  const bool need_s = !ADJ || k >= 1;
   if (need_s) {
-    if (warp == 0) {
-      const uint32_t bytes = (uint32_t)(P * 4);  // 16-byte multiple for b % 8 == 0
-      if (lane == 0) mbar_arrive_expect_tx(bar_theta, bytes);
-      __syncwarp();
-      const uint32_t chunk = ((bytes / 8) + 15) & ~15u;
-      const uint32_t off = (uint32_t)lane * chunk;
-      if (lane < 8 && off < bytes)
-        bulk_load_1d(V1 + off, reinterpret_cast<const char*>(SD.theta + z * P) + off, min(chunk, bytes - off), bar_theta);
-    }
     if (ok) ok = mbar_wait(bar_theta, 0, KID_CNP_CHIP, 1);
     ok = __all_sync(0xffffffffu, ok);
     const float* th = reinterpret_cast<const float*>(smem + C::REG);
@@ -490,31 +494,43 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     }
     uint32_t fcol = REG2;  // the TMEM columns holding G_S for PACK
     if (k >= 1) {
+      // Each product is issued as soon as its operands are in place; the rest of an epilogue (the
+      // bf16 copies that only a later product reads, and the exchange) runs beside it:
+      //   R_a = ACC + 2G goes back into ACC first (MMA_L accumulates onto it), its A form into V1
+      //   while MMA_L runs; L_a is read out of ACC, then MMA_R of the next level may overwrite ACC
+      //   while L_a's B form is written and exchanged.
+      constexpr int NCH = C::HALF / 32;  // 32-column chunks per thread
       fcol = ACC;
+      arrive_ready();
+      issue(V1, SC, false, false, false, 6);  // ACC = R_k . S^T = R_k T
 #pragma unroll 1
       for (int a = k - 1; a >= 0; --a) {
-        arrive_ready();
-        issue(V1, SC, false, false, false, 6);  // ACC = R_{a+1} . S^T = R_{a+1} T
         wait_mma(7);
-#pragma unroll 1
-        for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
-          float d[32], g[32];
-          tld2(ACC + j0, d, REG2 + j0, g);
+        float rv[NCH][32];
 #pragma unroll
-          for (int u = 0; u < 32; ++u) d[u] += 2.f * g[u];  // R_a
-          tst(ACC + j0, d);
-          if (a > 0) chip_put_aform(V1, r, j0, d);
+        for (int q = 0; q < NCH; ++q) {
+          float g[32];
+          tld2(ACC + c0 + 32 * q, rv[q], REG2 + c0 + 32 * q, g);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) rv[q][u] += 2.f * g[u];  // R_a
+          tst(ACC + c0 + 32 * q, rv[q]);
         }
-        arrive_ready(true);  // MMA_L reads V2 = L_{a+1}, the B form exchanged after its epilogue
+        arrive_ready(true);  // ACC = R_a; MMA_L reads V2 = L_{a+1}, the B form exchanged after its epilogue
         issue(SC, V2, true, true, true, 8, true);  // ACC += (-S) . L_{a+1} = T L_{a+1}
+        if (a > 0) {
+#pragma unroll
+          for (int q = 0; q < NCH; ++q) chip_put_aform(V1, r, c0 + 32 * q, rv[q]);  // R_a for the next level
+        }
         wait_mma(9);
         if (a > 0) {
-#pragma unroll 1
-          for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
-            float l[32];
-            tld(ACC + j0, l);
-            if (valid) put_bform(V2, j0, l);
-          }
+          float lv[NCH][32];
+#pragma unroll
+          for (int q = 0; q < NCH; ++q) tld(ACC + c0 + 32 * q, lv[q]);  // L_a
+          arrive_ready();  // L_a is out of ACC and R_a is in V1
+          issue(V1, SC, false, false, false, 6);  // ACC = R_a . S^T = R_a T (next level)
+#pragma unroll
+          for (int q = 0; q < NCH; ++q)
+            if (valid) put_bform(V2, c0 + 32 * q, lv[q]);
           send_bform(V2);
         }
       }
@@ -523,70 +539,98 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     }
     griddep_launch();
     // ---------------------------------------------------------------------------- PACK
-    // g[p(i,j)] = G_S[i][j] - G_S[j][i] for i < j, computed by the thread that owns row j of G_S
-    // (it holds G_S[j][i] in TMEM) from a row-major copy of the rows i in shared memory, so that
-    // each packed row p(i, .) leaves as coalesced stores along j.  Quadrants (QN x QN, rows of
-    // QPITCH floats, written with 16-byte stores): Qd = G_S[O_c][O_c] of this CTA; for a pair,
-    // CTA 1 also receives Qx = G_S[O_0][O_1] from CTA 0 and handles the packed entries of that
-    // quadrant (rows i in O_0, columns j in O_1).
+    // g[p(i,j)] = G_S[i][j] - G_S[j][i] for i < j, written along j (lanes take consecutive j) so
+    // that every packed row p(i, .) leaves as coalesced stores.  Qd = G_S[O_c][O_c] (QN x QN, rows
+    // of QPITCH floats) is staged by the threads holding it; the thread owning row j of a diagonal
+    // quadrant reads G_S[j][i] from TMEM and G_S[i][j] from Qd.  For a pair, the cross quadrant
+    // (i in O_0, j in O_1) is split in two halves of 64 columns j, one per CTA, so that both do the
+    // same amount of work: CTA 1 takes j in [128, 192) (G_S[j][i] from its TMEM, G_S[i][j] sent by
+    // CTA 0), CTA 0 takes j in [192, 256) (G_S[i][j] staged from its TMEM, G_S[j][i] sent by CTA 1
+    // transposed).  Both halves cross in one bulk copy each way (XPITCH-float rows).
     {
-      const uint32_t QD = s0, QX = s0 + (uint32_t)(C::QN * C::QPITCH * 4);
+      constexpr int XPITCH = 68;                            // 64 columns + 4 (16-byte rows)
+      constexpr uint32_t XBYTES = 128u * XPITCH * 4u;       // one 128 x 64 half quadrant
+      const uint32_t QD = s0;
+      const uint32_t RX = s0 + (uint32_t)(C::QN * C::QPITCH * 4);  // received half quadrant
+      const uint32_t SX = RX + XBYTES;                              // half quadrant sent to the peer
+      const uint32_t XL = SX + XBYTES;                              // CTA 0: G_S[O_0][192..255] kept here
       const int own0 = C::PAIR ? 128 * c : 0;  // first column of this CTA's own quadrant
       const bool own_cols = !C::PAIR || half == c;
-      const bool to_peer = C::PAIR && c == 0 && half == 1;  // G_S[O_0][O_1] -> CTA 1's Qx
-      uint32_t dst = 0;
-      if (own_cols) dst = QD + (uint32_t)(r * C::QPITCH * 4);
-      if (to_peer) dst = QX + (uint32_t)(r * C::QPITCH * 4);  // staged here, sent in one copy below
 #pragma unroll 1
       for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
         float f[32];
         tld(fcol + j0, f);
-        if (valid && (own_cols || to_peer)) {
-          const uint32_t at = dst + (uint32_t)((j0 - (own_cols ? own0 : 128)) * 4);
+        if (!valid) continue;
+        uint32_t at = 0;
+        if (own_cols) at = QD + (uint32_t)(r * C::QPITCH + (j0 - own0)) * 4u;
+        else if (C::PAIR && c == 0) at = (j0 < 192 ? SX + (uint32_t)(r * XPITCH + (j0 - 128)) * 4u
+                                                   : XL + (uint32_t)(r * XPITCH + (j0 - 192)) * 4u);
+        if (own_cols || (C::PAIR && c == 0)) {
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(at + 16 * u), "r"(__float_as_uint(f[4 * u])),
                          "r"(__float_as_uint(f[4 * u + 1])), "r"(__float_as_uint(f[4 * u + 2])),
                          "r"(__float_as_uint(f[4 * u + 3]))
                          : "memory");
+        } else if (C::PAIR && i >= 192) {
+          // CTA 1, rows j in [192, 256): G_S[j][i] for i = j0.. into column j - 192 of the transposed
+          // staging (lanes write consecutive floats).
+          const uint32_t colp = SX + (uint32_t)(j0 * XPITCH + (i - 192)) * 4u;
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(colp + (uint32_t)(u * XPITCH * 4)), "f"(f[u]) : "memory");
         }
       }
-      constexpr uint32_t QBYTES = C::QN * C::QPITCH * 4;
-      if (C::PAIR && c == 1 && threadIdx.x == 0) mbar_arrive_expect_tx(bar_xin, QBYTES);
+      if (C::PAIR && threadIdx.x == 0) mbar_arrive_expect_tx(bar_xin, XBYTES);
       fence_proxy_async_smem();
       __syncthreads();
-      if (C::PAIR && c == 0 && threadIdx.x == 0)
-        bulk_copy_to_peer(mapa_shared(QX, 1), QX, QBYTES, mapa_shared(bar_xin, 1));
-      if (C::PAIR && c == 1) {  // both warps of a quarter read G_S[O_0][O_1], sent by CTA 0
+      if (C::PAIR && threadIdx.x == 0) bulk_copy_to_peer(mapa_shared(RX, peer), SX, XBYTES, mapa_shared(bar_xin, peer));
+      if (C::PAIR) {
         if (ok) ok = mbar_wait(bar_xin, xin_phase & 1u, KID_CNP_CHIP, 13);
         ok = __all_sync(0xffffffffu, ok);
       }
       ++xin_phase;
-      // Thread (row j): the entries (i, j), i < j, of 32-column chunks of i.  A lane quarter's
-      // chunks are Qd's chunks below its rows (and, in a pair's CTA 1, the four chunks of Qx);
-      // the two warps of the quarter take them in turn.  The TMEM loads are warp-collective: the
-      // chunk list is the same for every lane, and i < j only guards the stores.
       const int j = i;
       const int jwarp = rbase + quarter * 32;  // first row of this warp
-      const int ndiag = jwarp < B ? (jwarp - own0) / 32 + 1 : 0;  // warps past row b - 1 (b = 64) have none
-      const int ncross = (C::PAIR && c == 1) ? 4 : 0;
       const bool store = ok && valid;
       float* out = SD.grad + z * P;
+      // Items of 32 rows i against this warp's 32 rows j: the diagonal quadrant's chunks below the
+      // warp's rows and, in CTA 1 for j < 192, the four chunks of O_0.  The two warps of a lane
+      // quarter take them in turn.  The TMEM loads are warp-collective: the chunk list is the same
+      // for every lane, and i < j only guards the stores.
+      const int ndiag = jwarp < B ? (jwarp - own0) / 32 + 1 : 0;  // warps past row b - 1 (b = 64) have none
+      const int ncross = (C::PAIR && c == 1 && jwarp < 192) ? 4 : 0;
 #pragma unroll 1
       for (int item = half; item < ncross + ndiag; item += 2) {
         const bool cross = item < ncross;
         const int i0 = cross ? 32 * item : own0 + 32 * (item - ncross);
         float f[32];
         tld(fcol + i0, f);  // G_S[j][i0 .. i0 + 31]
-        // G_S[i0 + u][j] at qcol[u * QPITCH]; g[p(i0 + u, j)] at o_u, with
-        // p(i + 1, j) - p(i, j) = b - 2 - i.
-        const float* qcol = reinterpret_cast<const float*>(smem + (cross ? C::QN * C::QPITCH * 4 : 0)) +
-                            (i0 - (cross ? 0 : own0)) * C::QPITCH + (j - own0);
+        // G_S[i0 + u][j] at qcol[u * pitch]; g[p(i0 + u, j)] at o_u, with p(i + 1, j) - p(i, j) = b - 2 - i.
+        const float* qcol = cross ? reinterpret_cast<const float*>(smem + (RX - s0)) + i0 * XPITCH + (j - 128)
+                                  : reinterpret_cast<const float*>(smem) + (i0 - own0) * C::QPITCH + (j - own0);
+        const int pitch = cross ? XPITCH : C::QPITCH;
         float* o = out + ro(i0) + j;
         int step = B - 2 - i0;
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          if (store && i0 + u < j) *o = qcol[u * C::QPITCH] - f[u];
+          if (store && i0 + u < j) *o = qcol[u * pitch] - f[u];
+          o += step;
+          --step;
+        }
+      }
+      if (C::PAIR && c == 0) {
+        // CTA 0's half of the cross quadrant, one 32 x 32 item per warp, entirely from shared
+        // memory: G_S[i][j] (kept) minus G_S[j][i] (received transposed).
+        const int i0 = 32 * (warp & 3);
+        const int jx = 192 + 32 * (warp >> 2) + lane;
+        const float* xl = reinterpret_cast<const float*>(smem + (XL - s0)) + i0 * XPITCH + (jx - 192);
+        const float* yt = reinterpret_cast<const float*>(smem + (RX - s0)) + i0 * XPITCH + (jx - 192);
+        float* o = out + ro(i0) + jx;
+        int step = B - 2 - i0;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          if (ok) *o = xl[u * XPITCH] - yt[u * XPITCH];
           o += step;
           --step;
         }
