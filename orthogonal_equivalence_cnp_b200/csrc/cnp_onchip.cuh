@@ -482,27 +482,30 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     // R_k = G (A form in V1) and L_k = G (B form in V2, the peer's quadrant in the peer): every
     // CTA of the cluster has finished reading its G staging.
     if constexpr (C::PAIR) cluster_sync_all(); else __syncthreads();
-    if (k >= 1) {
-#pragma unroll 1
-      for (int j0 = c0; j0 < c0 + C::HALF; j0 += 32) {
-        float g[32];
-        tld(REG2 + j0, g);
-        chip_put_aform(V1, r, j0, g);
-        if (valid) put_bform(V2, j0, g);
-      }
-      send_bform(V2);
-    }
     uint32_t fcol = REG2;  // the TMEM columns holding G_S for PACK
     if (k >= 1) {
       // Each product is issued as soon as its operands are in place; the rest of an epilogue (the
       // bf16 copies that only a later product reads, and the exchange) runs beside it:
       //   R_a = ACC + 2G goes back into ACC first (MMA_L accumulates onto it), its A form into V1
       //   while MMA_L runs; L_a is read out of ACC, then MMA_R of the next level may overwrite ACC
-      //   while L_a's B form is written and exchanged.
+      //   while L_a's B form is written and exchanged.  The first product needs only R_k = G in
+      //   A form, so L_k = G's B form is written and exchanged beside it.
       constexpr int NCH = C::HALF / 32;  // 32-column chunks per thread
       fcol = ACC;
-      arrive_ready();
-      issue(V1, SC, false, false, false, 6);  // ACC = R_k . S^T = R_k T
+      {
+        float gv[NCH][32];
+#pragma unroll
+        for (int q = 0; q < NCH; ++q) {
+          tld(REG2 + c0 + 32 * q, gv[q]);
+          chip_put_aform(V1, r, c0 + 32 * q, gv[q]);
+        }
+        arrive_ready();
+        issue(V1, SC, false, false, false, 6);  // ACC = R_k . S^T = R_k T
+#pragma unroll
+        for (int q = 0; q < NCH; ++q)
+          if (valid) put_bform(V2, c0 + 32 * q, gv[q]);
+        send_bform(V2);
+      }
 #pragma unroll 1
       for (int a = k - 1; a >= 0; --a) {
         wait_mma(7);
@@ -585,31 +588,23 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
       fence_proxy_async_smem();
       __syncthreads();
       if (C::PAIR && threadIdx.x == 0) bulk_copy_to_peer(mapa_shared(RX, peer), SX, XBYTES, mapa_shared(bar_xin, peer));
-      if (C::PAIR) {
-        if (ok) ok = mbar_wait(bar_xin, xin_phase & 1u, KID_CNP_CHIP, 13);
-        ok = __all_sync(0xffffffffu, ok);
-      }
-      ++xin_phase;
       const int j = i;
       const int jwarp = rbase + quarter * 32;  // first row of this warp
-      const bool store = ok && valid;
       float* out = SD.grad + z * P;
       // Items of 32 rows i against this warp's 32 rows j: the diagonal quadrant's chunks below the
-      // warp's rows and, in CTA 1 for j < 192, the four chunks of O_0.  The two warps of a lane
-      // quarter take them in turn.  The TMEM loads are warp-collective: the chunk list is the same
-      // for every lane, and i < j only guards the stores.
+      // warp's rows, then (once the peer's half quadrant has landed) in CTA 1 for j < 192 the four
+      // chunks of O_0.  The two warps of a lane quarter take them in turn.  The TMEM loads are
+      // warp-collective: the chunk list is the same for every lane, and i < j only guards the stores.
       const int ndiag = jwarp < B ? (jwarp - own0) / 32 + 1 : 0;  // warps past row b - 1 (b = 64) have none
       const int ncross = (C::PAIR && c == 1 && jwarp < 192) ? 4 : 0;
-#pragma unroll 1
-      for (int item = half; item < ncross + ndiag; item += 2) {
-        const bool cross = item < ncross;
-        const int i0 = cross ? 32 * item : own0 + 32 * (item - ncross);
+      auto pack_item = [&](bool cross, int i0) {
         float f[32];
         tld(fcol + i0, f);  // G_S[j][i0 .. i0 + 31]
         // G_S[i0 + u][j] at qcol[u * pitch]; g[p(i0 + u, j)] at o_u, with p(i + 1, j) - p(i, j) = b - 2 - i.
         const float* qcol = cross ? reinterpret_cast<const float*>(smem + (RX - s0)) + i0 * XPITCH + (j - 128)
                                   : reinterpret_cast<const float*>(smem) + (i0 - own0) * C::QPITCH + (j - own0);
         const int pitch = cross ? XPITCH : C::QPITCH;
+        const bool store = ok && valid;
         float* o = out + ro(i0) + j;
         int step = B - 2 - i0;
 #pragma unroll
@@ -618,7 +613,16 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
           o += step;
           --step;
         }
+      };
+#pragma unroll 1
+      for (int item = half; item < ndiag; item += 2) pack_item(false, own0 + 32 * item);
+      if (C::PAIR) {
+        if (ok) ok = mbar_wait(bar_xin, xin_phase & 1u, KID_CNP_CHIP, 13);
+        ok = __all_sync(0xffffffffu, ok);
       }
+      ++xin_phase;
+#pragma unroll 1
+      for (int item = half; item < ncross; item += 2) pack_item(true, 32 * item);
       if (C::PAIR && c == 0) {
         // CTA 0's half of the cross quadrant, one 32 x 32 item per warp, entirely from shared
         // memory: G_S[i][j] (kept) minus G_S[j][i] (received transposed).
