@@ -52,6 +52,9 @@ struct GemmDesc {
   bool a_mn = false, b_mn = false;
   Epilogue epi;
   const float* b_scale = nullptr;  // set: B is int8 codes, B row r scaled by b_scale[r] (W0' GEMM only)
+  // B was not written by the kernel launched just before this one (W0' GEMM only): its first
+  // stages may be requested before the wait for that kernel.
+  bool b_static = false;
 };
 
 // Kernel ids recorded in the device error word.
@@ -572,6 +575,7 @@ struct WideArgs {
   void* out2;  // bf16 [M, N] block-factor result, or null (plain GEMM)
   long ld2;
   const float* bscale;  // Q8 only: scale of each row of the int8 B array
+  int b_early;          // B's first stages are requested before griddep_wait (B is not the previous kernel's output)
 };
 
 constexpr int TCW_BM = 256, TCW_BN = 256, TCW_STAGES = 3;
@@ -662,33 +666,41 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_holder;
-  griddep_wait();
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    bool ok = true;
-    for (int i = 0; i < nkt; ++i) {
-      const int s = i % STAGES;
-      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-      if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 11)) { ok = false; break; }
+    // The B tile of step i (W0' or its int8 codes) into the stage's B region.
+    auto load_b = [&](int i, int s) {
       const int k0 = i * TC_BK;
-      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
+      const uint32_t sb = smem0 + s * STAGE_BYTES + A_BYTES;
       if (Q8) {
-        // Codes of step i into the first 16 KiB of the stage's B region.
-        mbar_arrive_expect_tx(full_bar(s), A_BYTES + TCW_Q8_TILE);
-        tma_load_2d(sa, &tmA, full_bar(s), k0, m0);
         if (!B_MN) tma_load_2d(sb, &tmB, full_bar(s), k0, n0);  // box 64 (k) x 256 (n) codes
         else tma_load_2d(sb, &tmB, full_bar(s), n0, k0);        // box 256 (n) x 64 (k) codes
-        continue;
-      }
-      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
-      tma_load_2d(sa, &tmA, full_bar(s), k0, m0);  // box 64 x 256: both halves
-      if (!B_MN) {
+      } else if (!B_MN) {
         tma_load_2d(sb, &tmB, full_bar(s), k0, n0);
       } else {
 #pragma unroll
         for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmB, full_bar(s), n0 + 64 * h, k0);
       }
+    };
+    const uint32_t stage_tx = Q8 ? A_BYTES + TCW_Q8_TILE : STAGE_BYTES;
+    // B of the first stages while the previous kernel (which wrote A) finishes.
+    const int early = args.b_early ? min(nkt, STAGES) : 0;
+    for (int i = 0; i < early; ++i) {
+      mbar_arrive_expect_tx(full_bar(i), stage_tx);
+      load_b(i, i);
+    }
+    griddep_wait();
+    bool ok = true;
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (i >= early) {
+        if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 11)) { ok = false; break; }
+        mbar_arrive_expect_tx(full_bar(s), stage_tx);
+        load_b(i, s);
+      }
+      tma_load_2d(smem0 + s * STAGE_BYTES, &tmA, full_bar(s), i * TC_BK, m0);  // box 64 x 256: both halves
     }
     if (ok && fuse) {
       // Q's K chunks t = 0..3 into stages sq0 (t = 0, 1) and sq1 (t = 2, 3), each as soon as the
@@ -711,7 +723,10 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
         }
       }
     }
-  } else if (warp == 1 && lane == 0) {
+  } else {
+    griddep_wait();
+  }
+  if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: both halves per k step
     for (int i = 0; i < nkt; ++i) {
       const int s = i % STAGES;

@@ -476,11 +476,12 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
     tq = ta;  // unused without the block factor
     to = ta;
   }
-  WideArgs a;
+  WideArgs a = {};
   a.M = g.M; a.N = g.N; a.K = g.K;
   a.d1 = g.epi.d1; a.ld1 = g.epi.ld1;
   a.out2 = out2; a.ld2 = ld2;
   a.bscale = g.b_scale;
+  a.b_early = g.b_static ? 1 : 0;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(cls, st);
   if (launch_pdl_prio(kern, grid, dim3(Q8 ? 128 + TCW_CONV_THREADS : 128), smem, st, true, ta, tb, tq, td, to, a) != cudaSuccess)
@@ -1049,6 +1050,7 @@ poetx_status forward_chain(const poetx_desc* d, long n, const void* X, const voi
   g.A = view(V, n, d->d_in, d->d_in);
   g.B = view(W0p, d->d_out, d->d_in, d->d_in);
   g.b_scale = W0s;  // POET-XQ: W0' is int8 codes with per-row scales
+  g.b_static = true;  // W0' is the caller's, not the output of the launch before (BD_P)
   g.epi.d1 = Z; g.epi.d1_dtype = dt; g.epi.ld1 = d->d_out;
   if (Y == nullptr) return run_w_gemm(dt, g, nullptr, 0, false, nullptr, 0, st);  // recompute only (mem-mode backward)
   if (bd_fusable(dt, b, g)) {
@@ -1369,6 +1371,7 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   g.A = view(ws + w.dZ, n, dout, dout);
   g.B = view(W0p, dout, din, din); g.b_mn = true;
   g.b_scale = W0s;
+  g.b_static = true;  // W0' is the caller's, not the output of the launch before (dZ)
   g.epi.d1 = ws + w.dV; g.epi.d1_dtype = dt; g.epi.ld1 = din;
   const bool fused_du = bd_fusable(dt, b, g);
   if (fused_du) POETX_TRY(run_w_gemm(dt, g, Q_P, din, true, ws + w.dU, din, stream, POETX_KC_W_GEMM_ADJ));
