@@ -604,8 +604,13 @@ __device__ __forceinline__ bool converters_all(bool p, int count) {
   return r != 0;
 }
 
+// Threads of a launch: bf16, 8 warps (warps 0 and 1 also issue the loads and the MMAs; all eight
+// drain TMEM, two per lane quarter, each taking half of the columns); Q8, 4 draining warps plus
+// the converter warps.
+__host__ __device__ constexpr int tcw_threads(bool q8) { return q8 ? 128 + TCW_CONV_THREADS : 256; }
+
 template <bool B_MN, bool Q_MN, bool Q8 = false>
-__global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
+__global__ void __launch_bounds__(tcw_threads(Q8), 1)
     gemm_w256_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmD,
                  const __grid_constant__ CUtensorMap tmO, const WideArgs args) {
@@ -806,16 +811,19 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
   griddep_launch();
-  const int r = warp * 32 + lane;  // TMEM lane = row within a half
-  const uint32_t tl = tmem_d + ((uint32_t)(warp * 32) << 16);
-  const bool epi_warp = !Q8 || warp < 4;  // the four warps that own the TMEM lanes drain them
+  const int lq = warp & 3;                          // TMEM lane quarter of this warp
+  const int r = lq * 32 + lane;                     // TMEM lane = row within a half
+  const uint32_t tl = tmem_d + ((uint32_t)(lq * 32) << 16);
+  const bool epi_warp = !Q8 || warp < 4;            // Q8: the converter warps do not drain
+  constexpr int EPI_COLS = Q8 ? BN : BN / 2;        // columns of a 256-column drain per warp
+  const int col_lo = Q8 ? 0 : (warp >> 2) * EPI_COLS;
 
-  // Drains 256 columns of TMEM at column offset col0 (row m of the output): bf16 to global
-  // `dst` (if set) and, if stage >= 0, into that ring stage as four swizzled K-major 128 x 64
-  // tiles, which are both the A operand of the block factor and TMA-store boxes of D.
+  // Drains this warp's columns of 256 TMEM columns at offset col0 (row m of the output): bf16 to
+  // global `dst` (if set) and, if stage >= 0, into that ring stage as four swizzled K-major
+  // 128 x 64 tiles, which are both the A operand of the block factor and TMA-store boxes of D.
   auto drain = [&](uint32_t col0, int m, void* dst, long ld, int stage) {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = col_lo; c < col_lo + EPI_COLS; c += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tl + col0 + (uint32_t)c, v);
       tmem_wait_ld();
@@ -894,16 +902,18 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
       ok2 = __all_sync(0xffffffffu, ok2);
       tc_fence_after();
     };
-    // The block-factor result of half h (TMEM columns col0..): 32-row x 64-column boxes per warp
-    // through two staging buffers, stored with TMA (rows past M clipped by the map).
+    // The block-factor result of half h (TMEM columns col0..): 32-row x 64-column boxes of this
+    // warp's columns, stored with TMA (rows past M clipped by the map) from `stage` (nbuf buffers
+    // of 4 KiB per warp, used in turn).
     int nbox = 0;
-    uint8_t* ostage = smem + STAGES * STAGE_BYTES + warp * 8192;
-    auto drain_out = [&](uint32_t col0, int h) {
+    auto drain_out = [&](uint32_t col0, int h, uint8_t* stage, int nbuf) {
 #pragma unroll 1
-      for (int c64 = 0; c64 < BN / 64; ++c64, ++nbox) {
-        uint8_t* buf = ostage + (nbox & 1) * 4096;
-        if (nbox >= 2) {
-          if (lane == 0) bulk_wait_read<1>();  // the store two boxes back has read this buffer
+      for (int c64 = col_lo / 64; c64 < (col_lo + EPI_COLS) / 64; ++c64, ++nbox) {
+        uint8_t* buf = stage + (nbox % nbuf) * 4096;
+        if (nbox >= nbuf) {
+          if (lane == 0) {
+            if (nbuf == 1) bulk_wait_read<0>(); else bulk_wait_read<1>();  // this buffer's last store has read it
+          }
           __syncwarp();
         }
 #pragma unroll
@@ -925,7 +935,7 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
         fence_proxy_async_smem();  // the TMA engine reads what the threads wrote
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmO, smem_u32(buf), n0 + c64 * 64, m0 + h * TC_BM + warp * 32);
+          tma_store_2d(&tmO, smem_u32(buf), n0 + c64 * 64, m0 + h * TC_BM + lq * 32);
           bulk_commit();
         }
       }
@@ -938,6 +948,9 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
       tc_fence_after();
       if (ok2) store_half(sdh, h);
     };
+    // Store staging past the ring: Q8, two 4 KiB buffers for each of the 4 draining warps; bf16,
+    // one for each of the 8.
+    uint8_t* ostage = smem + STAGES * STAGE_BYTES + (Q8 ? warp * 8192 : warp * 4096);
     stage_d(0);
     block_product(0);
     wait_product(0);
@@ -945,9 +958,17 @@ __global__ void __launch_bounds__(Q8 ? 128 + TCW_CONV_THREADS : 128, 1)
     __syncthreads();
     stage_d(1);
     block_product(1);
-    if (ok2 && epi_warp) drain_out(0, 0);  // beside the second product (other TMEM columns)
+    if (ok2 && epi_warp) drain_out(0, 0, ostage, Q8 ? 2 : 1);  // beside the second product (other TMEM columns)
     wait_product(1);
-    if (ok2 && epi_warp) drain_out(BN, 1);
+    if (Q8) {
+      if (ok2 && epi_warp) drain_out(BN, 1, ostage, 2);
+    } else {
+      // The D stage is free once D_1's stores have read it: two buffers per warp there.
+      if (threadIdx.x == 0) bulk_wait_read<0>();
+      __syncthreads();
+      nbox = 0;  // fresh buffers
+      if (ok2) drain_out(BN, 1, smem + sdh * STAGE_BYTES + warp * 8192, 2);
+    }
     if (epi_warp && lane == 0) bulk_wait_read<0>();
     __syncwarp();
   }

@@ -484,7 +484,7 @@ poetx_status launch_w256(const GemmDesc& g, const void* Q, long q_rows, void* ou
   a.b_early = g.b_static ? 1 : 0;
   dim3 grid(g.N / TCW_BN, (g.M + TCW_BM - 1) / TCW_BM, 1);
   LaunchScope ls(cls, st);
-  if (launch_pdl_prio(kern, grid, dim3(Q8 ? 128 + TCW_CONV_THREADS : 128), smem, st, true, ta, tb, tq, td, to, a) != cudaSuccess)
+  if (launch_pdl_prio(kern, grid, dim3(tcw_threads(Q8)), smem, st, true, ta, tb, tq, td, to, a) != cudaSuccess)
     return POETX_ERR_CUDA;
   return last_launch();
 }
