@@ -822,33 +822,54 @@ __global__ void __launch_bounds__(tcw_threads(Q8), 1)
   // global `dst` (if set) and, if stage >= 0, into that ring stage as four swizzled K-major
   // 128 x 64 tiles, which are both the A operand of the block factor and TMA-store boxes of D.
   auto drain = [&](uint32_t col0, int m, void* dst, long ld, int stage) {
-#pragma unroll 1
-    for (int c = col_lo; c < col_lo + EPI_COLS; c += 32) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tl + col0 + (uint32_t)c, v);
-      tmem_wait_ld();
-      uint4 q[4];
+    // 64 columns (two TMEM loads) per round; the next round's loads are in flight while this
+    // round's values are converted and written.
+    uint32_t va[2][32], vb[2][32];
+    tmem_ld_32x32b_x32(tl + col0 + (uint32_t)col_lo, va[0]);
+    tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(col_lo + 32), va[1]);
+    tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        q[u] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1])),
-                          pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
-                          pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
-                          pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
-      if (dst != nullptr && m < args.M) {
-        uint4* g = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + (long)m * ld + n0 + c);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) g[u] = q[u];
+    for (int c = col_lo; c < col_lo + EPI_COLS; c += 64) {
+      const bool more = c + 64 < col_lo + EPI_COLS;
+      if (more) {
+        tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(c + 64), vb[0]);
+        tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(c + 96), vb[1]);
       }
-      if (stage >= 0) {
-        // K chunk c/64: 16 KiB tile at the stage + (c/64)*16 KiB, 16-byte chunk ch of row r at
-        // chunk position ch ^ (r % 8).
-        uint8_t* tileA = smem + stage * STAGE_BYTES + (c / 64) * HALF_A + r * 128;
-        const int ch0 = (c % 64) / 8;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(tileA + (((ch0 + u) ^ (r & 7)) * 16)) = q[u];
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t* v = va[hh];
+        uint4 q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          q[u] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+        const int cc = c + 32 * hh;
+        if (dst != nullptr && m < args.M) {
+          uint4* g = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + (long)m * ld + n0 + cc);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) g[u] = q[u];
+        }
+        if (stage >= 0) {
+          // K chunk cc/64: 16 KiB tile at the stage + (cc/64)*16 KiB, 16-byte chunk ch of row r at
+          // chunk position ch ^ (r % 8).
+          uint8_t* tileA = smem + stage * STAGE_BYTES + (cc / 64) * HALF_A + r * 128;
+          const int ch0 = (cc % 64) / 8;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(tileA + (((ch0 + u) ^ (r & 7)) * 16)) = q[u];
+        }
+      }
+      if (more) {
+        tmem_wait_ld();
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int u = 0; u < 32; ++u) va[hh][u] = vb[hh][u];
       }
     }
   };
+
 
   // D goes out through TMA stores of the swizzled tiles (whole 128-byte lines; rows past M are
   // clipped by the tensor map), issued by thread 0 in its bulk group.
@@ -907,8 +928,20 @@ __global__ void __launch_bounds__(tcw_threads(Q8), 1)
     // of 4 KiB per warp, used in turn).
     int nbox = 0;
     auto drain_out = [&](uint32_t col0, int h, uint8_t* stage, int nbuf) {
-#pragma unroll 1
-      for (int c64 = col_lo / 64; c64 < (col_lo + EPI_COLS) / 64; ++c64, ++nbox) {
+      // One 64-column box per round (two TMEM loads); the next box's loads are in flight while
+      // this one is converted, staged and stored.
+      const int b0 = col_lo / 64, b1 = (col_lo + EPI_COLS) / 64;
+      uint32_t va[2][32], vb[2][32];
+      tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(b0 * 64), va[0]);
+      tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(b0 * 64 + 32), va[1]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c64 = b0; c64 < b1; ++c64, ++nbox) {
+        const bool more = c64 + 1 < b1;
+        if (more) {
+          tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(c64 * 64 + 64), vb[0]);
+          tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(c64 * 64 + 96), vb[1]);
+        }
         uint8_t* buf = stage + (nbox % nbuf) * 4096;
         if (nbox >= nbuf) {
           if (lane == 0) {
@@ -918,9 +951,7 @@ __global__ void __launch_bounds__(tcw_threads(Q8), 1)
         }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tl + col0 + (uint32_t)(c64 * 64 + hh * 32), v);
-          tmem_wait_ld();
+          const uint32_t* v = va[hh];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int j = 8 * u;
@@ -938,8 +969,16 @@ __global__ void __launch_bounds__(tcw_threads(Q8), 1)
           tma_store_2d(&tmO, smem_u32(buf), n0 + c64 * 64, m0 + h * TC_BM + lq * 32);
           bulk_commit();
         }
+        if (more) {
+          tmem_wait_ld();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int u = 0; u < 32; ++u) va[hh][u] = vb[hh][u];
+        }
       }
     };
+
     auto stage_d = [&](int h) {
       if (ok2 && epi_warp) drain((uint32_t)(h * BN), m0 + h * TC_BM + r, nullptr, 0, sdh);
       fence_proxy_async_smem();  // the tensor core and the TMA engine read what the threads wrote
