@@ -175,7 +175,10 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     if (need_s) {
       // The block's packed theta (8 bulk copies into V1 + V2) is requested first, so that the
       // TMEM allocation and the cluster barrier below overlap the copy.
-      griddep_wait();  // theta may come from the previous kernel (an optimiser step)
+      // The forward's theta may come from the launch just before (an optimiser step).  The
+      // adjoint's never does (the launches before it are the layer's own backward products), so
+      // it is read, and S built, while that launch finishes; only G waits for it.
+      if (!ADJ) griddep_wait();
       const uint32_t bytes = (uint32_t)(P * 4);  // 16-byte multiple for b % 8 == 0
       mbar_arrive_expect_tx(bar_theta, bytes);
       const uint32_t chunk = ((bytes / 8) + 15) & ~15u;
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
   const uint32_t tlane = tbase + ((uint32_t)(quarter * 32) << 16);
   const uint32_t ACC = tlane, REG2 = tlane + B;
   const uint32_t ready_dst = (C::PAIR && !leader) ? mapa_shared(bar_ready, 0) : bar_ready;
-  griddep_wait();  // theta and the gradient partials come from earlier kernels
+  if (!ADJ) griddep_wait();  // Q is written over what earlier kernels may still read
 
   bool ok = true;
   uint32_t mma_phase = 0, ready_phase = 0, xin_phase = 0;
@@ -448,6 +451,7 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
     // with conflict-free 16-byte loads.  The staging overlaps V1 / V2 (and the theta staging):
     // every CTA of the cluster has finished its theta reads before the first round starts.
     if constexpr (C::PAIR) cluster_sync_all(); else __syncthreads();
+    griddep_wait();  // the partials come from the launch just before
 #pragma unroll 1
     for (int sp = 0; sp < SD.splits; ++sp) {
       if (sp > 0) __syncthreads();  // every thread has read the previous round
