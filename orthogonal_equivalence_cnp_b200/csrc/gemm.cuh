@@ -188,6 +188,7 @@ struct TcArgs {
   int M, N, K, splits;
   int a_zrow, a_zcol, b_zrow, b_zcol;
   int tma_store;  // plain bf16 d1 (no addend/alpha/diag/d2/splits, zrow1 = 0): TMA-store epilogue
+  int b_early;    // B is not the previous launch's output: its first stages are requested before the wait
   Epilogue epi;
 };
 
@@ -251,24 +252,11 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_holder;
-  griddep_wait();  // operands and epilogue addends may come from the previous kernel
-
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    for (int i = 0; i < nkt; ++i) {
-      const int s = i % STAGES;
-      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-      if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 1)) break;
-      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+    auto load_b = [&](int i, int s) {
       const int k0 = (kt0 + i) * TC_BK;
-      const uint32_t sa = smem0 + s * STAGE_BYTES, sb = sa + A_BYTES;
-      if (!A_MN) {
-        tma_load_2d(sa, &tmA, full_bar(s), z * args.a_zcol + k0, z * args.a_zrow + m0);
-      } else {
-#pragma unroll
-        for (int h = 0; h < TC_BM / 64; ++h)
-          tma_load_2d(sa + h * 8192, &tmA, full_bar(s), z * args.a_zcol + m0 + 64 * h, z * args.a_zrow + k0);
-      }
+      const uint32_t sb = smem0 + s * STAGE_BYTES + A_BYTES;
       if (!B_MN) {
         tma_load_2d(sb, &tmB, full_bar(s), z * args.b_zcol + k0, z * args.b_zrow + n0);
       } else {
@@ -276,8 +264,36 @@ __global__ void __launch_bounds__(128)
         for (int h = 0; h < BN / 64; ++h)
           tma_load_2d(sb + h * 8192, &tmB, full_bar(s), z * args.b_zcol + n0 + 64 * h, z * args.b_zrow + k0);
       }
+    };
+    // B of the first stages while the previous kernel (which wrote A) finishes.
+    const int early = args.b_early ? min(nkt, STAGES) : 0;
+    for (int i = 0; i < early; ++i) {
+      mbar_arrive_expect_tx(full_bar(i), STAGE_BYTES);
+      load_b(i, i);
     }
-  } else if (warp == 1 && lane == 0) {
+    griddep_wait();  // A and the epilogue's addends may come from the previous kernel
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (i >= early) {
+        if (!mbar_wait(empty_bar(s), ph ^ 1u, KID_GEMM_TC, 1)) break;
+        mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+        load_b(i, s);
+      }
+      const int k0 = (kt0 + i) * TC_BK;
+      const uint32_t sa = smem0 + s * STAGE_BYTES;
+      if (!A_MN) {
+        tma_load_2d(sa, &tmA, full_bar(s), z * args.a_zcol + k0, z * args.a_zrow + m0);
+      } else {
+#pragma unroll
+        for (int h = 0; h < TC_BM / 64; ++h)
+          tma_load_2d(sa + h * 8192, &tmA, full_bar(s), z * args.a_zcol + m0 + 64 * h, z * args.a_zrow + k0);
+      }
+    }
+  } else {
+    griddep_wait();  // operands and epilogue addends may come from the previous kernel
+  }
+  if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     for (int i = 0; i < nkt; ++i) {
       const int s = i % STAGES;

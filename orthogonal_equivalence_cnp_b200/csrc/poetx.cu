@@ -254,6 +254,7 @@ poetx_status launch_tc(const GemmDesc& g, cudaStream_t st, int cls) {
   a.M = g.M; a.N = g.N; a.K = g.K; a.splits = g.splits;
   a.a_zrow = (int)g.A.zrow; a.a_zcol = (int)g.A.zcol; a.b_zrow = (int)g.B.zrow; a.b_zcol = (int)g.B.zcol;
   a.epi = g.epi;
+  a.b_early = g.b_static ? 1 : 0;
   // TMA-store epilogue for a plain bf16 result batched (if at all) along columns: the map spans
   // every batch's columns, boxes of 64 columns x 32 rows.
   const Epilogue& e = g.epi;
@@ -543,8 +544,10 @@ poetx_status bd_forward(int dt, long n, int d, int b, const void* in, const void
 }
 
 // Out[:, blk z] = In[:, blk z] . Q_z  (adjoint of bd_forward w.r.t. its input).
-poetx_status bd_backward(int dt, long n, int d, int b, const void* in, const void* Q, void* out, cudaStream_t st) {
+poetx_status bd_backward(int dt, long n, int d, int b, const void* in, const void* Q, void* out, cudaStream_t st,
+                         bool q_static = false) {
   GemmDesc g;
+  g.b_static = q_static;
   g.M = (int)n; g.N = b; g.K = b; g.batch = d / b;
   g.A = view(in, n, d, d, 0, b);
   g.B = view(Q, d, b, b, b, 0);
@@ -567,8 +570,9 @@ int grad_splits(int dt, long n, int nb, int b) {
 }
 
 poetx_status block_grads(int dt, long n, int d, int b, const void* lhs, const void* rhs, float* part, int splits,
-                         cudaStream_t st, bool few_ctas = false) {
+                         cudaStream_t st, bool few_ctas = false, bool rhs_static = false) {
   GemmDesc g;
+  g.b_static = rhs_static;
   g.M = b; g.N = b; g.K = (int)n; g.batch = d / b; g.splits = splits;
   g.A = view(lhs, n, d, d, 0, b); g.a_mn = true;
   g.B = view(rhs, n, d, d, 0, b); g.b_mn = true;
@@ -1360,10 +1364,11 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   // BD_R^T-adjoint (both read dY', so it is shared through L2), leaving the W0' GEMM below the
   // whole GPU.
   POETX_TRY(permute_cols(dt, dY, dout, ws + w.dYp, dout, n, dout, perm_L, nullptr, false, stream));
-  POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream));
+  POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream, true));  // Q_R: from the CNP forward
   POETX_TRY(stream_edge(stream, side, ss->ev[0]));
   SideJoin join{stream, side, ss->ev[3], true};
-  POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, side, w.sR == 1));
+  POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, side, w.sR == 1,
+                        true));  // Z: saved by the forward or recomputed several launches before
   if (cudaEventRecord(ss->ev[1], side) != cudaSuccess) return POETX_ERR_CUDA;  // G_R partials done
   // dV = dZ . W0' (and, for b = 256, dU_i = dV_i . Q_P,i in the same kernel)
   GemmDesc g;
@@ -1382,7 +1387,8 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   // runs in the adjoint's launch on the SMs its pairs leave free (b = 256), else on the side
   // stream from the moment dU exists.
   if (cudaEventRecord(ss->ev[2], stream) != cudaSuccess) return POETX_ERR_CUDA;  // dU done
-  POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream));
+  POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream, false,
+                        true));  // U: saved by the forward or recomputed several launches before
   if (cudaStreamWaitEvent(stream, ss->ev[1], 0) != cudaSuccess) return POETX_ERR_CUDA;
   CnpSide sides[2];
   sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + w.GpR);
