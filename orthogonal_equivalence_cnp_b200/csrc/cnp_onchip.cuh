@@ -305,18 +305,22 @@ __global__ void __launch_bounds__(256, 1) cnp_chip_kernel(const __grid_constant_
   };
   // The exchange of a B form written by put_bform (pair only; every thread calls it): the peer
   // expects 32 KiB on its xin barrier; this CTA's XS (rows O_c of the peer's two column atoms)
-  // goes out as two 16 KiB copies into the peer's buffer `buf`.
+  // goes out as two 16 KiB copies into the peer's buffer `buf`.  Only the four warps holding the
+  // peer's column half wrote XS, so only they meet before the copy: the leader's warp 0, which
+  // may still be blocked issuing the product that runs meanwhile, is not waited for.
   auto send_bform = [&](uint32_t buf) {
     if constexpr (C::PAIR) {
-      if (threadIdx.x == 0) mbar_arrive_expect_tx(bar_xin, 2u * 128u * 128u);
-      fence_proxy_async_smem();  // XS was written by the generic proxy; the copy engine reads it
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        const uint32_t bar_peer = mapa_shared(bar_xin, peer);
+      if (half == (c ^ 1)) {
+        fence_proxy_async_smem();  // XS was written by the generic proxy; the copy engine reads it
+        named_bar_sync(1, 128);
+        if (quarter == 0 && lane == 0) {
+          mbar_arrive_expect_tx(bar_xin, 2u * 128u * 128u);  // this CTA's incoming half
+          const uint32_t bar_peer = mapa_shared(bar_xin, peer);
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
-          bulk_copy_to_peer(mapa_shared(buf + (uint32_t)t * C::BFORM_ATOM + (uint32_t)(128 * c) * 128u, peer),
-                            s0 + C::XS_OFF + (uint32_t)t * (128u * 128u), 128u * 128u, bar_peer);
+          for (int t = 0; t < 2; ++t)
+            bulk_copy_to_peer(mapa_shared(buf + (uint32_t)t * C::BFORM_ATOM + (uint32_t)(128 * c) * 128u, peer),
+                              s0 + C::XS_OFF + (uint32_t)t * (128u * 128u), 128u * 128u, bar_peer);
+        }
       }
     }
   };

@@ -231,9 +231,14 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
-// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.
+// Arrive on an mbarrier given by its shared::cluster address (default semantics: release at CTA
+// scope).  Used by the threads of both CTAs of a pair to tell the issuing CTA that their operands
+// for the next pair MMA are in place: each thread has written its own CTA's shared memory and
+// fenced it for the async proxy (and waited for its TMEM stores) before arriving, the same
+// handshake the CUTLASS 2-SM transform pipelines use.  A release at cluster scope was measured
+// to delay every such handshake by about 0.4 us.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -260,6 +265,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
       return false;
     }
   }
+}
+// Barrier among `nthreads` threads (whole warps) of the CTA on hardware barrier `id` (0 is the
+// one __syncthreads uses).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 // Every thread of every CTA of the cluster meets here (release / acquire at cluster scope).
 __device__ __forceinline__ void cluster_sync_all() {
