@@ -37,6 +37,7 @@ struct Epilogue {
   int d1_dtype = F32;
   float alpha1 = 1.f, beta1 = 0.f;
   int diag1 = 0;
+  int red1 = 0;  // f32 d1 only: added into d1 (red.global.add) instead of stored; every split adds into the same tile
   float* d2 = nullptr;
   long ld2 = 0, zrow2 = 0, zcol2 = 0;
   float alpha2 = 1.f, beta2 = 0.f;
@@ -123,7 +124,16 @@ __device__ __forceinline__ void epilogue32c(const Epilogue& e, int z, int split,
       o[j] = v;
     }
     const long off = ((long)z * e.zrow1 + m) * e.ld1 + (long)z * e.zcol1 + n + (long)split * e.split_stride1;
-    store32(e.d1, off, e.d1_dtype, o);
+    if (e.red1) {
+      float* p = reinterpret_cast<float*>(e.d1) + off;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p + 4 * q), "f"(o[4 * q]), "f"(o[4 * q + 1]),
+                     "f"(o[4 * q + 2]), "f"(o[4 * q + 3])
+                     : "memory");
+    } else {
+      store32(e.d1, off, e.d1_dtype, o);
+    }
   }
   if (e.d2 != nullptr) {
     const long off = ((long)z * e.zrow2 + m) * e.ld2 + (long)z * e.zcol2 + n;
@@ -173,8 +183,9 @@ __device__ __forceinline__ void epilogue1(const Epilogue& e, int z, int split, i
   if (e.c != nullptr) c = load_elem(e.c, ((long)z * e.zrowc + m) * e.ldc + (long)z * e.zcolc + n, e.c_dtype);
   if (e.d1 != nullptr) {
     float v = e.alpha1 * acc + e.beta1 * c + ((e.diag1 && m == n) ? 1.f : 0.f);
-    store_elem(e.d1, ((long)z * e.zrow1 + m) * e.ld1 + (long)z * e.zcol1 + n + (long)split * e.split_stride1,
-               e.d1_dtype, v);
+    const long off = ((long)z * e.zrow1 + m) * e.ld1 + (long)z * e.zcol1 + n + (long)split * e.split_stride1;
+    if (e.red1) atomicAdd(reinterpret_cast<float*>(e.d1) + off, v);
+    else store_elem(e.d1, off, e.d1_dtype, v);
   }
   if (e.d2 != nullptr) {
     const long off = ((long)z * e.zrow2 + m) * e.ld2 + (long)z * e.zcol2 + n;

@@ -186,6 +186,7 @@ poetx_status check_gemm(const GemmDesc& g, int dt) {
       if (!aligned16(op->base) || op->ld % 8 || op->zcol % 8) return POETX_ERR_ALIGNMENT;
     const Epilogue& e = g.epi;
     if (e.d1 && (!aligned16(e.d1) || e.ld1 % 8 || e.zcol1 % 8 || e.split_stride1 % 8)) return POETX_ERR_ALIGNMENT;
+    if (e.red1 && (!e.d1 || e.d1_dtype != F32)) return POETX_ERR_INVALID_ARG;
     if (e.d2 && (!aligned16(e.d2) || e.ld2 % 4 || e.zcol2 % 4)) return POETX_ERR_ALIGNMENT;
     if (e.c && (!aligned16(e.c) || e.ldc % 8 || e.zcolc % 8)) return POETX_ERR_ALIGNMENT;
   }
@@ -259,7 +260,7 @@ poetx_status launch_tc(const GemmDesc& g, cudaStream_t st, int cls) {
   // every batch's columns, boxes of 64 columns x 32 rows.
   const Epilogue& e = g.epi;
   a.tma_store = e.d1 != nullptr && e.d1_dtype == BF16 && e.alpha1 == 1.f && e.beta1 == 0.f && !e.c && !e.diag1 &&
-                !e.d2 && e.split_stride1 == 0 && e.zrow1 == 0 && g.splits == 1 && e.zcol1 % 8 == 0;
+                !e.d2 && !e.red1 && e.split_stride1 == 0 && e.zrow1 == 0 && g.splits == 1 && e.zcol1 % 8 == 0;
   if (a.tma_store) {
     if (!make_tmap(&td, view(e.d1, g.M, (long)(g.batch - 1) * e.zcol1 + g.N, e.ld1), 64, 32)) return POETX_ERR_CUDA;
   } else {
@@ -569,14 +570,18 @@ int grad_splits(int dt, long n, int nb, int b) {
   return (int)std::max<long>(1, std::min<long>(s, 64));
 }
 
+// reduce: every split adds its partial into the one [nb*b, b] tile set at `part` (zeroed by the
+// caller) instead of writing its own.
 poetx_status block_grads(int dt, long n, int d, int b, const void* lhs, const void* rhs, float* part, int splits,
-                         cudaStream_t st, bool few_ctas = false, bool rhs_static = false) {
+                         cudaStream_t st, bool few_ctas = false, bool rhs_static = false, bool reduce = false) {
   GemmDesc g;
   g.b_static = rhs_static;
   g.M = b; g.N = b; g.K = (int)n; g.batch = d / b; g.splits = splits;
   g.A = view(lhs, n, d, d, 0, b); g.a_mn = true;
   g.B = view(rhs, n, d, d, 0, b); g.b_mn = true;
-  g.epi.d1 = part; g.epi.d1_dtype = F32; g.epi.ld1 = b; g.epi.zrow1 = b; g.epi.split_stride1 = (long)d * b;
+  g.epi.d1 = part; g.epi.d1_dtype = F32; g.epi.ld1 = b; g.epi.zrow1 = b;
+  g.epi.split_stride1 = reduce ? 0 : (long)d * b;
+  g.epi.red1 = reduce ? 1 : 0;
   // few_ctas: the widest tile and the deep ring whatever the CTA count, for a launch that runs
   // beside a GEMM on the SMs that one leaves free.
   if (few_ctas && dt == BF16 && b % 256 == 0) {
@@ -1367,6 +1372,10 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   POETX_TRY(bd_backward(dt, n, dout, b, ws + w.dYp, Q_R, ws + w.dZ, stream, true));  // Q_R: from the CNP forward
   POETX_TRY(stream_edge(stream, side, ss->ev[0]));
   SideJoin join{stream, side, ss->ev[3], true};
+  // With the on-chip adjoint, G_P's K splits add into one zeroed tile set (the adjoint then reads
+  // one partial per block instead of one per split); it is zeroed here, beside the W0' GEMM.
+  const bool red_P = cnp_fused_ok(b, dt) && w.sP > 1;
+  if (red_P && cudaMemsetAsync(ws + w.GpP, 0, (size_t)nbi * b * b * 4, side) != cudaSuccess) return POETX_ERR_CUDA;
   POETX_TRY(block_grads(dt, n, dout, b, ws + w.dYp, Z, reinterpret_cast<float*>(ws + w.GpR), w.sR, side, w.sR == 1,
                         true));  // Z: saved by the forward or recomputed several launches before
   if (cudaEventRecord(ss->ev[1], side) != cudaSuccess) return POETX_ERR_CUDA;  // G_R partials done
@@ -1387,14 +1396,15 @@ static poetx_status backward_impl(const poetx_desc* desc, int n_tokens, const vo
   // runs in the adjoint's launch on the SMs its pairs leave free (b = 256), else on the side
   // stream from the moment dU exists.
   if (cudaEventRecord(ss->ev[2], stream) != cudaSuccess) return POETX_ERR_CUDA;  // dU done
+  if (red_P && cudaStreamWaitEvent(stream, ss->ev[1], 0) != cudaSuccess) return POETX_ERR_CUDA;  // zeroed, G_R done
   POETX_TRY(block_grads(dt, n, din, b, ws + w.dV, U, reinterpret_cast<float*>(ws + w.GpP), w.sP, stream, false,
-                        true));  // U: saved by the forward or recomputed several launches before
-  if (cudaStreamWaitEvent(stream, ss->ev[1], 0) != cudaSuccess) return POETX_ERR_CUDA;
+                        true, red_P));  // U: saved by the forward or recomputed several launches before
+  if (!red_P && cudaStreamWaitEvent(stream, ss->ev[1], 0) != cudaSuccess) return POETX_ERR_CUDA;
   CnpSide sides[2];
   sides[0].nb = nbo; sides[0].theta = theta_R; sides[0].part = reinterpret_cast<const float*>(ws + w.GpR);
   sides[0].splits = w.sR; sides[0].grad = grad_theta_R;
   sides[1].nb = nbi; sides[1].theta = theta_P; sides[1].part = reinterpret_cast<const float*>(ws + w.GpP);
-  sides[1].splits = w.sP; sides[1].grad = grad_theta_P;
+  sides[1].splits = red_P ? 1 : w.sP; sides[1].grad = grad_theta_P;
   poetx_status cst = POETX_OK;
   if (cnp_fused_ok(b, dt) &&
       cnp_with_permute<true>(b, desc->k, sides, 2, ws + w.dU, din, dX, din, n, din, perm_R, true, stream, &cst))
