@@ -211,6 +211,24 @@ def test_cnp_forward_call_equals_the_two_calls(dtype, b, mode):
         assert torch.equal(L.saved, saved_ref)
 
 
+@pytest.mark.parametrize("mode", ["fast", "mem"])
+def test_repeated_steps_are_bit_identical(mode):
+    # 600 tokens, two 256-blocks per side: theta_P's block gradients run as two K splits that add
+    # into one tile set zeroed in every backward call, so a second step on the same inputs must
+    # reproduce the first bit for bit (two addends onto zero: the order cannot change the sum).
+    s = I.small_shape(512, 512, 256, 3, 600, "bf16", theta_std=0.005, w_std=0.02)
+    inp = I.make_layer(s, 4242)
+    g1, L = gpu_layer(inp, mode=mode)
+    X, dY = L.to_dev(inp.X), L.to_dev(inp.dY)
+    L.step(X, dY)
+    torch.cuda.synchronize()
+    g2 = dict(Q_R=to_np(L.Q_R), Q_P=to_np(L.Q_P), Y=to_np(L.Y), dX=to_np(L.dX), g_R=to_np(L.g_R), g_P=to_np(L.g_P))
+    device_clean()
+    for k in KEYS:
+        assert np.array_equal(g1[k], g2[k]), k
+    _check_all(g2, oracle_layer(inp), TOL["bf16"])
+
+
 def test_fast_and_mem_agree():
     s = I.small_shape(512, 512, 128, 3, 200, "bf16", theta_std=0.005, w_std=0.02)
     inp = I.make_layer(s, 77)
