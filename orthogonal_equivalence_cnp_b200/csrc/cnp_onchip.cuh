@@ -36,8 +36,8 @@
 // same number of packed entries) and writes the packed rows coalesced.
 //
 // Synchronisation.  One thread of the (even) CTA issues every product once all epilogue warps
-// of the pair have arrived on its `ready` barrier (release at cluster scope after their shared
-// memory writes, TMEM stores and proxy fences); the product's completion is committed to the
+// of the pair have arrived on its `ready` barrier (each after its shared memory writes, TMEM
+// stores and proxy fences; the odd CTA's arrivals are remote); the product's completion is committed to the
 // `mma` barrier of both CTAs.  Every wait is bounded (a timeout records the device error word,
 // and the kernel skips the rest of its work but still runs every cluster barrier and frees TMEM).
 #pragma once
